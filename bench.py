@@ -1,0 +1,354 @@
+"""Benchmark of the B200 Gated DeltaNet mixer.
+
+Default workload (N=1): the decode batch — 64 rows x 128 successive single-token
+steps with the 27B model's GDN shapes, each row with its own f32 state
+[48,128,128] ~ N(0,0.05) and conv history ~ N(0,1).  One bench step = that
+whole pass (128 decode launches, 8192 row-tokens).  Metric: row-tokens/s.
+A second measured object, "prefill", times the chunked prefill of one row of
+8192 tokens (zero initial state) in tokens/s against the tensor roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N>1) every rank runs its own replica of the workload (the rows
+are independent: weak scaling, no collective on the data path); the time is
+the max over ranks.  ``--impl reference`` times the float64 CPU oracle on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_mixer_gdn_b200 import synth  # noqa: E402
+
+ROWS, DECODE_STEPS = 64, 128
+STATE_BYTES_PER_ROW_TOKEN = 2 * 48 * 128 * 128 * 4          # f32 state read + write
+PREFILL_T = 8192
+PREFILL_FLOP_PER_TOKEN = 7602176                               # chunk-64 contraction FLOPs, 48 heads
+PREFILL_BYTES_PER_TOKEN = 10240 * 2 + 6144 * 2 + 2 * 48 * 2 + 6144 * 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        finally:
+            os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- oracle timing
+
+def oracle_decode_sample(case, steps: int, rows: int):
+    """Time the float64 oracle on `rows` rows x `steps` decode tokens (all 48 heads)."""
+    import numpy as np
+    import oracle
+    f = synth.to_f64
+    w = case["weights"]
+    st = f(case["init_state"][:rows])
+    cv = f(case["init_conv"][:rows])
+    cu = np.arange(rows + 1)
+    t0 = time.perf_counter()
+    for s in range(steps):
+        r = oracle.mixer(case["dims"], cu, f(case["qkv"][s, :rows]), f(case["z"][s, :rows]), f(case["a"][s, :rows]),
+                         f(case["b"][s, :rows]), f(w["conv_w"]), f(w["A_log"]), f(w["dt_bias"]), f(w["norm_w"]),
+                         st, cv)
+        st, cv = r["state"], r["conv"]
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_line(case, budget_s: float = 15.0):
+    import oracle
+    oracle.build()
+    rows = 16
+    dt = oracle_decode_sample(case, 1, rows)  # also warms up
+    steps = max(1, min(DECODE_STEPS, int(budget_s / max(dt, 1e-3))))
+    dt = oracle_decode_sample(case, steps, rows)
+    return {"value": rows * steps / dt, "unit": "row-tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{rows} rows x {steps} decode tokens of the 64x128 decode batch (all 48 heads), f64"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    case = synth.config(1)
+    import oracle
+    oracle.build()
+    rows, steps = 16, 4
+    for _ in range(args.warmup):
+        oracle_decode_sample(case, steps, rows)
+    t = 0.0
+    for _ in range(args.steps):
+        t += oracle_decode_sample(case, steps, rows)
+    value = rows * steps * args.steps / t
+    line = {"impl": "reference", "metric": "GDN decode row-tokens/s (64-row batch)", "value": value,
+            "unit": "row-tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode 64 rows x 128 steps, Qwen3.8-27B GDN shapes (oracle sample)"},
+            "cpu_baseline": {"value": value, "unit": "row-tokens/s", "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": f"{rows} rows x {steps} tokens per step, all 48 heads"},
+            "e2e": {"value": value, "unit": "row-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------- our path
+
+def run_ours(args, world, rank, local):
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    case = synth.config(1)
+    w = gdn.weights_to(case["weights"], dev)
+    qkv = case["qkv"].to(dev)
+    z = case["z"].to(dev)
+    a = case["a"].to(dev)
+    b = case["b"].to(dev)
+    state0 = case["init_state"].to(dev)
+    conv0 = case["init_conv"].to(dev)
+    state = state0.clone()
+    conv = conv0.clone()
+    out = torch.empty((DECODE_STEPS, ROWS, 6144), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def one_pass():
+        for s in range(DECODE_STEPS):
+            gdn.decode(qkv[s], z[s], a[s], b[s], w, state, conv, out=out[s])
+
+    # capture the 128-launch pass in a CUDA graph (inputs already resident)
+    with torch.cuda.stream(stream):
+        one_pass()  # warm, loads the library
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        one_pass()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    t_ms = e0.elapsed_time(e1)
+    t_max = max_over_ranks(t_ms, world)
+    clocks = clk.summary()
+    launches = args.steps * DECODE_STEPS
+    per_launch_s = t_ms / 1000.0 / launches
+    value = world * ROWS * DECODE_STEPS * args.steps / (t_max / 1000.0)
+    achieved = ROWS * STATE_BYTES_PER_ROW_TOKEN / per_launch_s / 1e9
+
+    # ---- end to end through the public API with host buffers
+    pin = {k: case[k].pin_memory() for k in ("qkv", "z", "a", "b")}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in pin.items()}
+    host_out = torch.empty((DECODE_STEPS, ROWS, 6144), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e2.record(stream)
+        for _ in range(e2e_steps):
+            for k in dev_in:
+                dev_in[k].copy_(pin[k], non_blocking=True)
+            for s in range(DECODE_STEPS):
+                gdn.decode(dev_in["qkv"][s], dev_in["z"][s], dev_in["a"][s], dev_in["b"][s], w, state, conv,
+                           out=out[s])
+            host_out.copy_(out, non_blocking=True)
+        e3.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    t_e2e = max_over_ranks(e2.elapsed_time(e3), world)
+    e2e_value = world * ROWS * DECODE_STEPS * e2e_steps / (t_e2e / 1000.0)
+
+    # ---- chunked prefill, one row of 8192 tokens (secondary measurement)
+    pcase = synth.config(2)
+    pw = gdn.weights_to(pcase["weights"], dev)
+    pin_acts = {k: pcase[k].to(dev) for k in ("qkv", "z", "a", "b")}
+    pout = torch.empty((1, PREFILL_T, 6144), dtype=torch.bfloat16, device=dev)
+    pst = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
+    pcv = torch.empty((1, 3, 10240), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > L2, written between iterations
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            gdn.prefill(pin_acts["qkv"], pin_acts["z"], pin_acts["a"], pin_acts["b"], pw, out=pout,
+                        final_state=pst, final_conv=pcv)
+        torch.cuda.synchronize(dev)
+        pt = []
+        for _ in range(max(5, args.steps)):
+            flush.fill_(1)
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            gdn.prefill(pin_acts["qkv"], pin_acts["z"], pin_acts["a"], pin_acts["b"], pw, out=pout,
+                        final_state=pst, final_conv=pcv)
+            s1.record(stream)
+            s1.synchronize()
+            pt.append(s0.elapsed_time(s1) / 1000.0)
+    p_med = statistics.median(pt)
+    prefill = {"workload": "prefill B=1 T=8192, zero initial state (3 kernels: load stage, history, chunk)",
+               "value": PREFILL_T / p_med, "unit": "tokens/s", "ms": p_med * 1000.0,
+               "tflops": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12,
+               "frac_of_bf16_peak": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12 / peaks["bf16_tflops"],
+               "peak_source": peaks["source"], "l2": "flushed (256 MiB write) before each timed call"}
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": "GDN decode row-tokens/s (64-row batch, 128 steps)",
+            "value": value, "unit": "row-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "decode 64 rows x 128 steps, Qwen3.8-27B GDN layer shapes (16 qk / 48 v heads, "
+                                   "dim 128), per-row f32 state", "rows": ROWS, "tokens_per_row": DECODE_STEPS,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (402.7 MB of state per step)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "gdn_decode_kernel", "peak_source": peaks["source"],
+                         "algorithmic_bytes_per_launch": ROWS * STATE_BYTES_PER_ROW_TOKEN},
+            "e2e": {"value": e2e_value, "unit": "row-tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "clocks": clocks,
+            "gpu_launches": launches,
+            "prefill": prefill,
+        }
+    return line, case
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        line, case = run_ours(args, world, rank, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline_line(case)
+            print(json.dumps(line))
+        return 0
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,237 @@
-"""B200-native Gated DeltaNet token mixer (sm_100a CUDA kernels behind a C ABI)."""
+"""B200-native Gated DeltaNet token mixer.
+
+Python binding of the C ABI in ``include/gdn.h`` (``libgdn_b200.so``, built for
+sm_100a by ``build.py``).  This module only marshals torch CUDA tensors into
+pointers, allocates outputs and the workspace through torch, and passes the
+current CUDA stream; every step of the mixer runs in the library's kernels.
+There is no CPU path: if the library is missing the calls raise.
+
+    weights = {"conv_w": bf16 [C,4], "A_log": f32 [Vh], "dt_bias": f32 [Vh], "norm_w": f32 [128]}
+    out, state, conv = prefill(qkv, z, a, b, weights)               # qkv [B,T,C] ...
+    out, state, conv = prefill_varlen(cu_seqlens, qkv, z, a, b, weights, state0, conv0)
+    out = decode(qkv, z, a, b, weights, state, conv)                 # state, conv updated in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Dict, Optional, Sequence
+
+import torch
+
+from .synth import Dims, MODEL
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
+
+EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen_workspace_size",
+           "gdn_prefill_varlen", "gdn_decode", "gdn_last_device_error", "gdn_status_string", "gdn_version")
+
+GDN_OK = 0
+
+
+class GdnError(RuntimeError):
+    pass
+
+
+class _DimsC(ctypes.Structure):
+    _fields_ = [("num_k_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("conv_width", ctypes.c_int32)]
+
+
+class _WeightsC(ctypes.Structure):
+    _fields_ = [("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
+                ("dt_bias", ctypes.c_void_p), ("norm_w", ctypes.c_void_p)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libgdn_b200.so; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise GdnError(f"{LIB_PATH} is missing: build it first (python -m gated_deltanet_mixer_gdn_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        dp, wp = ctypes.POINTER(_DimsC), ctypes.POINTER(_WeightsC)
+        L.gdn_prefill_workspace_size.restype = sz
+        L.gdn_prefill_workspace_size.argtypes = [dp, i32, i32]
+        L.gdn_prefill_varlen_workspace_size.restype = sz
+        L.gdn_prefill_varlen_workspace_size.argtypes = [dp, i32, i32]
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_prefill.argtypes = [dp, wp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.gdn_prefill_varlen.restype = ctypes.c_int
+        L.gdn_prefill_varlen.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.gdn_decode.restype = ctypes.c_int
+        L.gdn_decode.argtypes = [dp, wp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.gdn_last_device_error.restype = ctypes.c_int
+        L.gdn_last_device_error.argtypes = []
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_version.restype = ctypes.c_int
+        _lib = L
+        return L
+
+
+def status_string(status: int) -> str:
+    return load_library().gdn_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != GDN_OK:
+        raise GdnError(f"{what} failed: {status_string(status)} ({status})")
+
+
+def _dims_c(dims: Dims) -> _DimsC:
+    return _DimsC(dims.num_k_heads, dims.num_v_heads, dims.head_dim, dims.conv_width)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, device: torch.device) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _weights_c(weights: Dict[str, torch.Tensor], device: torch.device) -> _WeightsC:
+    cw = _need(weights["conv_w"], torch.bfloat16, "conv_w", device)
+    al = _need(weights["A_log"], torch.float32, "A_log", device)
+    dt = _need(weights["dt_bias"], torch.float32, "dt_bias", device)
+    nw = _need(weights["norm_w"], torch.float32, "norm_w", device)
+    return _WeightsC(cw.data_ptr(), al.data_ptr(), dt.data_ptr(), nw.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _device_of(qkv: torch.Tensor) -> torch.device:
+    if not qkv.is_cuda:
+        raise GdnError("the mixer runs on the GPU only: pass CUDA tensors")
+    return qkv.device
+
+
+def prefill(qkv, z, a, b, weights, init_state=None, init_conv=None, *, out=None, final_state=None,
+            final_conv=None, dims: Dims = MODEL, in_place: bool = False):
+    """Dense prefill of B rows x T tokens.  qkv [B,T,C], z [B,T,Vh*D], a/b [B,T,Vh] bf16.
+    Returns (out bf16 [B,T,Vh*D], final_state f32 [B,Vh,D,D], final_conv f32 [B,W-1,C]).
+    ``in_place`` writes the final state and history over the initial ones."""
+    dev = _device_of(qkv)
+    L = load_library()
+    B, T = int(qkv.shape[0]), int(qkv.shape[1])
+    C, VD, Vh, D, Wm = dims.conv_channels, dims.value_width, dims.num_v_heads, dims.head_dim, dims.conv_width - 1
+    _need(qkv, torch.bfloat16, "qkv", dev)
+    _need(z, torch.bfloat16, "z", dev)
+    _need(a, torch.bfloat16, "a", dev)
+    _need(b, torch.bfloat16, "b", dev)
+    if tuple(qkv.shape) != (B, T, C) or tuple(z.shape) != (B, T, VD) or tuple(a.shape) != (B, T, Vh) \
+            or tuple(b.shape) != (B, T, Vh):
+        raise ValueError("prefill: shape mismatch")
+    if init_state is not None:
+        _need(init_state, torch.float32, "init_state", dev)
+    if init_conv is not None:
+        _need(init_conv, torch.float32, "init_conv", dev)
+    if out is None:
+        out = torch.empty((B, T, VD), dtype=torch.bfloat16, device=dev)
+    if final_state is None:
+        final_state = init_state if (in_place and init_state is not None) else \
+            torch.empty((B, Vh, D, D), dtype=torch.float32, device=dev)
+    if final_conv is None:
+        final_conv = init_conv if (in_place and init_conv is not None) else \
+            torch.empty((B, Wm, C), dtype=torch.float32, device=dev)
+    dc = _dims_c(dims)
+    ws_bytes = L.gdn_prefill_workspace_size(ctypes.byref(dc), B, T)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    st = L.gdn_prefill(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), B, T,
+                       _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(init_state), _ptr(init_conv),
+                       _ptr(out), _ptr(final_state), _ptr(final_conv), _ptr(ws), ws_bytes, _stream(dev))
+    _check(st, "gdn_prefill")
+    return out, final_state, final_conv
+
+
+def prefill_varlen(cu_seqlens, qkv, z, a, b, weights, init_state=None, init_conv=None, *, out=None,
+                   final_state=None, final_conv=None, dims: Dims = MODEL, cu_seqlens_dev=None,
+                   in_place: bool = False):
+    """Packed prefill of N rows.  cu_seqlens: N+1 int32 (host tensor, list, or CUDA
+    tensor).  qkv [total,C], z [total,Vh*D], a/b [total,Vh].
+    Returns (out [total,Vh*D], final_state [N,Vh,D,D], final_conv [N,W-1,C])."""
+    dev = _device_of(qkv)
+    L = load_library()
+    if isinstance(cu_seqlens, torch.Tensor):
+        cu_host = cu_seqlens.detach().to("cpu", torch.int32).contiguous()
+    else:
+        cu_host = torch.tensor(list(cu_seqlens), dtype=torch.int32)
+    N = int(cu_host.numel()) - 1
+    total = int(qkv.shape[0])
+    C, VD, Vh, D, Wm = dims.conv_channels, dims.value_width, dims.num_v_heads, dims.head_dim, dims.conv_width - 1
+    for t, dt, nm in ((qkv, torch.bfloat16, "qkv"), (z, torch.bfloat16, "z"), (a, torch.bfloat16, "a"),
+                      (b, torch.bfloat16, "b")):
+        _need(t, dt, nm, dev)
+    if tuple(qkv.shape) != (total, C) or tuple(z.shape) != (total, VD) or tuple(a.shape) != (total, Vh) \
+            or tuple(b.shape) != (total, Vh):
+        raise ValueError("prefill_varlen: shape mismatch")
+    if cu_seqlens_dev is None:
+        cu_seqlens_dev = cu_host.to(dev, non_blocking=False)
+    _need(cu_seqlens_dev, torch.int32, "cu_seqlens_dev", dev)
+    if out is None:
+        out = torch.empty((total, VD), dtype=torch.bfloat16, device=dev)
+    if final_state is None:
+        final_state = init_state if (in_place and init_state is not None) else \
+            torch.empty((N, Vh, D, D), dtype=torch.float32, device=dev)
+    if final_conv is None:
+        final_conv = init_conv if (in_place and init_conv is not None) else \
+            torch.empty((N, Wm, C), dtype=torch.float32, device=dev)
+    dc = _dims_c(dims)
+    ws_bytes = L.gdn_prefill_varlen_workspace_size(ctypes.byref(dc), N, total)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    st = L.gdn_prefill_varlen(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), N,
+                              ctypes.c_void_p(cu_host.data_ptr()), _ptr(cu_seqlens_dev), total,
+                              _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(init_state), _ptr(init_conv),
+                              _ptr(out), _ptr(final_state), _ptr(final_conv), _ptr(ws), ws_bytes, _stream(dev))
+    _check(st, "gdn_prefill_varlen")
+    return out, final_state, final_conv
+
+
+def decode(qkv, z, a, b, weights, state, conv, *, out=None, dims: Dims = MODEL):
+    """One token for each of `rows` rows.  qkv [rows,C], z [rows,Vh*D], a/b [rows,Vh] bf16;
+    state f32 [rows,Vh,D,D] and conv f32 [rows,W-1,C] are updated in place.  Returns out."""
+    dev = _device_of(qkv)
+    L = load_library()
+    rows = int(qkv.shape[0])
+    for t, dt, nm in ((qkv, torch.bfloat16, "qkv"), (z, torch.bfloat16, "z"), (a, torch.bfloat16, "a"),
+                      (b, torch.bfloat16, "b"), (state, torch.float32, "state"), (conv, torch.float32, "conv")):
+        _need(t, dt, nm, dev)
+    if out is None:
+        out = torch.empty((rows, dims.value_width), dtype=torch.bfloat16, device=dev)
+    dc = _dims_c(dims)
+    st = L.gdn_decode(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), rows,
+                      _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(state), _ptr(conv), _ptr(out), _stream(dev))
+    _check(st, "gdn_decode")
+    return out
+
+
+def last_device_error() -> int:
+    return load_library().gdn_last_device_error()
+
+
+def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tensor]:
+    return {k: v.to(device).contiguous() for k, v in weights.items()}
+
+
+__all__ = ["prefill", "prefill_varlen", "decode", "last_device_error", "status_string", "load_library",
+           "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

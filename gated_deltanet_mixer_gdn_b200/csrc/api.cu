@@ -1,0 +1,346 @@
+// C ABI of the Gated DeltaNet mixer (declared in include/gdn.h): argument
+// checks, workspace carving, TMA descriptor set-up and kernel launches.
+// This is the library's only translation unit; the kernels are included.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/gdn.h"
+#include "chunk.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prep.cuh"
+
+namespace {
+
+using namespace gdn;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const gdn_dims* d) {
+    if (d == nullptr) return GDN_ERR_INVALID_ARG;
+    if (d->num_k_heads <= 0 || d->num_v_heads <= 0) return GDN_ERR_INVALID_ARG;
+    if (d->head_dim != 128 || d->conv_width != 4) return GDN_ERR_UNSUPPORTED;
+    if (d->num_v_heads % d->num_k_heads != 0) return GDN_ERR_UNSUPPORTED;
+    if (d->num_v_heads / d->num_k_heads > 8) return GDN_ERR_UNSUPPORTED;
+    if (d->num_v_heads > 1024 || d->num_k_heads > 1024) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+int check_weights(const gdn_weights* w) {
+    if (w == nullptr || w->conv_w == nullptr || w->A_log == nullptr || w->dt_bias == nullptr || w->norm_w == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(w->conv_w) || !aligned16(w->norm_w)) return GDN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(w->A_log) & 3u) || (reinterpret_cast<uintptr_t>(w->dt_bias) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return GDN_ERR_CUDA;
+    return major == 10 ? GDN_OK : GDN_ERR_UNSUPPORTED;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major map over [rows][cols] 16-bit elements, box {box_cols, box_rows}.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows, uint32_t box_cols,
+              uint32_t box_rows, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct Workspace {
+    size_t off_q, off_k, off_v, off_g, off_b, bytes;
+};
+
+Workspace plan_workspace(const gdn_dims* d, int64_t total) {
+    Workspace w{};
+    const size_t qk = (size_t)total * d->num_k_heads * 128 * 2;
+    const size_t vv = (size_t)total * d->num_v_heads * 128 * 2;
+    const size_t gb = (size_t)total * d->num_v_heads * 4;
+    w.off_q = 0;
+    w.off_k = align_up(qk);
+    w.off_v = w.off_k + align_up(qk);
+    w.off_g = w.off_v + align_up(vv);
+    w.off_b = w.off_g + align_up(gb);
+    w.bytes = w.off_b + align_up(gb);
+    return w;
+}
+
+int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32_t* cu_dev, int32_t uniform_T,
+                 int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                 const float* init_state, const float* init_conv, uint16_t* out, float* final_state,
+                 float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    const int Kh = d->num_k_heads, Vh = d->num_v_heads;
+    const int C = (2 * Kh + Vh) * 128;
+    const size_t state_bytes = (size_t)N * Vh * 128 * 128 * 4;
+    const size_t conv_bytes = (size_t)N * 3 * C * 4;
+    SeqIndex seq{cu_dev, uniform_T, N};
+
+    if (N == 0) return GDN_OK;
+    if (total == 0) {
+        // Nothing to run: states and histories pass through.
+        if (final_state != nullptr && final_state != init_state) {
+            cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
+                                       : cudaMemsetAsync(final_state, 0, state_bytes, stream);
+            if (e != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        if (final_conv != nullptr && final_conv != init_conv) {
+            cudaError_t e = init_conv ? cudaMemcpyAsync(final_conv, init_conv, conv_bytes, cudaMemcpyDeviceToDevice, stream)
+                                      : cudaMemsetAsync(final_conv, 0, conv_bytes, stream);
+            if (e != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        return GDN_OK;
+    }
+
+    const Workspace ws = plan_workspace(d, total);
+    if (workspace == nullptr || workspace_bytes < ws.bytes) return GDN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    __half* Qs = reinterpret_cast<__half*>(wsb + ws.off_q);
+    __half* Ks = reinterpret_cast<__half*>(wsb + ws.off_k);
+    __half* Vs = reinterpret_cast<__half*>(wsb + ws.off_v);
+    float* Gs = reinterpret_cast<float*>(wsb + ws.off_g);
+    float* Bs = reinterpret_cast<float*>(wsb + ws.off_b);
+
+    // 1. load stage: conv + silu, L2 norms, gates
+    {
+        PrepParams pp{};
+        pp.Kh = Kh;
+        pp.Vh = Vh;
+        pp.C = C;
+        pp.total = total;
+        pp.seq = seq;
+        pp.qkv = qkv;
+        pp.a = a;
+        pp.b = b;
+        pp.conv_w = w->conv_w;
+        pp.A_log = w->A_log;
+        pp.dt_bias = w->dt_bias;
+        pp.init_conv = init_conv;
+        pp.Qs = Qs;
+        pp.Ks = Ks;
+        pp.Vs = Vs;
+        pp.Gs = Gs;
+        pp.Bs = Bs;
+        dim3 grid((total + kPrepTokens - 1) / kPrepTokens, (2 * Kh + Vh + 15) / 16);
+        gdn_prep_kernel<<<grid, 256, 0, stream>>>(pp);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    // 2. final conv history (after the load stage has read the initial one)
+    if (final_conv != nullptr) {
+        ConvOutParams cp{};
+        cp.C = C;
+        cp.N = N;
+        cp.seq = seq;
+        cp.qkv = qkv;
+        cp.init_conv = init_conv;
+        cp.final_conv = final_conv;
+        dim3 grid((C + 255) / 256, N);
+        gdn_conv_out_kernel<<<grid, 256, 0, stream>>>(cp);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    // 3. chunked recurrence on tensor cores, gated RMSNorm epilogue
+    {
+        CUtensorMap mK, mQ, mV, mZ;
+        if (!make_map(&mK, Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mQ, Qs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mV, Vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Vh * 128, total, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return GDN_ERR_CUDA;
+        ChunkParams cp{};
+        cp.Kh = Kh;
+        cp.Vh = Vh;
+        cp.total = total;
+        cp.seq = seq;
+        cp.Gs = Gs;
+        cp.Bs = Bs;
+        cp.init_state = init_state;
+        cp.final_state = final_state;
+        cp.norm_w = w->norm_w;
+        cp.out = out;
+        static std::once_flag attr_once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(attr_once, [] {
+            attr_err = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)chunk::SMEM_BYTES);
+        });
+        if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
+        dim3 grid(Vh, N);
+        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mK, mQ, mV, mZ, cp);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
+}
+
+int check_io(int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+             const uint16_t* out, const float* init_state, const float* init_conv, const float* final_state,
+             const float* final_conv) {
+    if (total > 0) {
+        if (!qkv || !z || !a || !b || !out) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(qkv) || !aligned16(z) || !aligned16(out)) return GDN_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(a) & 1u) || (reinterpret_cast<uintptr_t>(b) & 1u)) return GDN_ERR_INVALID_ARG;
+    }
+    const void* fs[4] = {init_state, init_conv, final_state, final_conv};
+    for (const void* p : fs)
+        if (p != nullptr && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
+    if (check_dims(dims) != GDN_OK || B < 0 || T < 0) return 0;
+    const int64_t total = (int64_t)B * T;
+    if (total > INT32_MAX) return 0;
+    return plan_workspace(dims, total).bytes;
+}
+
+size_t gdn_prefill_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T) {
+    if (check_dims(dims) != GDN_OK || N < 0 || total_T < 0) return 0;
+    return plan_workspace(dims, total_T).bytes;
+}
+
+int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, const uint16_t* qkv,
+                const uint16_t* z, const uint16_t* a, const uint16_t* b, const float* init_state,
+                const float* init_conv, uint16_t* out, float* final_state, float* final_conv, void* workspace,
+                size_t workspace_bytes, void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (B < 0 || T < 0 || B > 65535) return GDN_ERR_INVALID_ARG;
+    const int64_t total = (int64_t)B * T;
+    if (total > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if ((st = check_io((int32_t)total, qkv, z, a, b, out, init_state, init_conv, final_state, final_conv)) != GDN_OK)
+        return st;
+    if ((st = check_device()) != GDN_OK) return st;
+    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, qkv, z, a, b, init_state, init_conv, out, final_state,
+                        final_conv, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_host,
+                       const int32_t* cu_dev, int32_t total_T, const uint16_t* qkv, const uint16_t* z,
+                       const uint16_t* a, const uint16_t* b, const float* init_state, const float* init_conv,
+                       uint16_t* out, float* final_state, float* final_conv, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (N < 0 || N > 65535 || total_T < 0) return GDN_ERR_INVALID_ARG;
+    if (cu_host == nullptr || (N > 0 && cu_dev == nullptr)) return GDN_ERR_INVALID_ARG;
+    if (cu_host[0] != 0 || cu_host[N] != total_T) return GDN_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < N; ++i)
+        if (cu_host[i + 1] < cu_host[i]) return GDN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_dev) & 3u) != 0) return GDN_ERR_INVALID_ARG;
+    if ((st = check_io(total_T, qkv, z, a, b, out, init_state, init_conv, final_state, final_conv)) != GDN_OK)
+        return st;
+    if ((st = check_device()) != GDN_OK) return st;
+    return prefill_impl(dims, w, N, cu_dev, 0, total_T, qkv, z, a, b, init_state, init_conv, out, final_state,
+                        final_conv, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const uint16_t* qkv, const uint16_t* z,
+               const uint16_t* a, const uint16_t* b, float* state, float* conv, uint16_t* out, void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (rows < 0 || rows > 65535) return GDN_ERR_INVALID_ARG;
+    if (rows == 0) return GDN_OK;
+    if (!state || !conv || !aligned16(state) || !aligned16(conv)) return GDN_ERR_INVALID_ARG;
+    if ((st = check_io(rows, qkv, z, a, b, out, nullptr, nullptr, nullptr, nullptr)) != GDN_OK) return st;
+    if ((st = check_device()) != GDN_OK) return st;
+    DecodeParams p{};
+    p.Kh = dims->num_k_heads;
+    p.Vh = dims->num_v_heads;
+    p.C = (2 * p.Kh + p.Vh) * 128;
+    p.rows = rows;
+    p.qkv = qkv;
+    p.z = z;
+    p.a = a;
+    p.b = b;
+    p.conv_w = w->conv_w;
+    p.A_log = w->A_log;
+    p.dt_bias = w->dt_bias;
+    p.norm_w = w->norm_w;
+    p.state = state;
+    p.conv = conv;
+    p.out = out;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.Vh, rows);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.Vh / p.Kh;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p));
+}
+
+int gdn_last_device_error(void) {
+    int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, gdn::g_device_error, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(gdn::g_device_error, &zero, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    return v;
+}
+
+const char* gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported dimensions or device";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+        case GDN_ERR_TIMEOUT: return "bounded device wait expired";
+        default: return "unknown status";
+    }
+}
+
+int gdn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,524 @@
+// Chunked prefill of the gated delta rule on 5th-generation tensor cores.
+//
+// The recurrence (Qwen3.8 27B model card, "Gated DeltaNet" bullet), per value
+// head with state S [128 v][128 k]:
+//     S_t = exp(g_t) S_{t-1} + u_t k_t^T,   u_t = beta_t (v_t - exp(g_t) S_{t-1} k_t),
+//     o_t = S_t q_t.
+// In chunks of 64 tokens with G = inclusive cumsum of g inside the chunk,
+// A_ij = beta_i exp(G_i - G_j) (k_i . k_j) for j < i and T = (I + A)^-1:
+//     U   = T diag(beta) V - T diag(beta e^G) K S0^T   ( = U~ - W S0^T )
+//     O   = diag(e^G) Q S0^T + (tril_incl(Q K^T) * E) U,   E_ij = exp(G_i - G_j)
+//     S_C = e^{G_C} S0 + U^T diag(e^{G_C - G}) K.
+// (Obtained by unrolling the recurrence inside a chunk; every ratio of decays
+// is formed as exp of a difference over j <= i, so nothing overflows.)
+//
+// One CTA owns one (row, value head) and walks its chunks in order.  All seven
+// contractions run as tcgen05.mma (f16 operands in 128B-swizzled shared
+// memory, f32 accumulators in TMEM), arranged so that M = 128 every time:
+//   MMA1  KQ   [128 x 64]  = [K;Q] K^T                (A K-major, B K-major)
+//   MMA2  U~^T [128v x 64] = V^T (T diag beta)^T       (A = V tile read MN-major)
+//   MMA3  W^T  [128k x 64] = K^T (T diag(beta e^G))^T  (A = K tile read MN-major)
+//   MMA4  U^T  += -S0 W^T                             (negated A, B = W^T MN-major)
+//   MMA5  Oi^T [128v x 64] = S0 Q^T                    (e^G applied in the epilogue)
+//   MMA6  dS   [128v x128k]= (U^T diag e^{G_C-G}) K    (B = K tile read MN-major)
+//   MMA7  Oa^T [128v x 64] = U^T (tril(QK^T)*E)^T
+// The unit lower-triangular inverse T is formed on the CUDA cores (blocked
+// 16 x 16 forward substitution in f32).  The state lives in registers in
+// f32 (thread = one v row, one half of k) and is re-staged as f16 in shared
+// memory for the next chunk.  The gated RMSNorm is fused into the epilogue
+// and the 64 x 128 bf16 output tile leaves with coalesced 16-byte stores.
+//
+// Inputs come from the load-stage kernel (conv, L2 norm, gates) as f16 tiles
+// fetched with TMA: K and Q of the q/k head (double-buffered), V of the
+// value head, and the z tile for the gate of the norm.
+#pragma once
+
+#include "common.cuh"
+#include "prep.cuh"
+
+namespace gdn {
+
+struct ChunkParams {
+    int Kh, Vh, total;
+    SeqIndex seq;
+    const float* Gs;          // f32 [Vh][total] log-decay
+    const float* Bs;          // f32 [Vh][total] write rate
+    const float* init_state;  // f32 [N][Vh][128][128] or nullptr
+    float* final_state;       // f32 [N][Vh][128][128] or nullptr (may alias init_state)
+    const float* norm_w;      // f32 [128]
+    uint16_t* out;            // bf16 [total][Vh*128]
+};
+
+namespace chunk {
+constexpr int C = 64;              // tokens per chunk
+constexpr int kThreads = 256;
+constexpr int LDA = 68;            // f32 row stride of the A / T matrix (conflict-free float4 rows)
+// shared-memory map (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_KQ0 = 0;        // [K rows 0-63 | Q rows 64-127] x k 0-63, then x k 64-127
+constexpr uint32_t OFF_KQ1 = 32768;    // second buffer
+constexpr uint32_t OFF_V = 65536;      // V [64 t][64 v] x 2 blocks
+constexpr uint32_t OFF_Z = 81920;      // z bf16 [64][128], plain row-major; reused for y
+constexpr uint32_t OFF_WT = 98304;     // W^T f16 [128 k][64 t]
+constexpr uint32_t OFF_UT = 114688;    // U^T f16 [128 v][64 t]; T-solve scratch before that
+constexpr uint32_t OFF_UTS = 131072;   // U^T diag(e^{G_C-G}) f16
+constexpr uint32_t OFF_S = 147456;     // S0 f16 [128 v][64 k] x 2 blocks
+constexpr uint32_t OFF_T1 = 180224;    // T diag(beta) f16 [64][64]
+constexpr uint32_t OFF_T2 = 188416;    // T diag(beta e^G) f16 [64][64]
+constexpr uint32_t OFF_M = 196608;     // tril(Q K^T) * E f16 [64][64]
+constexpr uint32_t OFF_A = 204800;     // A, then T, f32 [64][LDA]
+constexpr uint32_t OFF_MISC = OFF_A + 64 * LDA * 4;  // 222208
+constexpr uint32_t MISC_BYTES = 2048;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+// TMEM columns (f32, 128 lanes)
+constexpr uint32_t T_KQ = 0, T_UT = 64, T_WT = 128, T_OI = 192, T_OA = 256, T_S = 320;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t KQV_BYTES = 6 * 8192;
+constexpr uint32_t Z_BYTES = 64 * 128 * 2;
+constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, false, false, false);
+constexpr uint32_t ID_AMN = idesc_f16_f32(128, 64, true, false, false);
+constexpr uint32_t ID_NEG_BMN = idesc_f16_f32(128, 64, false, true, true);
+constexpr uint32_t ID_DS = idesc_f16_f32(128, 128, false, true, false);
+}  // namespace chunk
+
+// (I + A)^-1 of a unit lower-triangular 64 x 64 system, in place in sA (row
+// stride LDA): 16 x 16 diagonal blocks by forward substitution, then block
+// rows 1..3 as T_i,<i = -T_ii (sum_m A_im T_m,<i).  Uses sP (16 x 48 f32).
+__device__ __forceinline__ void chunk_tsolve(float* sA, float* sP, int tid) {
+    using namespace chunk;
+    float x[16];
+    const int b = tid >> 4, c = tid & 15;
+    if (tid < 64) {
+        const float* Ab = sA + (16 * b) * LDA + 16 * b;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float s = 0.f;
+#pragma unroll
+            for (int m = 0; m < r; ++m) s = fmaf(Ab[r * LDA + m], x[m], s);
+            x[r] = (r == c) ? 1.f : ((r < c) ? 0.f : -s);
+        }
+    }
+    __syncthreads();
+    if (tid < 64) {
+        float* Ab = sA + (16 * b) * LDA + 16 * b;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Ab[r * LDA + c] = x[r];
+    }
+    __syncthreads();
+    for (int i = 1; i < 4; ++i) {
+        const int ncol = 16 * i;
+        const int nout = 16 * ncol;
+        for (int o = tid; o < nout; o += kThreads) {
+            const int r = o / ncol, cc = o % ncol;
+            const float* Ar = sA + (16 * i + r) * LDA;
+            float s = 0.f;
+            for (int m = cc; m < ncol; ++m) s = fmaf(Ar[m], sA[m * LDA + cc], s);
+            sP[r * 48 + cc] = s;
+        }
+        __syncthreads();
+        for (int o = tid; o < nout; o += kThreads) {
+            const int r = o / ncol, cc = o % ncol;
+            const float* Tr = sA + (16 * i + r) * LDA + 16 * i;
+            float s = 0.f;
+            for (int m = 0; m <= r; ++m) s = fmaf(Tr[m], sP[m * 48 + cc], s);
+            sA[(16 * i + r) * LDA + cc] = -s;
+        }
+        __syncthreads();
+    }
+}
+
+// Lane l of the warp ends with sum over the 32 lanes of v[l] (31 shuffles).
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+            const float send = upper ? v[i] : v[i + off];
+            const float keep = upper ? v[i + off] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return v[0];
+}
+
+__device__ __forceinline__ void store_row_f16_sw128(uint8_t* tile, uint32_t row, uint32_t chunk0, const float* vals,
+                                                    float scale_all) {
+    // 32 values -> 4 chunks of 8 f16 starting at 16-byte chunk index chunk0
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 pk;
+        pk.x = pack_half2(vals[8 * j + 0] * scale_all, vals[8 * j + 1] * scale_all);
+        pk.y = pack_half2(vals[8 * j + 2] * scale_all, vals[8 * j + 3] * scale_all);
+        pk.z = pack_half2(vals[8 * j + 4] * scale_all, vals[8 * j + 5] * scale_all);
+        pk.w = pack_half2(vals[8 * j + 6] * scale_all, vals[8 * j + 7] * scale_all);
+        *reinterpret_cast<uint4*>(tile + sw128_chunk(row, chunk0 + j)) = pk;
+    }
+}
+
+#define CHUNK_WAIT(bar, parity, code)                  \
+    {                                                  \
+        const bool ok_ = mbar_wait((bar), (parity));   \
+        if (__syncthreads_or(!ok_)) {                  \
+            if (tid == 0) record_error(code);          \
+            failed = true;                             \
+            break;                                     \
+        }                                              \
+    }
+
+__global__ void __launch_bounds__(chunk::kThreads, 1)
+    gdn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZ,
+                     const ChunkParams p) {
+    using namespace chunk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+
+    const int h = blockIdx.x;
+    const int n = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3;        // TMEM lane quarter of this warp
+    const int hf = warp >> 2;       // column half handled by this warp
+    const int row = 32 * q4 + lane; // TMEM lane = v row / k row / token row
+    const int kap = h / (p.Vh / p.Kh);
+
+    uint64_t* bar_kqv = reinterpret_cast<uint64_t*>(smem + OFF_MISC);
+    uint64_t* bar_z = bar_kqv + 1;
+    uint64_t* bar_mma = bar_kqv + 2;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 32);
+    float* s_G = reinterpret_cast<float*>(smem + OFF_MISC + 64);     // [64]
+    float* s_eG = s_G + 64;                                            // [64]
+    float* s_beta = s_G + 128;                                         // [64]
+    float* s_red = reinterpret_cast<float*>(smem + OFF_MISC + 1024);  // [4][64]
+    float* sA = reinterpret_cast<float*>(smem + OFF_A);
+    float* sP = reinterpret_cast<float*>(smem + OFF_UT);
+
+    int start, len;
+    p.seq.bounds(n, start, len);
+    const int nchunks = (len + C - 1) / C;
+
+    if (tid == 0) {
+        mbar_init(bar_kqv, 1);
+        mbar_init(bar_z, 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmV);
+        prefetch_tensormap(&tmZ);
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    const uint32_t tlane = tbase + (static_cast<uint32_t>(32 * q4) << 16);
+
+    // Initial state: thread holds S[row][64*hf .. 64*hf+63] in f32.
+    float S[64];
+    {
+        const float* src = p.init_state ? p.init_state + (((size_t)n * p.Vh + h) * 128 + row) * 128 + 64 * hf : nullptr;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float4 v = src ? __ldg(reinterpret_cast<const float4*>(src) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[4 * j] = v.x;
+            S[4 * j + 1] = v.y;
+            S[4 * j + 2] = v.z;
+            S[4 * j + 3] = v.w;
+        }
+        uint8_t* sS = smem + OFF_S + 16384 * hf;
+        store_row_f16_sw128(sS, row, 0, S, 1.f);
+        store_row_f16_sw128(sS, row, 4, S + 32, 1.f);
+    }
+    fence_proxy_async_smem();
+    if (tid == 0 && nchunks > 0) {
+        mbar_arrive_expect_tx(bar_kqv, KQV_BYTES);
+        tma_load_2d(smem + OFF_KQ0, &tmK, kap * 128, start, bar_kqv);
+        tma_load_2d(smem + OFF_KQ0 + 16384, &tmK, kap * 128 + 64, start, bar_kqv);
+        tma_load_2d(smem + OFF_KQ0 + 8192, &tmQ, kap * 128, start, bar_kqv);
+        tma_load_2d(smem + OFF_KQ0 + 24576, &tmQ, kap * 128 + 64, start, bar_kqv);
+        tma_load_2d(smem + OFF_V, &tmV, h * 128, start, bar_kqv);
+        tma_load_2d(smem + OFF_V + 8192, &tmV, h * 128 + 64, start, bar_kqv);
+        mbar_arrive_expect_tx(bar_z, Z_BYTES);
+        tma_load_2d(smem + OFF_Z, &tmZ, h * 128, start, bar_z);
+    }
+    __syncthreads();
+
+    const float wn = 1.0f + __ldg(p.norm_w + row);  // (1 + w) of this thread's v channel
+    bool failed = false;
+    uint32_t mma_phase = 0;
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int tok0 = start + c * C;
+        const int nv = min(C, len - c * C);
+        const uint32_t kq_off = (c & 1) ? OFF_KQ1 : OFF_KQ0;
+        const uint32_t aKQ = sbase + kq_off;
+
+        // ---- gates of the chunk: G = inclusive cumsum of g, e^G, beta
+        if (tid < 64) {
+            const float g = (tid < nv) ? __ldg(p.Gs + (size_t)h * p.total + tok0 + tid) : 0.f;
+            const float bt = (tid < nv) ? __ldg(p.Bs + (size_t)h * p.total + tok0 + tid) : 0.f;
+            float x = g;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            s_G[tid] = x;
+            s_beta[tid] = bt;
+        }
+        CHUNK_WAIT(bar_kqv, c & 1, kErrTimeoutTma);  // includes a CTA barrier
+        if (tid < 64) {
+            float G = s_G[tid];
+            if (tid >= 32) G += s_G[31];
+            s_G[tid] = G;
+            s_eG[tid] = expf(G);
+        }
+        // ---- MMA1: [K;Q] K^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                mma_f16(tbase + T_KQ, sw128_desc(aKQ + off, 16, 1024), sw128_desc(aKQ + off, 16, 1024), ID_KK,
+                        s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        CHUNK_WAIT(bar_mma, mma_phase, kErrTimeoutMma);
+        mma_phase ^= 1;
+        tc_fence_after();
+        const float GC = s_G[63];
+        const float eGC = s_eG[63];
+
+        // ---- A (rows of K K^T) and M (rows of Q K^T), masked before the exp
+        {
+            float v[32];
+            tmem_ld32(tlane + T_KQ + 32 * hf, v);
+            tmem_ld_wait();
+            if (q4 < 2) {
+                const int i = row;
+                const float Gi = s_G[i], bi = s_beta[i];
+                float a[32];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = 32 * hf + jj;
+                    a[jj] = (j < i) ? bi * __expf(Gi - s_G[j]) * v[jj] : 0.f;
+                }
+                float4* dst = reinterpret_cast<float4*>(sA + i * LDA + 32 * hf);
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) dst[j4] = make_float4(a[4 * j4], a[4 * j4 + 1], a[4 * j4 + 2], a[4 * j4 + 3]);
+            } else {
+                const int i = row - 64;
+                const float Gi = s_G[i];
+                float m[32];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = 32 * hf + jj;
+                    m[jj] = (j <= i) ? v[jj] * __expf(Gi - s_G[j]) : 0.f;
+                }
+                store_row_f16_sw128(smem + OFF_M, i, 4 * hf, m, 1.f);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- T = (I + A)^-1, then T diag(beta) and T diag(beta e^G) as f16 B operands
+        chunk_tsolve(sA, sP, tid);
+        {
+            const int t = tid >> 2, part = tid & 3;
+            const float* Tr = sA + t * LDA + 16 * part;
+            float t1[16], t2[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int tp = 16 * part + e;
+                const float tv = Tr[e];
+                t1[e] = tv * s_beta[tp];
+                t2[e] = t1[e] * s_eG[tp];
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint4 p1, p2;
+                p1.x = pack_half2(t1[8 * j], t1[8 * j + 1]);
+                p1.y = pack_half2(t1[8 * j + 2], t1[8 * j + 3]);
+                p1.z = pack_half2(t1[8 * j + 4], t1[8 * j + 5]);
+                p1.w = pack_half2(t1[8 * j + 6], t1[8 * j + 7]);
+                p2.x = pack_half2(t2[8 * j], t2[8 * j + 1]);
+                p2.y = pack_half2(t2[8 * j + 2], t2[8 * j + 3]);
+                p2.z = pack_half2(t2[8 * j + 4], t2[8 * j + 5]);
+                p2.w = pack_half2(t2[8 * j + 6], t2[8 * j + 7]);
+                *reinterpret_cast<uint4*>(smem + OFF_T1 + sw128_chunk(t, 2 * part + j)) = p1;
+                *reinterpret_cast<uint4*>(smem + OFF_T2 + sw128_chunk(t, 2 * part + j)) = p2;
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- MMA2: U~^T = V^T (T diag beta)^T ; MMA3: W^T = K^T (T diag(beta e^G))^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_f16(tbase + T_UT, sw128_desc(sbase + OFF_V + s * 2048, 8192, 1024),
+                        sw128_desc(sbase + OFF_T1 + s * 32, 16, 1024), ID_AMN, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_f16(tbase + T_WT, sw128_desc(aKQ + s * 2048, 16384, 1024),
+                        sw128_desc(sbase + OFF_T2 + s * 32, 16, 1024), ID_AMN, s > 0);
+            mma_commit(bar_mma);
+        }
+        CHUNK_WAIT(bar_mma, mma_phase, kErrTimeoutMma);
+        mma_phase ^= 1;
+        tc_fence_after();
+
+        // V and the other K/Q buffer are free: fetch the next chunk's K, Q, V.
+        if (tid == 0 && c + 1 < nchunks) {
+            const uint32_t nxt = (c & 1) ? OFF_KQ0 : OFF_KQ1;
+            const int y = tok0 + C;
+            mbar_arrive_expect_tx(bar_kqv, KQV_BYTES);
+            tma_load_2d(smem + nxt, &tmK, kap * 128, y, bar_kqv);
+            tma_load_2d(smem + nxt + 16384, &tmK, kap * 128 + 64, y, bar_kqv);
+            tma_load_2d(smem + nxt + 8192, &tmQ, kap * 128, y, bar_kqv);
+            tma_load_2d(smem + nxt + 24576, &tmQ, kap * 128 + 64, y, bar_kqv);
+            tma_load_2d(smem + OFF_V, &tmV, h * 128, y, bar_kqv);
+            tma_load_2d(smem + OFF_V + 8192, &tmV, h * 128 + 64, y, bar_kqv);
+        }
+
+        // ---- W^T to shared memory (MN-major B operand: row k, 64 tokens)
+        {
+            float v[32];
+            tmem_ld32(tlane + T_WT + 32 * hf, v);
+            tmem_ld_wait();
+            store_row_f16_sw128(smem + OFF_WT, row, 4 * hf, v, 1.f);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- MMA4: U^T = U~^T - S0 W^T ; MMA5: Oi^T = S0 Q^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint64_t a = sw128_desc(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+                mma_f16(tbase + T_UT, a, sw128_desc(sbase + OFF_WT + s * 2048, 8192, 1024), ID_NEG_BMN, 1);
+            }
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                mma_f16(tbase + T_OI, sw128_desc(sbase + OFF_S + off, 16, 1024),
+                        sw128_desc(aKQ + 8192 + off, 16, 1024), ID_KK, s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        CHUNK_WAIT(bar_mma, mma_phase, kErrTimeoutMma);
+        mma_phase ^= 1;
+        tc_fence_after();
+
+        // ---- U^T to shared memory, plain and scaled by e^{G_C - G_t}
+        {
+            float v[32];
+            tmem_ld32(tlane + T_UT + 32 * hf, v);
+            tmem_ld_wait();
+            store_row_f16_sw128(smem + OFF_UT, row, 4 * hf, v, 1.f);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) v[jj] *= __expf(GC - s_G[32 * hf + jj]);
+            store_row_f16_sw128(smem + OFF_UTS, row, 4 * hf, v, 1.f);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- MMA6: dS = (U^T diag e^{G_C-G}) K ; MMA7: Oa^T = U^T M^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_f16(tbase + T_S, sw128_desc(sbase + OFF_UTS + s * 32, 16, 1024),
+                        sw128_desc(aKQ + s * 2048, 16384, 1024), ID_DS, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_f16(tbase + T_OA, sw128_desc(sbase + OFF_UT + s * 32, 16, 1024),
+                        sw128_desc(sbase + OFF_M + s * 32, 16, 1024), ID_KK, s > 0);
+            mma_commit(bar_mma);
+        }
+        CHUNK_WAIT(bar_mma, mma_phase, kErrTimeoutMma);
+        mma_phase ^= 1;
+        tc_fence_after();
+
+        // ---- state update in registers, re-staged as f16 for the next chunk
+        {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float d[32];
+                tmem_ld32(tlane + T_S + 64 * hf + 32 * half, d);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(eGC, S[32 * half + j], d[j]);
+            }
+            uint8_t* sS = smem + OFF_S + 16384 * hf;
+            store_row_f16_sw128(sS, row, 0, S, 1.f);
+            store_row_f16_sw128(sS, row, 4, S + 32, 1.f);
+        }
+
+        // ---- epilogue: o = e^G * Oi + Oa, gated RMSNorm over the 128 v channels
+        CHUNK_WAIT(bar_z, c & 1, kErrTimeoutTma);
+        {
+            float o[32], oa[32];
+            tmem_ld32(tlane + T_OI + 32 * hf, o);
+            tmem_ld32(tlane + T_OA + 32 * hf, oa);
+            tmem_ld_wait();
+            float sq[32];
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                o[jj] = fmaf(s_eG[32 * hf + jj], o[jj], oa[jj]);
+                sq[jj] = o[jj] * o[jj];
+            }
+            const float part = warp_transpose_sum(sq, lane);
+            s_red[q4 * 64 + 32 * hf + lane] = part;
+            __syncthreads();
+            uint16_t* zt = reinterpret_cast<uint16_t*>(smem + OFF_Z);
+#pragma unroll 8
+            for (int jj = 0; jj < 32; ++jj) {
+                const int t = 32 * hf + jj;
+                const float ms = (s_red[t] + s_red[64 + t] + s_red[128 + t] + s_red[192 + t]) * (1.0f / 128.0f);
+                const float zv = bf16_bits_to_float(zt[t * 128 + row]);
+                const float y = o[jj] * rsqrtf(ms + kEps) * wn * silu_f(zv);
+                zt[t * 128 + row] = float_to_bf16_bits(y);
+            }
+        }
+        __syncthreads();
+        for (int idx = tid; idx < C * 16; idx += kThreads) {
+            const int t = idx >> 4, cc = idx & 15;
+            if (t < nv) {
+                const uint4 v = *reinterpret_cast<const uint4*>(smem + OFF_Z + t * 256 + cc * 16);
+                *reinterpret_cast<uint4*>(p.out + (size_t)(tok0 + t) * p.Vh * 128 + h * 128 + cc * 8) = v;
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && c + 1 < nchunks) {
+            mbar_arrive_expect_tx(bar_z, Z_BYTES);
+            tma_load_2d(smem + OFF_Z, &tmZ, h * 128, tok0 + C, bar_z);
+        }
+    }
+
+    if (!failed && p.final_state != nullptr) {
+        float* dst = p.final_state + (((size_t)n * p.Vh + h) * 128 + row) * 128 + 64 * hf;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            reinterpret_cast<float4*>(dst)[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, TMEM_COLS);
+}
+
+#undef CHUNK_WAIT
+
+}  // namespace gdn

@@ -1,0 +1,205 @@
+// Load stage of the chunked prefill: per token, the depthwise causal conv
+// (width 4) + silu over all qkv channels, L2 normalisation of the q and k
+// heads (q also scaled by 1/sqrt(128)), and the two gates of every value head
+// (Qwen3.8 27B model card, "Gated DeltaNet" bullet).  Results are staged as
+// f16 operands for the tensor-core chunk kernel:
+//   Qs, Ks  f16 [total][Kh*128]   (q / (|q| sqrt(128)), k / |k|)
+//   Vs      f16 [total][Vh*128]
+//   Gs, Bs  f32 [Vh][total]       (g = log-decay, beta = write rate)
+// A second tiny kernel writes each row's final conv history.
+//
+// Mapping: a CTA of 256 threads is 16 groups of 16; a group owns one
+// 128-channel head slot, each thread 8 contiguous channels (16-byte loads and
+// stores), so the per-token L2 norm is a 16-lane shuffle reduction.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdn {
+
+struct SeqIndex {
+    const int* cu;   // device cu_seqlens [N+1], or nullptr for uniform rows
+    int uniform_T;   // row length when cu == nullptr
+    int N;
+    __device__ __forceinline__ void locate(int t, int& n, int& start, int& len) const {
+        if (cu == nullptr) {
+            n = t / uniform_T;
+            start = n * uniform_T;
+            len = uniform_T;
+            return;
+        }
+        int lo = 0, hi = N;  // find n with cu[n] <= t < cu[n+1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(cu + mid) <= t) lo = mid;
+            else hi = mid;
+        }
+        // skip empty rows that share the same start
+        n = lo;
+        start = __ldg(cu + n);
+        len = __ldg(cu + n + 1) - start;
+    }
+    __device__ __forceinline__ void bounds(int n, int& start, int& len) const {
+        if (cu == nullptr) {
+            start = n * uniform_T;
+            len = uniform_T;
+        } else {
+            start = __ldg(cu + n);
+            len = __ldg(cu + n + 1) - start;
+        }
+    }
+};
+
+struct PrepParams {
+    int Kh, Vh, C, total;
+    SeqIndex seq;
+    const uint16_t* qkv;      // bf16 [total][C]
+    const uint16_t* a;        // bf16 [total][Vh]
+    const uint16_t* b;        // bf16 [total][Vh]
+    const uint16_t* conv_w;   // bf16 [C][4]
+    const float* A_log;
+    const float* dt_bias;
+    const float* init_conv;   // f32 [N][3][C] or nullptr
+    __half* Qs;
+    __half* Ks;
+    __half* Vs;
+    float* Gs;
+    float* Bs;
+};
+
+constexpr int kPrepTokens = 16;
+
+__global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
+    const int tid = threadIdx.x;
+    const int grp = tid >> 4;
+    const int gl = tid & 15;
+    const int nheads = 2 * p.Kh + p.Vh;
+    // Slots past the last head run along (clamped, no stores) so that every
+    // lane of a warp reaches the shuffles.
+    const bool active = blockIdx.y * 16 + grp < nheads;
+    const int slot = active ? blockIdx.y * 16 + grp : nheads - 1;
+    const int ch0 = slot * kD + gl * 8;
+    const bool is_q = slot < p.Kh;
+    const bool is_k = !is_q && slot < 2 * p.Kh;
+    const bool is_v = slot >= 2 * p.Kh;
+    const int vh = slot - 2 * p.Kh;
+
+    // conv taps of the 8 channels: w[e][j] at conv_w[(ch0+e)*4 + j]
+    float w[8][4];
+    {
+        const uint4* wp = reinterpret_cast<const uint4*>(p.conv_w + (size_t)ch0 * 4);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = __ldg(wp + q);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int e = q * 2 + m / 2;  // two channels per uint4 (8 bf16 = 2 x 4 taps)
+                const int j = (m % 2) * 2;
+                w[e][j] = __uint_as_float(u[m] << 16);
+                w[e][j + 1] = __uint_as_float(u[m] & 0xffff0000u);
+            }
+        }
+    }
+    float gA = 0.f, gdt = 0.f;
+    if (is_v) {
+        gA = expf(__ldg(p.A_log + vh));
+        gdt = __ldg(p.dt_bias + vh);
+    }
+
+    const int t_begin = blockIdx.x * kPrepTokens;
+    for (int tt = 0; tt < kPrepTokens; ++tt) {
+        const int t = t_begin + tt;
+        if (t >= p.total) break;
+        int n, start, len;
+        p.seq.locate(t, n, start, len);
+        const int s = t - start;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int xi = s + j;  // index into [history (3 rows); tokens of the row]
+            float x[8];
+            if (xi >= 3) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)(t + j - 3) * p.C + ch0));
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    x[2 * m] = __uint_as_float(u[m] << 16);
+                    x[2 * m + 1] = __uint_as_float(u[m] & 0xffff0000u);
+                }
+            } else if (p.init_conv != nullptr) {
+                const float4* hp = reinterpret_cast<const float4*>(p.init_conv + ((size_t)n * 3 + xi) * p.C + ch0);
+                const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
+                x[0] = h0.x; x[1] = h0.y; x[2] = h0.z; x[3] = h0.w;
+                x[4] = h1.x; x[5] = h1.y; x[6] = h1.z; x[7] = h1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[e][j], x[e], acc[e]);
+        }
+        float act[8];
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            act[e] = silu_f(acc[e]);
+            ss = fmaf(act[e], act[e], ss);
+        }
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        float scale = 1.0f;
+        if (!is_v) {
+            scale = rsqrtf(ss + kEps);
+            if (is_q) scale *= rsqrtf((float)kD);
+        }
+        if (!active) continue;
+        uint4 pk;
+        pk.x = pack_half2(act[0] * scale, act[1] * scale);
+        pk.y = pack_half2(act[2] * scale, act[3] * scale);
+        pk.z = pack_half2(act[4] * scale, act[5] * scale);
+        pk.w = pack_half2(act[6] * scale, act[7] * scale);
+        __half* dst;
+        if (is_q) dst = p.Qs + (size_t)t * p.Kh * kD + slot * kD + gl * 8;
+        else if (is_k) dst = p.Ks + (size_t)t * p.Kh * kD + (slot - p.Kh) * kD + gl * 8;
+        else dst = p.Vs + (size_t)t * p.Vh * kD + vh * kD + gl * 8;
+        *reinterpret_cast<uint4*>(dst) = pk;
+        if (is_v && gl == 0) {
+            const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
+            const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);
+            p.Gs[(size_t)vh * p.total + t] = -gA * softplus_f(av + gdt);
+            p.Bs[(size_t)vh * p.total + t] = sigmoid_f(bv);
+        }
+    }
+}
+
+struct ConvOutParams {
+    int C, N;
+    SeqIndex seq;
+    const uint16_t* qkv;     // bf16 [total][C]
+    const float* init_conv;  // f32 [N][3][C] or nullptr
+    float* final_conv;       // f32 [N][3][C]; may alias init_conv
+};
+
+// final_conv[n][r] = row L+r of [history (3 rows); the row's L tokens].
+// In place is safe: for each channel the thread reads index L+r >= r before
+// writing index r, in increasing r.
+__global__ void __launch_bounds__(256) gdn_conv_out_kernel(const ConvOutParams p) {
+    const int n = blockIdx.y;
+    const int ch = blockIdx.x * blockDim.x + threadIdx.x;
+    if (ch >= p.C) return;
+    int start, len;
+    p.seq.bounds(n, start, len);
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+        const int e = len + r;
+        float v;
+        if (e >= 3) v = bf16_bits_to_float(p.qkv[(size_t)(start + e - 3) * p.C + ch]);
+        else v = p.init_conv ? p.init_conv[((size_t)n * 3 + e) * p.C + ch] : 0.f;
+        p.final_conv[((size_t)n * 3 + r) * p.C + ch] = v;
+    }
+}
+
+}  // namespace gdn

@@ -1,0 +1,150 @@
+/*
+ * gdn.h — C ABI of the B200 (sm_100a) Gated DeltaNet token mixer.
+ *
+ * The mixer is the linear-attention layer of the Qwen3.8-27B hybrid decoder
+ * (Qwen3.8 27B model card, "Gated DeltaNet" bullet): from the projected qkv
+ * (10240 channels), z (6144), a and b (48 each) it runs a width-4 depthwise
+ * causal conv with silu, L2-normalises q and k, forms the decay
+ * g = -exp(A_log) * softplus(a + dt_bias) and the write rate beta = sigmoid(b),
+ * runs the gated delta rule on a [128,128] f32 state per value head (16 q/k
+ * heads, each read by 3 of the 48 value heads), reads out o = S (q / sqrt(128)),
+ * and applies the zero-centred gated RMSNorm o * rsqrt(mean(o^2) + 1e-6) *
+ * (1 + w) * silu(z) (same card, "Norms" bullet; Qwen/Qwen3.8-27B architecture
+ * page, header table: eps 1e-06).  Each row keeps its conv history and its
+ * recurrent state in f32 between calls (same card, cache paragraph).
+ *
+ * Conventions (readings where the pages are silent):
+ *   - qkv channel order [q | k | v], heads contiguous, 128 channels each;
+ *   - value head h reads q/k head h / (Vh / Kh);
+ *   - conv tap W-1 multiplies the current token, tap 0 the token W-1 back;
+ *     no conv bias; missing history is zero;
+ *   - state layout [row][value head][v index i][k index j] (row i of S maps
+ *     keys to value channel i, so S k is a per-row dot product);
+ *   - conv history layout [row][W-1][C], oldest row first, stored as the
+ *     exact f32 widening of the bf16 inputs.
+ *
+ * Memory: every pointer is DEVICE memory owned by the caller, 16-byte
+ * aligned, densely packed in the layouts given.  bf16 tensors are passed as
+ * uint16_t bit patterns.  The library allocates nothing and keeps no state
+ * between calls other than a per-process cache of driver entry points.
+ *
+ * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ * Every call only enqueues work on it and returns; results are ready when
+ * the stream reaches that point.  Calls that share buffers must be ordered
+ * by the caller.
+ *
+ * Errors: functions return GDN_OK (0) or a negative status.  Argument errors
+ * are detected on the host before anything is enqueued.  A launch failure
+ * returns GDN_ERR_CUDA.  A device-side wait that ran past its limit sets the
+ * error word read by gdn_last_device_error(); faults inside a kernel surface
+ * as CUDA errors at the caller's next synchronisation.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = -1, /* null / misaligned pointer, negative size, bad cu_seqlens */
+    GDN_ERR_UNSUPPORTED = -2, /* head_dim != 128, conv_width != 4, Vh % Kh != 0, Vh/Kh > 8, not sm_100 */
+    GDN_ERR_CUDA = -3,        /* a CUDA runtime / driver call failed */
+    GDN_ERR_WORKSPACE = -4,   /* workspace missing or smaller than the *_workspace_size query */
+    GDN_ERR_TIMEOUT = -5      /* a bounded device-side wait expired (see gdn_last_device_error) */
+};
+
+typedef struct gdn_dims {
+    int32_t num_k_heads; /* Kh: query/key heads (16 in the 27B model) */
+    int32_t num_v_heads; /* Vh: value heads (48) */
+    int32_t head_dim;    /* D: width of every head (128; the only supported value) */
+    int32_t conv_width;  /* W: conv taps (4; the only supported value) */
+} gdn_dims;
+
+typedef struct gdn_weights {
+    const uint16_t* conv_w; /* bf16 [C][W], C = (2*Kh + Vh) * D, depthwise conv taps */
+    const float* A_log;     /* f32 [Vh] */
+    const float* dt_bias;   /* f32 [Vh] */
+    const float* norm_w;    /* f32 [D], zero-centred: the norm scales by (1 + w) */
+} gdn_weights;
+
+/* Bytes of device workspace gdn_prefill needs for B rows of T tokens.
+ * Returns 0 for invalid dims. */
+size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
+
+/*
+ * Dense prefill: B rows of T tokens each, all rows at their own state.
+ *   qkv  bf16 [B][T][C]         z bf16 [B][T][Vh*D]       a, b bf16 [B][T][Vh]
+ *   init_state f32 [B][Vh][D][D] or NULL (zero state)
+ *   init_conv  f32 [B][W-1][C]    or NULL (zero history)
+ *   out        bf16 [B][T][Vh*D]  gated-norm output, head-major
+ *   final_state f32 [B][Vh][D][D] may alias init_state (updated in place)
+ *   final_conv  f32 [B][W-1][C]   may alias init_conv
+ *   workspace: at least gdn_prefill_workspace_size(dims, B, T) bytes.
+ * T = 0 is legal: states and histories are copied through.
+ * The prefill computes the recurrence in chunks of 64 tokens (WY form) on
+ * tensor cores with f16 operands and f32 accumulation.
+ */
+int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T,
+                const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                const float* init_state, const float* init_conv,
+                uint16_t* out, float* final_state, float* final_conv,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace gdn_prefill_varlen needs for N rows with
+ * total_T tokens in all.  Returns 0 for invalid dims. */
+size_t gdn_prefill_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T);
+
+/*
+ * Packed (variable-length) prefill of N rows ("prefill_slots": a server's
+ * rows, each at its own length).  Row n owns tokens [cu[n], cu[n+1]) of the
+ * packed tensors.  cu_seqlens_host (host memory) and cu_seqlens_dev (device
+ * memory) hold the same N+1 int32 values: cu[0] = 0, non-decreasing,
+ * cu[N] = total_T.  The host copy is read during the call for validation and
+ * planning; the device copy is read by the kernels.
+ *   qkv bf16 [total_T][C], z bf16 [total_T][Vh*D], a, b bf16 [total_T][Vh]
+ *   init_state / final_state f32 [N][Vh][D][D], init_conv / final_conv f32
+ *   [N][W-1][C], out bf16 [total_T][Vh*D]; aliasing and NULL rules as for
+ *   gdn_prefill.  Zero-length rows are legal (state and history copied).
+ */
+int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N,
+                       const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int32_t total_T,
+                       const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                       const float* init_state, const float* init_conv,
+                       uint16_t* out, float* final_state, float* final_conv,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step for `rows` rows ("decode_rows": each row at its own
+ * length; GDN has no positional encoding, so a row's position enters only
+ * through its state and history).  Every step reads and rewrites each row's
+ * f32 state once.
+ *   qkv bf16 [rows][C], z bf16 [rows][Vh*D], a, b bf16 [rows][Vh]
+ *   state f32 [rows][Vh][D][D]   in/out, updated in place
+ *   conv  f32 [rows][W-1][C]     in/out, shifted by one token in place
+ *   out   bf16 [rows][Vh*D]
+ * rows = 0 is a legal no-op.  No workspace.
+ */
+int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
+               const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+               float* state, float* conv, uint16_t* out, void* stream);
+
+/* Device-side error word of the current device: 0, or the code of the last
+ * bounded wait that expired (cleared by reading).  Synchronises the device. */
+int gdn_last_device_error(void);
+
+/* Human-readable text of a gdn_status value (static storage). */
+const char* gdn_status_string(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

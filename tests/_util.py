@@ -1,0 +1,69 @@
+"""Shared helpers of the tests: run the oracle on a synthetic case, move a case
+to the GPU, and the parity measures with their bars.
+
+Bars (stated for the GDN path): outputs max|y - y_ref| / rms(y_ref) <= 2e-2
+per output tensor; final states ||S - S_ref||_F / ||S_ref||_F <= 1e-3 per row;
+conv histories bit-exact.
+"""
+import numpy as np
+import torch
+
+import oracle
+from gated_deltanet_mixer_gdn_b200 import synth
+
+OUT_TOL = 2e-2
+STATE_TOL = 1e-3
+
+
+def oracle_prefill(case, cu=None, heads=None, nthreads=0, init_state=None, init_conv=None, acts=None):
+    """Oracle on a synth case (dense cases are flattened to packed rows)."""
+    d = case["dims"]
+    f = synth.to_f64
+    w = case["weights"]
+    acts = acts or {k: case[k] for k in ("qkv", "z", "a", "b")}
+    if cu is None:
+        if "cu_seqlens" in case:
+            cu = case["cu_seqlens"].numpy()
+        else:
+            B, T = acts["qkv"].shape[0], acts["qkv"].shape[1]
+            cu = np.arange(B + 1, dtype=np.int64) * T
+    flat = {k: v.reshape(-1, v.shape[-1]) for k, v in acts.items()}
+    st = case["init_state"] if init_state is None else init_state
+    cv = case["init_conv"] if init_conv is None else init_conv
+    return oracle.mixer(d, cu, f(flat["qkv"]), f(flat["z"]), f(flat["a"]), f(flat["b"]),
+                        f(w["conv_w"]), f(w["A_log"]), f(w["dt_bias"]), f(w["norm_w"]),
+                        None if st is None else (st.numpy() if isinstance(st, torch.Tensor) else st).astype(np.float64),
+                        None if cv is None else (cv.numpy() if isinstance(cv, torch.Tensor) else cv).astype(np.float64),
+                        heads=heads, nthreads=nthreads)
+
+
+def out_err(y, y_ref):
+    y = y.float().cpu().numpy().astype(np.float64) if isinstance(y, torch.Tensor) else y
+    y = y.reshape(y_ref.shape)
+    rms = np.sqrt(np.mean(y_ref * y_ref))
+    return float(np.abs(y - y_ref).max() / max(rms, 1e-30))
+
+
+def state_err(S, S_ref):
+    """Worst per-row relative Frobenius error; S, S_ref [N, H, D, D]."""
+    S = S.double().cpu().numpy() if isinstance(S, torch.Tensor) else S
+    S = S.reshape(S_ref.shape)
+    errs = []
+    for n in range(S_ref.shape[0]):
+        den = np.linalg.norm(S_ref[n])
+        num = np.linalg.norm(S[n] - S_ref[n])
+        errs.append(num / den if den > 0 else num)
+    return float(max(errs)) if errs else 0.0
+
+
+def conv_exact(cv, cv_ref):
+    cv = cv.double().cpu().numpy() if isinstance(cv, torch.Tensor) else cv
+    return bool(np.array_equal(cv.reshape(cv_ref.shape), cv_ref))
+
+
+def to_dev(case, device="cuda"):
+    w = {k: v.to(device) for k, v in case["weights"].items()}
+    acts = {k: case[k].to(device) for k in ("qkv", "z", "a", "b")}
+    st = None if case["init_state"] is None else case["init_state"].to(device)
+    cv = None if case["init_conv"] is None else case["init_conv"].to(device)
+    return w, acts, st, cv

@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads and exports
+every function include/gdn.h declares, the workspace queries, and argument
+validation (all rejected before any CUDA call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_deltanet_mixer_gdn_b200 as gdn
+from gated_deltanet_mixer_gdn_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return gdn.load_library()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert set(names) == set(gdn.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.gdn_version() >= 100
+    assert gdn.status_string(0) == "ok"
+    assert "workspace" in gdn.status_string(-4)
+
+
+def _dims(kh=16, vh=48, d=128, w=4):
+    return gdn._DimsC(kh, vh, d, w)
+
+
+def test_workspace_sizes(lib):
+    d = _dims()
+    one = lib.gdn_prefill_workspace_size(ctypes.byref(d), 1, 1)
+    big = lib.gdn_prefill_workspace_size(ctypes.byref(d), 2, 1000)
+    assert one > 0 and big >= 2000 * (2 * 16 * 128 * 2 + 48 * 128 * 2 + 2 * 48 * 4)
+    assert lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 3, 2000) == big
+    assert lib.gdn_prefill_workspace_size(ctypes.byref(_dims(d=64)), 1, 10) == 0
+    assert lib.gdn_prefill_workspace_size(ctypes.byref(d), -1, 10) == 0
+
+
+def test_unsupported_dims_rejected(lib):
+    w = gdn._WeightsC(16, 16, 16, 16)
+    for bad, code in ((_dims(d=64), -2), (_dims(w=3), -2), (_dims(kh=5, vh=48), -2), (_dims(kh=1, vh=16), -2),
+                      (_dims(kh=0), -1)):
+        st = lib.gdn_decode(ctypes.byref(bad), ctypes.byref(w), 1, *([None] * 7), None)
+        assert st == code
+
+
+def test_invalid_arguments_rejected(lib):
+    d = _dims()
+    w = gdn._WeightsC(16, 16, 16, 16)
+    # null weights
+    assert lib.gdn_decode(ctypes.byref(d), None, 1, *([None] * 7), None) == -1
+    # null buffers with rows > 0
+    assert lib.gdn_decode(ctypes.byref(d), ctypes.byref(w), 2, *([None] * 7), None) == -1
+    # misaligned state pointer
+    assert lib.gdn_decode(ctypes.byref(d), ctypes.byref(w), 2, 16, 16, 16, 16, 8, 16, 16, None) == -1
+    # rows < 0
+    assert lib.gdn_decode(ctypes.byref(d), ctypes.byref(w), -1, *([None] * 7), None) == -1
+    # varlen: cu_seqlens not starting at 0 / decreasing / wrong total
+    for cu, total in (([1, 5], 5), ([0, 5, 3], 3), ([0, 4], 5)):
+        arr = (ctypes.c_int32 * len(cu))(*cu)
+        st = lib.gdn_prefill_varlen(ctypes.byref(d), ctypes.byref(w), len(cu) - 1, arr, 16, total,
+                                    16, 16, 16, 16, None, None, 16, None, None, 16, 1 << 30, None)
+        assert st == -1
+    # prefill: negative T
+    assert lib.gdn_prefill(ctypes.byref(d), ctypes.byref(w), 1, -3, *([16] * 4), None, None, 16, None, None,
+                           16, 1 << 30, None) == -1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from gated_deltanet_mixer_gdn_b200 import synth
+    case = synth.dense_case(1, 1, 4)
+    with pytest.raises(gdn.GdnError):
+        gdn.prefill(case["qkv"], case["z"], case["a"], case["b"], case["weights"])
