@@ -84,7 +84,7 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t
 }
 
 struct Workspace {
-    size_t off_q, off_k, off_v, off_g, off_b, bytes;
+    size_t off_q, off_k, off_ql, off_kl, off_v, off_g, off_b, bytes;
 };
 
 Workspace plan_workspace(const gdn_dims* d, int64_t total) {
@@ -94,7 +94,9 @@ Workspace plan_workspace(const gdn_dims* d, int64_t total) {
     const size_t gb = (size_t)total * d->num_v_heads * 4;
     w.off_q = 0;
     w.off_k = align_up(qk);
-    w.off_v = w.off_k + align_up(qk);
+    w.off_ql = w.off_k + align_up(qk);
+    w.off_kl = w.off_ql + align_up(qk);
+    w.off_v = w.off_kl + align_up(qk);
     w.off_g = w.off_v + align_up(vv);
     w.off_b = w.off_g + align_up(gb);
     w.bytes = w.off_b + align_up(gb);
@@ -133,6 +135,8 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
     __half* Qs = reinterpret_cast<__half*>(wsb + ws.off_q);
     __half* Ks = reinterpret_cast<__half*>(wsb + ws.off_k);
+    __half* Ql = reinterpret_cast<__half*>(wsb + ws.off_ql);
+    __half* Kl = reinterpret_cast<__half*>(wsb + ws.off_kl);
     __half* Vs = reinterpret_cast<__half*>(wsb + ws.off_v);
     float* Gs = reinterpret_cast<float*>(wsb + ws.off_g);
     float* Bs = reinterpret_cast<float*>(wsb + ws.off_b);
@@ -154,6 +158,8 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         pp.init_conv = init_conv;
         pp.Qs = Qs;
         pp.Ks = Ks;
+        pp.Ql = Ql;
+        pp.Kl = Kl;
         pp.Vs = Vs;
         pp.Gs = Gs;
         pp.Bs = Bs;
@@ -176,8 +182,12 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     }
     // 3. chunked recurrence on tensor cores, gated RMSNorm epilogue
     {
-        CUtensorMap mK, mQ, mV, mZ;
+        CUtensorMap mK, mQ, mKl, mQl, mV, mZ;
         if (!make_map(&mK, Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mKl, Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mQl, Ql, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&mQ, Qs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -205,7 +215,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         });
         if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
         dim3 grid(Vh, N);
-        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mK, mQ, mV, mZ, cp);
+        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mK, mQ, mKl, mQl, mV, mZ, cp);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     return GDN_OK;

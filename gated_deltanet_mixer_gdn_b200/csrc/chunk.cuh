@@ -29,8 +29,11 @@
 // and the 64 x 128 bf16 output tile leaves with coalesced 16-byte stores.
 //
 // Inputs come from the load-stage kernel (conv, L2 norm, gates) as f16 tiles
-// fetched with TMA: K and Q of the q/k head (double-buffered), V of the
-// value head, and the z tile for the gate of the norm.
+// fetched with TMA: K and Q of the q/k head (double-buffered) with their f16
+// residuals, V of the value head, and the z tile for the gate of the norm.
+// MMA1 uses the residuals (hi.hi + hi.lo + lo.hi): the dot products of nearly
+// orthogonal q and k cancel, and one f16 rounding of q and k then dominates
+// the error of the normalised outputs.
 #pragma once
 
 #include "common.cuh"
@@ -54,25 +57,28 @@ constexpr int C = 64;              // tokens per chunk
 constexpr int kThreads = 256;
 constexpr int LDA = 68;            // f32 row stride of the A / T matrix (conflict-free float4 rows)
 // shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ0 = 0;        // [K rows 0-63 | Q rows 64-127] x k 0-63, then x k 64-127
+constexpr uint32_t OFF_KQ0 = 0;        // [K rows 0-63 | Q rows 64-127] x k 0-63, then x k 64-127 (f16 hi parts)
 constexpr uint32_t OFF_KQ1 = 32768;    // second buffer
-constexpr uint32_t OFF_V = 65536;      // V [64 t][64 v] x 2 blocks
-constexpr uint32_t OFF_Z = 81920;      // z bf16 [64][128], plain row-major; reused for y
-constexpr uint32_t OFF_WT = 98304;     // W^T f16 [128 k][64 t]
-constexpr uint32_t OFF_UT = 114688;    // U^T f16 [128 v][64 t]; T-solve scratch before that
-constexpr uint32_t OFF_UTS = 131072;   // U^T diag(e^{G_C-G}) f16
-constexpr uint32_t OFF_S = 147456;     // S0 f16 [128 v][64 k] x 2 blocks
-constexpr uint32_t OFF_T1 = 180224;    // T diag(beta) f16 [64][64]
-constexpr uint32_t OFF_T2 = 188416;    // T diag(beta e^G) f16 [64][64]
-constexpr uint32_t OFF_M = 196608;     // tril(Q K^T) * E f16 [64][64]
-constexpr uint32_t OFF_A = 204800;     // A, then T, f32 [64][LDA]
-constexpr uint32_t OFF_MISC = OFF_A + 64 * LDA * 4;  // 222208
+constexpr uint32_t OFF_LO = 65536;     // same layout, f16 residuals (lo parts); A / T f32 once MMA1 is done
+constexpr uint32_t OFF_V = 98304;      // V [64 t][64 v] x 2 blocks
+constexpr uint32_t OFF_WT = 114688;    // W^T f16 [128 k][64 t]; z / y bf16 [64][128] once MMA4 is done
+constexpr uint32_t OFF_UT = 131072;    // U^T f16 [128 v][64 t]; T-solve scratch before that
+constexpr uint32_t OFF_UTS = 147456;   // U^T diag(e^{G_C-G}) f16
+constexpr uint32_t OFF_S = 163840;     // S0 f16 [128 v][64 k] x 2 blocks
+constexpr uint32_t OFF_T1 = 196608;    // T diag(beta) f16 [64][64]
+constexpr uint32_t OFF_T2 = 204800;    // T diag(beta e^G) f16 [64][64]
+constexpr uint32_t OFF_M = 212992;     // tril(Q K^T) * E f16 [64][64]
+constexpr uint32_t OFF_A = OFF_LO;     // A, then T, f32 [64][LDA]
+constexpr uint32_t OFF_Z = OFF_WT;
+constexpr uint32_t OFF_MISC = 221184;
 constexpr uint32_t MISC_BYTES = 2048;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+static_assert(64 * LDA * 4 <= 32768, "A/T must fit in the residual tile");
 // TMEM columns (f32, 128 lanes)
 constexpr uint32_t T_KQ = 0, T_UT = 64, T_WT = 128, T_OI = 192, T_OA = 256, T_S = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t KQV_BYTES = 6 * 8192;
+constexpr uint32_t LO_BYTES = 4 * 8192;
 constexpr uint32_t Z_BYTES = 64 * 128 * 2;
 constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, false, false, false);
 constexpr uint32_t ID_AMN = idesc_f16_f32(128, 64, true, false, false);
@@ -167,6 +173,7 @@ __device__ __forceinline__ void store_row_f16_sw128(uint8_t* tile, uint32_t row,
 
 __global__ void __launch_bounds__(chunk::kThreads, 1)
     gdn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmQl,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZ,
                      const ChunkParams p) {
     using namespace chunk;
@@ -186,6 +193,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     uint64_t* bar_kqv = reinterpret_cast<uint64_t*>(smem + OFF_MISC);
     uint64_t* bar_z = bar_kqv + 1;
     uint64_t* bar_mma = bar_kqv + 2;
+    uint64_t* bar_lo = bar_kqv + 3;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 32);
     float* s_G = reinterpret_cast<float*>(smem + OFF_MISC + 64);     // [64]
     float* s_eG = s_G + 64;                                            // [64]
@@ -202,9 +210,12 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         mbar_init(bar_kqv, 1);
         mbar_init(bar_z, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_lo, 1);
         fence_barrier_init();
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmKl);
+        prefetch_tensormap(&tmQl);
         prefetch_tensormap(&tmV);
         prefetch_tensormap(&tmZ);
     }
@@ -243,8 +254,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         tma_load_2d(smem + OFF_KQ0 + 24576, &tmQ, kap * 128 + 64, start, bar_kqv);
         tma_load_2d(smem + OFF_V, &tmV, h * 128, start, bar_kqv);
         tma_load_2d(smem + OFF_V + 8192, &tmV, h * 128 + 64, start, bar_kqv);
-        mbar_arrive_expect_tx(bar_z, Z_BYTES);
-        tma_load_2d(smem + OFF_Z, &tmZ, h * 128, start, bar_z);
+        mbar_arrive_expect_tx(bar_lo, LO_BYTES);
+        tma_load_2d(smem + OFF_LO, &tmKl, kap * 128, start, bar_lo);
+        tma_load_2d(smem + OFF_LO + 16384, &tmKl, kap * 128 + 64, start, bar_lo);
+        tma_load_2d(smem + OFF_LO + 8192, &tmQl, kap * 128, start, bar_lo);
+        tma_load_2d(smem + OFF_LO + 24576, &tmQl, kap * 128 + 64, start, bar_lo);
     }
     __syncthreads();
 
@@ -272,20 +286,32 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             s_beta[tid] = bt;
         }
         CHUNK_WAIT(bar_kqv, c & 1, kErrTimeoutTma);  // includes a CTA barrier
+        CHUNK_WAIT(bar_lo, c & 1, kErrTimeoutTma);
         if (tid < 64) {
             float G = s_G[tid];
             if (tid >= 32) G += s_G[31];
             s_G[tid] = G;
             s_eG[tid] = expf(G);
         }
-        // ---- MMA1: [K;Q] K^T
+        // ---- MMA1: [K;Q] K^T from hi/lo f16 parts: hi.hi + hi.lo + lo.hi
         if (tid == 0) {
             tc_fence_after();
+            const uint32_t aLO = sbase + OFF_LO;
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
                 mma_f16(tbase + T_KQ, sw128_desc(aKQ + off, 16, 1024), sw128_desc(aKQ + off, 16, 1024), ID_KK,
                         s > 0);
+            }
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                mma_f16(tbase + T_KQ, sw128_desc(aKQ + off, 16, 1024), sw128_desc(aLO + off, 16, 1024), ID_KK, 1);
+            }
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                mma_f16(tbase + T_KQ, sw128_desc(aLO + off, 16, 1024), sw128_desc(aKQ + off, 16, 1024), ID_KK, 1);
             }
             mma_commit(bar_mma);
         }
@@ -360,6 +386,15 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
         // ---- MMA2: U~^T = V^T (T diag beta)^T ; MMA3: W^T = K^T (T diag(beta e^G))^T
         if (tid == 0) {
+            // A / T are consumed: the residual tile of the next chunk can land.
+            if (c + 1 < nchunks) {
+                const int y = tok0 + C;
+                mbar_arrive_expect_tx(bar_lo, LO_BYTES);
+                tma_load_2d(smem + OFF_LO, &tmKl, kap * 128, y, bar_lo);
+                tma_load_2d(smem + OFF_LO + 16384, &tmKl, kap * 128 + 64, y, bar_lo);
+                tma_load_2d(smem + OFF_LO + 8192, &tmQl, kap * 128, y, bar_lo);
+                tma_load_2d(smem + OFF_LO + 24576, &tmQl, kap * 128 + 64, y, bar_lo);
+            }
             tc_fence_after();
 #pragma unroll
             for (int s = 0; s < 4; ++s)
@@ -418,6 +453,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         CHUNK_WAIT(bar_mma, mma_phase, kErrTimeoutMma);
         mma_phase ^= 1;
         tc_fence_after();
+        // W^T is consumed: the z tile of this chunk lands in its place.
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar_z, Z_BYTES);
+            tma_load_2d(smem + OFF_Z, &tmZ, h * 128, tok0, bar_z);
+        }
 
         // ---- U^T to shared memory, plain and scaled by e^{G_C - G_t}
         {
@@ -482,7 +522,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             s_red[q4 * 64 + 32 * hf + lane] = part;
             __syncthreads();
             uint16_t* zt = reinterpret_cast<uint16_t*>(smem + OFF_Z);
-#pragma unroll 8
+#pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
                 const int t = 32 * hf + jj;
                 const float ms = (s_red[t] + s_red[64 + t] + s_red[128 + t] + s_red[192 + t]) * (1.0f / 128.0f);
@@ -502,10 +542,6 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0 && c + 1 < nchunks) {
-            mbar_arrive_expect_tx(bar_z, Z_BYTES);
-            tma_load_2d(smem + OFF_Z, &tmZ, h * 128, tok0 + C, bar_z);
-        }
     }
 
     if (!failed && p.final_state != nullptr) {

@@ -62,6 +62,8 @@ struct PrepParams {
     const float* init_conv;   // f32 [N][3][C] or nullptr
     __half* Qs;
     __half* Ks;
+    __half* Ql;
+    __half* Kl;
     __half* Vs;
     float* Gs;
     float* Bs;
@@ -156,16 +158,29 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
             if (is_q) scale *= rsqrtf((float)kD);
         }
         if (!active) continue;
+        float xs[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xs[e] = act[e] * scale;
         uint4 pk;
-        pk.x = pack_half2(act[0] * scale, act[1] * scale);
-        pk.y = pack_half2(act[2] * scale, act[3] * scale);
-        pk.z = pack_half2(act[4] * scale, act[5] * scale);
-        pk.w = pack_half2(act[6] * scale, act[7] * scale);
-        __half* dst;
-        if (is_q) dst = p.Qs + (size_t)t * p.Kh * kD + slot * kD + gl * 8;
-        else if (is_k) dst = p.Ks + (size_t)t * p.Kh * kD + (slot - p.Kh) * kD + gl * 8;
-        else dst = p.Vs + (size_t)t * p.Vh * kD + vh * kD + gl * 8;
-        *reinterpret_cast<uint4*>(dst) = pk;
+        pk.x = pack_half2(xs[0], xs[1]);
+        pk.y = pack_half2(xs[2], xs[3]);
+        pk.z = pack_half2(xs[4], xs[5]);
+        pk.w = pack_half2(xs[6], xs[7]);
+        if (is_v) {
+            *reinterpret_cast<uint4*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + gl * 8) = pk;
+        } else {
+            const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + gl * 8;
+            const __half2* hp = reinterpret_cast<const __half2*>(&pk);
+            uint4 lo;
+            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float2 hf = __half22float2(hp[m]);
+                lw[m] = pack_half2(xs[2 * m] - hf.x, xs[2 * m + 1] - hf.y);
+            }
+            *reinterpret_cast<uint4*>((is_q ? p.Qs : p.Ks) + off) = pk;
+            *reinterpret_cast<uint4*>((is_q ? p.Ql : p.Kl) + off) = lo;
+        }
         if (is_v && gl == 0) {
             const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
             const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);

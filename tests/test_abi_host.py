@@ -46,7 +46,7 @@ def test_workspace_sizes(lib):
     d = _dims()
     one = lib.gdn_prefill_workspace_size(ctypes.byref(d), 1, 1)
     big = lib.gdn_prefill_workspace_size(ctypes.byref(d), 2, 1000)
-    assert one > 0 and big >= 2000 * (2 * 16 * 128 * 2 + 48 * 128 * 2 + 2 * 48 * 4)
+    assert one > 0 and big >= 2000 * (4 * 16 * 128 * 2 + 48 * 128 * 2 + 2 * 48 * 4)
     assert lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 3, 2000) == big
     assert lib.gdn_prefill_workspace_size(ctypes.byref(_dims(d=64)), 1, 10) == 0
     assert lib.gdn_prefill_workspace_size(ctypes.byref(d), -1, 10) == 0
