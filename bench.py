@@ -270,8 +270,36 @@ def run_ours(args, world, rank, local):
     t_e2e = max_over_ranks(e2.elapsed_time(e3), world)
     e2e_value = world * ROWS * DECODE_STEPS * e2e_steps / (t_e2e / 1000.0)
 
-    # ---- chunked prefill, one row of 8192 tokens (secondary measurement)
-    pcase = synth.config(2)
+    line = None
+    if rank == 0:
+        line = {
+            "metric": "GDN decode row-tokens/s (64-row batch, 128 steps)",
+            "value": value, "unit": "row-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "decode 64 rows x 128 steps, Qwen3.8-27B GDN layer shapes (16 qk / 48 v heads, "
+                                   "dim 128), per-row f32 state", "rows": ROWS, "tokens_per_row": DECODE_STEPS,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (402.7 MB of state per step)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "gdn_decode_kernel", "peak_source": peaks["source"],
+                         "algorithmic_bytes_per_launch": ROWS * STATE_BYTES_PER_ROW_TOKEN},
+            "e2e": {"value": e2e_value, "unit": "row-tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "clocks": clocks,
+            "gpu_launches": launches,
+        }
+    return line, case
+
+
+def bench_prefill(args, world, rank, local, T):
+    """Chunked prefill of one row of T tokens (zero initial state), L2 flushed before each call."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(dev)
+    PREFILL_T = T
+    pcase = synth.config(2) if T == 8192 else synth.dense_case(1236, 1, T)
     pw = gdn.weights_to(pcase["weights"], dev)
     pin_acts = {k: pcase[k].to(dev) for k in ("qkv", "z", "a", "b")}
     pout = torch.empty((1, PREFILL_T, 6144), dtype=torch.bfloat16, device=dev)
@@ -295,33 +323,12 @@ def run_ours(args, world, rank, local):
             s1.synchronize()
             pt.append(s0.elapsed_time(s1) / 1000.0)
     p_med = statistics.median(pt)
-    prefill = {"workload": "prefill B=1 T=8192, zero initial state (3 kernels: load stage, history, chunk)",
-               "value": PREFILL_T / p_med, "unit": "tokens/s", "ms": p_med * 1000.0,
-               "tflops": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12,
-               "frac_of_bf16_peak": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12 / peaks["bf16_tflops"],
-               "peak_source": peaks["source"], "l2": "flushed (256 MiB write) before each timed call"}
-
-    line = None
-    if rank == 0:
-        line = {
-            "metric": "GDN decode row-tokens/s (64-row batch, 128 steps)",
-            "value": value, "unit": "row-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "decode 64 rows x 128 steps, Qwen3.8-27B GDN layer shapes (16 qk / 48 v heads, "
-                                   "dim 128), per-row f32 state", "rows": ROWS, "tokens_per_row": DECODE_STEPS,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (402.7 MB of state per step)"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "kernel": "gdn_decode_kernel", "peak_source": peaks["source"],
-                         "algorithmic_bytes_per_launch": ROWS * STATE_BYTES_PER_ROW_TOKEN},
-            "e2e": {"value": e2e_value, "unit": "row-tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "clocks": clocks,
-            "gpu_launches": launches,
-            "prefill": prefill,
-        }
-    return line, case
+    return {"workload": f"prefill B=1 T={T}, zero initial state (3 kernels: load stage, history, chunk)",
+            "value": PREFILL_T / p_med, "unit": "tokens/s", "ms": p_med * 1000.0,
+            "tflops": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12,
+            "frac_of_bf16_peak": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12 / peaks["bf16_tflops"],
+            "peak_source": peaks["source"], "l2": "flushed (256 MiB write) before each timed call",
+            "gpu_launches": 3 * len(pt)}
 
 
 def main():
@@ -331,6 +338,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+                    help="decode: the 64-row decode batch (default line); prefill: only the chunked prefill")
+    ap.add_argument("--prefill-T", type=int, default=PREFILL_T, help="tokens of the prefill measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -338,8 +348,15 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.workload == "prefill":
+            pre = bench_prefill(args, world, rank, local, args.prefill_T)
+            if rank == 0:
+                print(json.dumps({"metric": "GDN prefill tokens/s", **pre}))
+            return 0
         line, case = run_ours(args, world, rank, local)
+        pre = bench_prefill(args, world, rank, local, args.prefill_T)
         if rank == 0:
+            line["prefill"] = pre
             if world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline_line(case)
             print(json.dumps(line))
