@@ -26,7 +26,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen_workspace_size",
-           "gdn_prefill_varlen", "gdn_decode", "gdn_last_device_error", "gdn_status_string", "gdn_version")
+           "gdn_prefill_varlen", "gdn_decode", "gdn_prefill_noalloc", "gdn_last_device_error",
+           "gdn_status_string", "gdn_version")
 
 GDN_OK = 0
 

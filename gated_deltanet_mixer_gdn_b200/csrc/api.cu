@@ -235,6 +235,31 @@ int check_io(int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16
     return GDN_OK;
 }
 
+// Scratch of gdn_prefill_noalloc: one fixed array per device, never freed.
+// Host code must not pass g_noalloc_scratch itself to a kernel (on the host
+// it names a stand-in, not the device address): its device address is looked
+// up once per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (resolved on first use).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -328,6 +353,25 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cuda_status(cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p));
+}
+
+int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, const uint16_t* qkv,
+                        const uint16_t* z, const uint16_t* a, const uint16_t* b, const float* init_state,
+                        const float* init_conv, uint16_t* out, float* final_state, float* final_conv, void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (B < 0 || T < 0 || B > 65535) return GDN_ERR_INVALID_ARG;
+    const int64_t total = (int64_t)B * T;
+    if (total > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if ((st = check_io((int32_t)total, qkv, z, a, b, out, init_state, init_conv, final_state, final_conv)) != GDN_OK)
+        return st;
+    if (plan_workspace(dims, total).bytes > (size_t)GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
+    if ((st = check_device()) != GDN_OK) return st;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != GDN_OK) return st;
+    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, qkv, z, a, b, init_state, init_conv, out, final_state,
+                        final_conv, scratch, (size_t)GDN_NOALLOC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
 }
 
 int gdn_last_device_error(void) {

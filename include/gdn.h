@@ -26,7 +26,8 @@
  * Memory: every pointer is DEVICE memory owned by the caller, 16-byte
  * aligned, densely packed in the layouts given.  bf16 tensors are passed as
  * uint16_t bit patterns.  The library allocates nothing and keeps no state
- * between calls other than a per-process cache of driver entry points.
+ * between calls other than a per-process cache of driver entry points, a
+ * device-side error word, and the fixed scratch array of gdn_prefill_noalloc.
  *
  * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  * Every call only enqueues work on it and returns; results are ready when
@@ -132,6 +133,35 @@ int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N,
 int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
                const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
                float* state, float* conv, uint16_t* out, void* stream);
+
+/*
+ * gdn_prefill without a caller-supplied workspace, for callers that cannot
+ * call cudaMalloc: for example a plugin inside an inference engine that owns
+ * every device allocation, or a latency-critical path that must not take the
+ * implicit device synchronisation of an allocation.  (The pages have no
+ * counterpart: this is a deployment convenience of this library.)
+ *
+ * Same arguments, layouts, aliasing and results as gdn_prefill, minus
+ * workspace / workspace_bytes.  The scratch lives in one file-scope device
+ * array of GDN_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads this
+ * library holds until the process exits.  A request whose scratch exceeds it
+ * is rejected with GDN_ERR_WORKSPACE before anything is enqueued; for the
+ * 27B model's dims (16/48 heads) that is B*T > 1154 tokens (29,056 bytes per
+ * token plus alignment).  The call itself allocates nothing.
+ *
+ * The first call on each device resolves the device address of the array
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call shares the one array and the array
+ * keeps the previous call's contents; nothing in it needs to start at zero
+ * (every byte is written before it is read within a call).  Calls whose work
+ * overlaps on the GPU (different streams, or different host threads without
+ * ordering) race on the array: order them on one stream.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T,
+                        const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                        const float* init_state, const float* init_conv,
+                        uint16_t* out, float* final_state, float* final_conv, void* stream);
 
 /* Device-side error word of the current device: 0, or the code of the last
  * bounded wait that expired (cleared by reading).  Synchronises the device. */
