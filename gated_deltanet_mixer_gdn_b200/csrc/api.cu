@@ -21,6 +21,7 @@ namespace {
 using namespace gdn;
 
 constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -241,7 +242,6 @@ int check_io(int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16
 // up once per device below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
 
@@ -340,16 +340,43 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
     p.state = state;
     p.conv = conv;
     p.out = out;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(p.Vh, rows);
-    cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = static_cast<cudaStream_t>(stream);
+    static std::once_flag dec_once;
+    static cudaError_t dec_err = cudaSuccess;
+    std::call_once(dec_once, [] {
+        dec_err = cudaFuncSetAttribute(gdn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)dec::SMEM_BYTES);
+    });
+    if (dec_err != cudaSuccess) return GDN_ERR_CUDA;
+    const int group = p.Vh / p.Kh;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.Vh / p.Kh;
+    attr[0].val.clusterDim.x = group;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // Persistent grid: as many row partitions P as keep every cluster resident at once
+    // (one CTA per SM; a partition is Vh / group clusters).
+    static int cached_clusters[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
+    int max_clusters = cached_clusters[dev];
+    if (max_clusters == 0) {
+        cudaLaunchConfig_t q{};
+        q.gridDim = dim3(p.Vh, 1);
+        q.blockDim = dim3(dec::kThreads);
+        q.dynamicSmemBytes = dec::SMEM_BYTES;
+        q.attrs = attr;
+        q.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, gdn_decode_kernel, &q) != cudaSuccess) return GDN_ERR_CUDA;
+        cached_clusters[dev] = max_clusters;
+    }
+    p.P = max_clusters / p.Kh;
+    if (p.P < 1) p.P = 1;
+    if (p.P > rows) p.P = rows;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.Vh, p.P);
+    cfg.blockDim = dim3(dec::kThreads);
+    cfg.dynamicSmemBytes = dec::SMEM_BYTES;
+    cfg.stream = static_cast<cudaStream_t>(stream);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cuda_status(cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p));
