@@ -370,6 +370,9 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
         cached_clusters[dev] = max_clusters;
     }
     p.P = max_clusters / p.Kh;
+#ifdef GDN_DECODE_PART
+    p.P = GDN_DECODE_PART;
+#endif
     if (p.P < 1) p.P = 1;
     if (p.P > rows) p.P = rows;
     cudaLaunchConfig_t cfg{};

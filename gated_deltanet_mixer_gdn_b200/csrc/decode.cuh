@@ -47,8 +47,18 @@ struct DecodeParams {
     uint16_t* out;           // bf16 [rows][Vh*128]
 };
 
+#ifndef GDN_DECODE_STAGES
+#define GDN_DECODE_STAGES 6
+#endif
+#ifndef GDN_DECODE_STORE_LAG
+#define GDN_DECODE_STORE_LAG 1
+#endif
+
 namespace dec {
-constexpr int kStages = 6;
+constexpr int kStages = GDN_DECODE_STAGES;
+// A stage is refilled once the bulk store issued this many units later has
+// been started, so a store has that long to drain before its stage is reused.
+constexpr int kStoreLag = GDN_DECODE_STORE_LAG;
 constexpr uint32_t kTileBytes = 64 * 128 * 4;  // half of a head's state
 constexpr int kComputeThreads = 256;
 constexpr int kThreads = kComputeThreads + 32;  // + producer warp
@@ -141,10 +151,14 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                     bounded_wait(&empty[st], (u / kStages) & 1, broken);
                     bulk_store(tile_src(u), smem + st * kTileBytes, kTileBytes);
                     bulk_commit();
-                    if (u + kStages < nunits) {
-                        bulk_wait_read_all();
-                        mbar_arrive_expect_tx(&full[st], kTileBytes);
-                        bulk_load(smem + st * kTileBytes, tile_src(u + kStages), kTileBytes, &full[st]);
+                    // refill the stage of unit v = u - kStoreLag once its store has read the stage
+                    const int v = u - kStoreLag;
+                    if (v >= 0 && v + kStages < nunits) {
+                        if (kStoreLag == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                        else asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kStoreLag) : "memory");
+                        const int sv = v % kStages;
+                        mbar_arrive_expect_tx(&full[sv], kTileBytes);
+                        bulk_load(smem + sv * kTileBytes, tile_src(v + kStages), kTileBytes, &full[sv]);
                     }
                 }
             }

@@ -82,7 +82,6 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     const int slot = active ? blockIdx.y * 16 + grp : nheads - 1;
     const int ch0 = slot * kD + gl * 8;
     const bool is_q = slot < p.Kh;
-    const bool is_k = !is_q && slot < 2 * p.Kh;
     const bool is_v = slot >= 2 * p.Kh;
     const int vh = slot - 2 * p.Kh;
 
