@@ -347,41 +347,20 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
                                        (int)dec::SMEM_BYTES);
     });
     if (dec_err != cudaSuccess) return GDN_ERR_CUDA;
-    const int group = p.Vh / p.Kh;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = group;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    // Persistent grid: as many row partitions P as keep every cluster resident at once
-    // (one CTA per SM; a partition is Vh / group clusters).
-    static int cached_clusters[kMaxDevices] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
-    int max_clusters = cached_clusters[dev];
-    if (max_clusters == 0) {
-        cudaLaunchConfig_t q{};
-        q.gridDim = dim3(p.Vh, 1);
-        q.blockDim = dim3(dec::kThreads);
-        q.dynamicSmemBytes = dec::SMEM_BYTES;
-        q.attrs = attr;
-        q.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&max_clusters, gdn_decode_kernel, &q) != cudaSuccess) return GDN_ERR_CUDA;
-        cached_clusters[dev] = max_clusters;
-    }
-    p.P = max_clusters / p.Kh;
-#ifdef GDN_DECODE_PART
-    p.P = GDN_DECODE_PART;
-#endif
-    if (p.P < 1) p.P = 1;
-    if (p.P > rows) p.P = rows;
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    // persistent grid: one CTA per SM walking (row, q/k head) items round-robin
+    p.nitems = rows * p.Kh;
+    const int grid = p.nitems < nsm ? p.nitems : nsm;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(p.Vh, p.P);
+    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(dec::kThreads);
     cfg.dynamicSmemBytes = dec::SMEM_BYTES;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
     return cuda_status(cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p));
 }
 

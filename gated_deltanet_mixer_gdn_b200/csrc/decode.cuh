@@ -13,27 +13,29 @@
 // both dot products use the old state row, so each row is read and written
 // once.
 //
-// Layout of the work: a persistent CTA owns one value head h and the rows
-// p, p + P, p + 2P, ...  A producer warp streams the state in 32 KiB
-// half-tiles (64 state rows) with bulk copies into a ring of shared-memory
-// stages and writes each updated half-tile back with a bulk store; eight
-// compute warps update a half-tile in shared memory, 8 state rows per warp,
-// a 128-bit load per lane per row, with the 16 dot products of a warp reduced
-// by one transposed shuffle reduction.  The conv / norm / gate prologue of the
-// next row is prefetched into registers while the current row streams.
-//
-// The conv history of the q/k channels is shared by the value heads of one
-// q/k head; those CTAs form one thread-block cluster (same rows), read the
-// history first, and rewrite it only after a cluster barrier, so the in-place
-// shift is safe.
+// Work item = (row, q/k head): the conv of the q/k head's 256 channels and of
+// its value heads' 128-channel slices, the L2 norms and gates, then the states
+// of those value heads.  Every conv-history channel therefore has exactly one
+// reader and writer, and the in-place history shift needs no cross-CTA sync.
+// Persistent CTAs (one per SM) walk items round-robin.  A producer warp
+// streams each state in 32 KiB half-tiles (64 state rows) with bulk copies
+// into a ring of shared-memory stages, running up to a full item ahead; eight
+// compute warps read a half-tile (8 rows per warp, one 128-bit load per lane
+// per row), reduce the 16 dot products of a warp with one transposed shuffle
+// reduction, and write the updated rows straight back to HBM with coalesced
+// 128-bit stores.
 #pragma once
 
 #include "common.cuh"
 
+#ifndef GDN_DECODE_STAGES
+#define GDN_DECODE_STAGES 6
+#endif
+
 namespace gdn {
 
 struct DecodeParams {
-    int Kh, Vh, C, rows, P;
+    int Kh, Vh, C, rows, nitems;
     const uint16_t* qkv;     // bf16 [rows][C]
     const uint16_t* z;       // bf16 [rows][Vh*128]
     const uint16_t* a;       // bf16 [rows][Vh]
@@ -47,23 +49,17 @@ struct DecodeParams {
     uint16_t* out;           // bf16 [rows][Vh*128]
 };
 
-#ifndef GDN_DECODE_STAGES
-#define GDN_DECODE_STAGES 6
-#endif
-#ifndef GDN_DECODE_STORE_LAG
-#define GDN_DECODE_STORE_LAG 1
-#endif
-
 namespace dec {
 constexpr int kStages = GDN_DECODE_STAGES;
-// A stage is refilled once the bulk store issued this many units later has
-// been started, so a store has that long to drain before its stage is reused.
-constexpr int kStoreLag = GDN_DECODE_STORE_LAG;
-constexpr uint32_t kTileBytes = 64 * 128 * 4;  // half of a head's state
+constexpr int kMaxGroup = 8;                     // value heads per q/k head (Vh / Kh)
+constexpr uint32_t kTileBytes = 64 * 128 * 4;   // half of a head's state
 constexpr int kComputeThreads = 256;
 constexpr int kThreads = kComputeThreads + 32;  // + producer warp
+constexpr int kSlots = (2 + kMaxGroup) * 128 / kComputeThreads;  // conv channels per thread (max)
 constexpr uint32_t OFF_MISC = kStages * kTileBytes;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;
+// misc: barriers (256 B), q, k (2 x 512 B), v and o (2 x kMaxGroup x 512 B), reductions, gates
+constexpr uint32_t MISC_BYTES = 256 + 2 * 512 + 2 * kMaxGroup * 512 + 512 + 256;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
 }  // namespace dec
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -103,21 +99,19 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_MISC);
     uint64_t* empty = full + kStages;
-    float* s_q = reinterpret_cast<float*>(smem + OFF_MISC + 128);
+    float* s_q = reinterpret_cast<float*>(smem + OFF_MISC + 256);
     float* s_k = s_q + 128;
-    float* s_v = s_k + 128;
-    float* s_o = s_v + 128;
-    float* s_red = s_o + 128;     // [16]
-    float* s_gate = s_red + 16;   // [4]
+    float* s_v = s_k + 128;                 // [group][128]
+    float* s_o = s_v + kMaxGroup * 128;     // [group][128]
+    float* s_red = s_o + kMaxGroup * 128;   // [128]
+    float* s_gate = s_red + 128;            // [2 * group]
 
-    const int h = blockIdx.x;
-    const int part = blockIdx.y;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int group = p.Vh / p.Kh;
-    const int kap = h / group;
-    const int nrows = (p.rows > part) ? (p.rows - part + p.P - 1) / p.P : 0;
-    const int nunits = 2 * nrows;
+    const int G = p.Vh / p.Kh;
+    const int units_per_item = 2 * G;
+    const int nmine = (p.nitems > (int)blockIdx.x) ? (p.nitems - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    const int nunits = nmine * units_per_item;
     bool broken = false;
 
     if (tid == 0) {
@@ -129,201 +123,145 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     }
     __syncthreads();
 
-    auto tile_src = [&](int u) -> float* {
-        const int row = part + (u >> 1) * p.P;
-        return p.state + (((size_t)row * p.Vh + h) * 128 + (u & 1) * 64) * 128;
+    // unit u of this CTA: item u / (2G), value head (u % 2G) / 2 of its group, half u % 2
+    auto unit_ptr = [&](int u) -> float* {
+        const int it = blockIdx.x + (u / units_per_item) * gridDim.x;
+        const int row = it / p.Kh, kap = it % p.Kh;
+        const int r = u % units_per_item;
+        const int head = kap * G + (r >> 1);
+        return p.state + (((size_t)row * p.Vh + head) * 128 + (r & 1) * 64) * 128;
     };
 
     if (warp == kComputeThreads / 32) {
-        // ---------------- producer warp
+        // ---------------- producer warp: keep the ring of stages full
         if (lane == 0) {
-            for (int u = 0; u < nunits && u < kStages; ++u) {
-                mbar_arrive_expect_tx(&full[u], kTileBytes);
-                bulk_load(smem + u * kTileBytes, tile_src(u), kTileBytes, &full[u]);
+            for (int u = 0; u < nunits; ++u) {
+                const int st = u % kStages;
+                if (u >= kStages) bounded_wait(&empty[st], ((u / kStages) - 1) & 1, broken);
+                mbar_arrive_expect_tx(&full[st], kTileBytes);
+                bulk_load(smem + st * kTileBytes, unit_ptr(u), kTileBytes, &full[st]);
             }
         }
-        for (int j = 0; j < nrows; ++j) {
-            cluster_arrive();
-            if (lane == 0) {
-                for (int half = 0; half < 2; ++half) {
-                    const int u = 2 * j + half;
-                    const int st = u % kStages;
-                    bounded_wait(&empty[st], (u / kStages) & 1, broken);
-                    bulk_store(tile_src(u), smem + st * kTileBytes, kTileBytes);
-                    bulk_commit();
-                    // refill the stage of unit v = u - kStoreLag once its store has read the stage
-                    const int v = u - kStoreLag;
-                    if (v >= 0 && v + kStages < nunits) {
-                        if (kStoreLag == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                        else asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kStoreLag) : "memory");
-                        const int sv = v % kStages;
-                        mbar_arrive_expect_tx(&full[sv], kTileBytes);
-                        bulk_load(smem + sv * kTileBytes, tile_src(v + kStages), kTileBytes, &full[sv]);
-                    }
-                }
-            }
-            __syncwarp();
-            cluster_wait();
-        }
-        if (lane == 0) bulk_wait_all();
         return;
     }
 
     // ---------------- compute warps (tid < 256)
-    // channel slots of this thread: idx = tid (q for tid < 128, k otherwise) and tid + 256 (v, tid < 128)
-    int ch[2];
-    float w[2][4];
-    const int nslots = (tid < 128) ? 2 : 1;
+    const int nch = (2 + G) * 128;  // conv channels of one item: q, k, then G value slices
+    const float w_n = (tid < 128) ? 1.0f + p.norm_w[tid] : 0.f;
+    int u = 0;
+    for (int m = 0; m < nmine; ++m) {
+        const int it = blockIdx.x + m * gridDim.x;
+        const int row = it / p.Kh, kap = it % p.Kh;
+        named_barrier_sync(1, kComputeThreads);  // previous item's readers of s_* are done
+
+        // ---- conv + silu of the item's channels; shift their history in place
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int idx = tid + u * 256;
-        const int grp = idx >> 7, c = idx & 127;
-        ch[u] = (grp == 0) ? kap * 128 + c : (grp == 1) ? p.Kh * 128 + kap * 128 + c : 2 * p.Kh * 128 + h * 128 + c;
-        if (u < nslots) {
-            const uint2 wb = *reinterpret_cast<const uint2*>(p.conv_w + (size_t)ch[u] * 4);
-            w[u][0] = __uint_as_float(wb.x << 16);
-            w[u][1] = __uint_as_float(wb.x & 0xffff0000u);
-            w[u][2] = __uint_as_float(wb.y << 16);
-            w[u][3] = __uint_as_float(wb.y & 0xffff0000u);
+        for (int s = 0; s < kSlots; ++s) {
+            const int idx = tid + s * kComputeThreads;
+            if (idx < nch) {
+                const int grp = idx >> 7, c = idx & 127;
+                const int ch = (grp == 0) ? kap * 128 + c
+                             : (grp == 1) ? p.Kh * 128 + kap * 128 + c
+                                          : 2 * p.Kh * 128 + (kap * G + grp - 2) * 128 + c;
+                float* hr = p.conv + (size_t)row * 3 * p.C + ch;
+                const float h0 = hr[0], h1 = hr[p.C], h2 = hr[2 * p.C];
+                const float x = bf16_bits_to_float(p.qkv[(size_t)row * p.C + ch]);
+                const uint2 wb = *reinterpret_cast<const uint2*>(p.conv_w + (size_t)ch * 4);
+                const float cv = __uint_as_float(wb.x << 16) * h0 + __uint_as_float(wb.x & 0xffff0000u) * h1 +
+                                 __uint_as_float(wb.y << 16) * h2 + __uint_as_float(wb.y & 0xffff0000u) * x;
+                const float act = silu_f(cv);
+                if (grp == 0) s_q[c] = act;
+                else if (grp == 1) s_k[c] = act;
+                else s_v[(grp - 2) * 128 + c] = act;
+                hr[0] = h1;
+                hr[p.C] = h2;
+                hr[2 * p.C] = x;
+            }
         }
-    }
-    const bool hist_writer_qk = (h % group) == 0;
-    const float A_exp = expf(p.A_log[h]);
-    const float dtb = p.dt_bias[h];
-    const float wn = (tid < 128) ? 1.0f + p.norm_w[tid] : 0.f;
-
-    // prefetched inputs of the next row (plain registers: h0/h1/h2/x of the two slots, z, a, b)
-    float h00 = 0.f, h01 = 0.f, h02 = 0.f, x0 = 0.f, h10 = 0.f, h11 = 0.f, h12 = 0.f, x1 = 0.f;
-    float zn = 0.f, an = 0.f, bn = 0.f;
-#define GDN_DECODE_PREFETCH(jj)                                                              \
-    {                                                                                        \
-        const int prow = part + (jj) * p.P;                                                  \
-        const float* hr0 = p.conv + (size_t)prow * 3 * p.C + ch[0];                          \
-        h00 = hr0[0];                                                                        \
-        h01 = hr0[p.C];                                                                      \
-        h02 = hr0[2 * p.C];                                                                  \
-        x0 = bf16_bits_to_float(p.qkv[(size_t)prow * p.C + ch[0]]);                          \
-        if (nslots > 1) {                                                                    \
-            const float* hr1 = p.conv + (size_t)prow * 3 * p.C + ch[1];                      \
-            h10 = hr1[0];                                                                    \
-            h11 = hr1[p.C];                                                                  \
-            h12 = hr1[2 * p.C];                                                              \
-            x1 = bf16_bits_to_float(p.qkv[(size_t)prow * p.C + ch[1]]);                      \
-            zn = bf16_bits_to_float(p.z[(size_t)prow * p.Vh * 128 + h * 128 + tid]);         \
-        }                                                                                    \
-        if (tid == 0) {                                                                      \
-            an = bf16_bits_to_float(p.a[(size_t)prow * p.Vh + h]);                           \
-            bn = bf16_bits_to_float(p.b[(size_t)prow * p.Vh + h]);                           \
-        }                                                                                    \
-    }
-    if (nrows > 0) GDN_DECODE_PREFETCH(0);
-
-    for (int j = 0; j < nrows; ++j) {
-        const int row = part + j * p.P;
-        named_barrier_sync(1, kComputeThreads);  // previous row's readers of s_* are done
-        // ---- conv + silu of this row's channels (history was prefetched)
-        const float act0 = silu_f(w[0][0] * h00 + w[0][1] * h01 + w[0][2] * h02 + w[0][3] * x0);
-        const float act1 = silu_f(w[1][0] * h10 + w[1][1] * h11 + w[1][2] * h12 + w[1][3] * x1);
-        const float k00 = h01, k01 = h02, k02 = x0, k10 = h11, k11 = h12, k12 = x1;  // shifted history
-        const float zval = zn;
-        if (tid == 0) {
-            s_gate[0] = -A_exp * softplus_f(an + dtb);
-            s_gate[1] = sigmoid_f(bn);
+        if (tid < G) {
+            const int head = kap * G + tid;
+            const float av = bf16_bits_to_float(p.a[(size_t)row * p.Vh + head]);
+            const float bv = bf16_bits_to_float(p.b[(size_t)row * p.Vh + head]);
+            s_gate[2 * tid] = expf(-expf(p.A_log[head]) * softplus_f(av + p.dt_bias[head]));  // alpha
+            s_gate[2 * tid + 1] = sigmoid_f(bv);                                                // beta
         }
-        cluster_arrive();  // this CTA has read the row's history
-        if (j + 1 < nrows) GDN_DECODE_PREFETCH(j + 1);
-
+        named_barrier_sync(1, kComputeThreads);
         // ---- L2 norms: q in warps 0-3, k in warps 4-7
         {
-            const float ss = warp_sum(act0 * act0);
+            const float x = (tid < 128) ? s_q[tid] : s_k[tid - 128];
+            const float ss = warp_sum(x * x);
             if (lane == 0) s_red[warp] = ss;
         }
         named_barrier_sync(1, kComputeThreads);
-        {
-            const float qss = s_red[0] + s_red[1] + s_red[2] + s_red[3];
-            const float kss = s_red[4] + s_red[5] + s_red[6] + s_red[7];
-            if (tid < 128) {
-                s_q[tid] = act0 * rsqrtf(qss + kEps) * rsqrtf(128.0f);
-                s_v[tid] = act1;
-            } else {
-                s_k[tid - 128] = act0 * rsqrtf(kss + kEps);
-            }
-        }
-        named_barrier_sync(1, kComputeThreads);
-        const float4 qf = reinterpret_cast<const float4*>(s_q)[lane];
-        const float4 kf = reinterpret_cast<const float4*>(s_k)[lane];
+        const float qscale = rsqrtf(s_red[0] + s_red[1] + s_red[2] + s_red[3] + kEps) * rsqrtf(128.0f);
+        const float kscale = rsqrtf(s_red[4] + s_red[5] + s_red[6] + s_red[7] + kEps);
+        float4 qf = reinterpret_cast<const float4*>(s_q)[lane];
+        float4 kf = reinterpret_cast<const float4*>(s_k)[lane];
+        qf.x *= qscale; qf.y *= qscale; qf.z *= qscale; qf.w *= qscale;
+        kf.x *= kscale; kf.y *= kscale; kf.z *= kscale; kf.w *= kscale;
         const float kq = warp_sum(kf.x * qf.x + kf.y * qf.y + kf.z * qf.z + kf.w * qf.w);
-        const float alpha = expf(s_gate[0]);
-        const float beta = s_gate[1];
 
-        // ---- stream the two half-tiles of the state
+        // ---- stream the G value heads' states, two half-tiles each
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            const int u = 2 * j + half;
-            const int st = u % kStages;
-            bounded_wait(&full[st], (u / kStages) & 1, broken);
-            float* tile = reinterpret_cast<float*>(smem + st * kTileBytes);
-            float4 s[8];
+        for (int hh = 0; hh < G; ++hh) {
+            const float alpha = s_gate[2 * hh], beta = s_gate[2 * hh + 1];
+            const float* sv = s_v + hh * 128;
+            float* so = s_o + hh * 128;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half, ++u) {
+                const int st = u % kStages;
+                bounded_wait(&full[st], (u / kStages) & 1, broken);
+                const float* tile = reinterpret_cast<const float*>(smem + st * kTileBytes);
+                float4 s[8];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) s[r] = reinterpret_cast<const float4*>(tile + (warp * 8 + r) * 128)[lane];
-            float vals[16];
+                for (int r = 0; r < 8; ++r) s[r] = reinterpret_cast<const float4*>(tile + (warp * 8 + r) * 128)[lane];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done reading the stage
+                float vals[16];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                vals[2 * r] = s[r].x * kf.x + s[r].y * kf.y + s[r].z * kf.z + s[r].w * kf.w;
-                vals[2 * r + 1] = s[r].x * qf.x + s[r].y * qf.y + s[r].z * qf.z + s[r].w * qf.w;
+                for (int r = 0; r < 8; ++r) {
+                    vals[2 * r] = s[r].x * kf.x + s[r].y * kf.y + s[r].z * kf.z + s[r].w * kf.w;
+                    vals[2 * r + 1] = s[r].x * qf.x + s[r].y * qf.y + s[r].z * qf.z + s[r].w * qf.w;
+                }
+                // lane l: row l >> 2 of the warp's 8, S.k if bit 1 of l is clear, else S.q
+                const float tot = warp_transpose_sum16(vals, lane);
+                const int irow = half * 64 + warp * 8 + (lane >> 2);
+                const float u_k = beta * (sv[irow] - alpha * tot);  // meaningful on lanes 4r, 4r+1
+                const float u_r = __shfl_sync(0xffffffffu, u_k, lane & ~3);
+                if ((lane & 3) == 2) so[irow] = alpha * tot + u_r * kq;
+                float* gdst = unit_ptr(u) + (warp * 8) * 128;
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const float ur = __shfl_sync(0xffffffffu, u_k, 4 * r);
+                    float4 n;
+                    n.x = alpha * s[r].x + ur * kf.x;
+                    n.y = alpha * s[r].y + ur * kf.y;
+                    n.z = alpha * s[r].z + ur * kf.z;
+                    n.w = alpha * s[r].w + ur * kf.w;
+                    __stcs(reinterpret_cast<float4*>(gdst + r * 128) + lane, n);
+                }
             }
-            const float tot = warp_transpose_sum16(vals, lane);  // lane l: row l>>2, S.k if bit 1 clear else S.q
-            const int rr = lane >> 2;
-            const int irow = half * 64 + warp * 8 + rr;
-            const float u_k = beta * (s_v[irow] - alpha * tot);      // meaningful on lanes 4r, 4r+1
-            const float u_r = __shfl_sync(0xffffffffu, u_k, lane & ~3);
-            if ((lane & 3) == 2) s_o[irow] = alpha * tot + u_r * kq;
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const float ur = __shfl_sync(0xffffffffu, u_k, 4 * r);
-                float4 n;
-                n.x = alpha * s[r].x + ur * kf.x;
-                n.y = alpha * s[r].y + ur * kf.y;
-                n.z = alpha * s[r].z + ur * kf.z;
-                n.w = alpha * s[r].w + ur * kf.w;
-                reinterpret_cast<float4*>(tile + (warp * 8 + r) * 128)[lane] = n;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
         }
 
-        // ---- gated RMSNorm over the head's 128 outputs
+        // ---- gated RMSNorm of the G heads' 128 outputs each
         named_barrier_sync(1, kComputeThreads);
-        {
-            const float o = (tid < 128) ? s_o[tid] : 0.f;
+        for (int hh = 0; hh < G; ++hh) {
+            const float o = (tid < 128) ? s_o[hh * 128 + tid] : 0.f;
             const float ss = warp_sum(o * o);
-            if (lane == 0) s_red[8 + warp] = ss;
+            if (lane == 0) s_red[8 + hh * 8 + warp] = ss;
         }
         named_barrier_sync(1, kComputeThreads);
         if (tid < 128) {
-            const float ms = (s_red[8] + s_red[9] + s_red[10] + s_red[11]) * (1.0f / 128.0f);
-            const float y = s_o[tid] * rsqrtf(ms + kEps) * wn * silu_f(zval);
-            p.out[(size_t)row * p.Vh * 128 + h * 128 + tid] = float_to_bf16_bits(y);
-        }
-
-        // ---- history shift, after every CTA of the cluster has read the old values
-        cluster_wait();
-        if (hist_writer_qk) {  // slot 0: a q/k channel shared by the cluster
-            float* hr = p.conv + (size_t)row * 3 * p.C + ch[0];
-            hr[0] = k00;
-            hr[p.C] = k01;
-            hr[2 * p.C] = k02;
-        }
-        if (nslots > 1) {  // slot 1: a v channel of this head
-            float* hr = p.conv + (size_t)row * 3 * p.C + ch[1];
-            hr[0] = k10;
-            hr[p.C] = k11;
-            hr[2 * p.C] = k12;
+            for (int hh = 0; hh < G; ++hh) {
+                const float* r4 = s_red + 8 + hh * 8;
+                const float ms = (r4[0] + r4[1] + r4[2] + r4[3]) * (1.0f / 128.0f);
+                const int head = kap * G + hh;
+                const float zv = bf16_bits_to_float(p.z[(size_t)row * p.Vh * 128 + head * 128 + tid]);
+                const float y = s_o[hh * 128 + tid] * rsqrtf(ms + kEps) * w_n * silu_f(zv);
+                p.out[(size_t)row * p.Vh * 128 + head * 128 + tid] = float_to_bf16_bits(y);
+            }
         }
     }
 }
-
-#undef GDN_DECODE_PREFETCH
 
 }  // namespace gdn
