@@ -344,9 +344,10 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
     static cudaError_t dec_err = cudaSuccess;
     std::call_once(dec_once, [] {
         dec_err = cudaFuncSetAttribute(gdn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)dec::SMEM_BYTES);
+                                       (int)dec::kSmemLimit);
     });
     if (dec_err != cudaSuccess) return GDN_ERR_CUDA;
+    const dec::Plan dplan = dec::plan(p.Vh / p.Kh);
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -357,7 +358,7 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(dec::kThreads);
-    cfg.dynamicSmemBytes = dec::SMEM_BYTES;
+    cfg.dynamicSmemBytes = dplan.smem_bytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;

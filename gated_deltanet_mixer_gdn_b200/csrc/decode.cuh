@@ -29,7 +29,7 @@
 #include "common.cuh"
 
 #ifndef GDN_DECODE_STAGES
-#define GDN_DECODE_STAGES 6
+#define GDN_DECODE_STAGES 5
 #endif
 
 namespace gdn {
@@ -50,16 +50,40 @@ struct DecodeParams {
 };
 
 namespace dec {
-constexpr int kStages = GDN_DECODE_STAGES;
+constexpr int kMaxStages = GDN_DECODE_STAGES;
 constexpr int kMaxGroup = 8;                     // value heads per q/k head (Vh / Kh)
 constexpr uint32_t kTileBytes = 64 * 128 * 4;   // half of a head's state
 constexpr int kComputeThreads = 256;
 constexpr int kThreads = kComputeThreads + 32;  // + producer warp
 constexpr int kSlots = (2 + kMaxGroup) * 128 / kComputeThreads;  // conv channels per thread (max)
-constexpr uint32_t OFF_MISC = kStages * kTileBytes;
+constexpr uint32_t kSmemLimit = 232448;         // opt-in shared memory per block on sm_100
 // misc: barriers (256 B), q, k (2 x 512 B), v and o (2 x kMaxGroup x 512 B), reductions, gates
 constexpr uint32_t MISC_BYTES = 256 + 2 * 512 + 2 * kMaxGroup * 512 + 512 + 256;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
+
+// Shared-memory plan for a group size G: a ring of half-tile stages, then two
+// buffers of per-item inputs, bulk-copied one item ahead (history
+// [3][(2+G)*128] f32, new qkv [(2+G)*128] bf16, conv taps [(2+G)*128][4] bf16,
+// z [G*128] bf16), then small scratch.
+struct Plan {
+    int stages;
+    uint32_t aux_x, aux_w, aux_z, aux_bytes, aux_load_bytes, off_aux, off_misc, smem_bytes;
+};
+__host__ __device__ inline Plan plan(int G) {
+    Plan pl{};
+    const uint32_t nch = (2 + G) * 128;
+    pl.aux_x = 3 * nch * 4;
+    pl.aux_w = pl.aux_x + nch * 2;
+    pl.aux_z = pl.aux_w + nch * 8;
+    pl.aux_load_bytes = pl.aux_z + G * 256;
+    pl.aux_bytes = (pl.aux_load_bytes + 127) / 128 * 128;
+    const uint32_t rest = 2 * pl.aux_bytes + MISC_BYTES + 1024;
+    int st = (int)((kSmemLimit - rest) / kTileBytes);
+    pl.stages = st > kMaxStages ? kMaxStages : st;
+    pl.off_aux = pl.stages * kTileBytes;
+    pl.off_misc = pl.off_aux + 2 * pl.aux_bytes;
+    pl.smem_bytes = pl.off_misc + MISC_BYTES + 1024;
+    return pl;
+}
 }  // namespace dec
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -97,9 +121,14 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_MISC);
-    uint64_t* empty = full + kStages;
-    float* s_q = reinterpret_cast<float*>(smem + OFF_MISC + 256);
+    const int G = p.Vh / p.Kh;
+    const Plan pl = plan(G);
+    const int nst = pl.stages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.off_misc);
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* auxfull = empty + kMaxStages;
+    uint64_t* auxempty = auxfull + 2;
+    float* s_q = reinterpret_cast<float*>(smem + pl.off_misc + 256);
     float* s_k = s_q + 128;
     float* s_v = s_k + 128;                 // [group][128]
     float* s_o = s_v + kMaxGroup * 128;     // [group][128]
@@ -108,16 +137,20 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int G = p.Vh / p.Kh;
+    const int nch = (2 + G) * 128;  // conv channels of one item: q, k, then G value slices
     const int units_per_item = 2 * G;
     const int nmine = (p.nitems > (int)blockIdx.x) ? (p.nitems - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     const int nunits = nmine * units_per_item;
     bool broken = false;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < nst; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kComputeThreads / 32);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&auxfull[s], 1);
+            mbar_init(&auxempty[s], kComputeThreads / 32);
         }
         fence_barrier_init();
     }
@@ -133,11 +166,45 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     };
 
     if (warp == kComputeThreads / 32) {
-        // ---------------- producer warp: keep the ring of stages full
+        // ---------------- producer warp: per-item inputs one item ahead, state half-tiles in a ring
         if (lane == 0) {
+            auto aux_load = [&](int m) {
+                const int it = blockIdx.x + m * gridDim.x;
+                const int row = it / p.Kh, kap = it % p.Kh;
+                uint8_t* ax = smem + pl.off_aux + (m & 1) * pl.aux_bytes;
+                uint64_t* bar = &auxfull[m & 1];
+                mbar_arrive_expect_tx(bar, pl.aux_load_bytes);
+                const int chq = kap * 128, chk = p.Kh * 128 + kap * 128, chv = 2 * p.Kh * 128 + kap * G * 128;
+                for (int r = 0; r < 3; ++r) {
+                    const float* hrow = p.conv + ((size_t)row * 3 + r) * p.C;
+                    float* dst = reinterpret_cast<float*>(ax) + r * nch;
+                    bulk_load(dst, hrow + chq, 512, bar);
+                    bulk_load(dst + 128, hrow + chk, 512, bar);
+                    bulk_load(dst + 256, hrow + chv, G * 512, bar);
+                }
+                const uint16_t* xrow = p.qkv + (size_t)row * p.C;
+                uint16_t* dx = reinterpret_cast<uint16_t*>(ax + pl.aux_x);
+                bulk_load(dx, xrow + chq, 256, bar);
+                bulk_load(dx + 128, xrow + chk, 256, bar);
+                bulk_load(dx + 256, xrow + chv, G * 256, bar);
+                uint16_t* dw = reinterpret_cast<uint16_t*>(ax + pl.aux_w);
+                bulk_load(dw, p.conv_w + (size_t)chq * 4, 1024, bar);
+                bulk_load(dw + 512, p.conv_w + (size_t)chk * 4, 1024, bar);
+                bulk_load(dw + 1024, p.conv_w + (size_t)chv * 4, G * 1024, bar);
+                bulk_load(ax + pl.aux_z, p.z + ((size_t)row * p.Vh + kap * G) * 128, G * 256, bar);
+            };
+            // the next item's inputs are requested once the ring holds this item's first stages,
+            // by which time the item two back has released their buffer
+            const int lead = nst < units_per_item - 1 ? nst : units_per_item - 1;
+            if (nmine > 0) aux_load(0);
             for (int u = 0; u < nunits; ++u) {
-                const int st = u % kStages;
-                if (u >= kStages) bounded_wait(&empty[st], ((u / kStages) - 1) & 1, broken);
+                const int m = u / units_per_item, r = u % units_per_item;
+                if (r == lead && m + 1 < nmine) {
+                    if (m >= 1) bounded_wait(&auxempty[(m + 1) & 1], ((m - 1) >> 1) & 1, broken);
+                    aux_load(m + 1);
+                }
+                const int st = u % nst;
+                if (u >= nst) bounded_wait(&empty[st], ((u / nst) - 1) & 1, broken);
                 mbar_arrive_expect_tx(&full[st], kTileBytes);
                 bulk_load(smem + st * kTileBytes, unit_ptr(u), kTileBytes, &full[st]);
             }
@@ -146,15 +213,30 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     }
 
     // ---------------- compute warps (tid < 256)
-    const int nch = (2 + G) * 128;  // conv channels of one item: q, k, then G value slices
     const float w_n = (tid < 128) ? 1.0f + p.norm_w[tid] : 0.f;
+    // gate inputs of the next item, loaded one item ahead (threads tid < G)
+    float ga = 0.f, gb = 0.f, gA = 0.f, gdt = 0.f;
+    auto gate_prefetch = [&](int m) {
+        const int it = blockIdx.x + m * gridDim.x;
+        const int row = it / p.Kh, head = (it % p.Kh) * G + tid;
+        ga = bf16_bits_to_float(p.a[(size_t)row * p.Vh + head]);
+        gb = bf16_bits_to_float(p.b[(size_t)row * p.Vh + head]);
+        gA = p.A_log[head];
+        gdt = p.dt_bias[head];
+    };
+    if (tid < G && nmine > 0) gate_prefetch(0);
     int u = 0;
     for (int m = 0; m < nmine; ++m) {
         const int it = blockIdx.x + m * gridDim.x;
         const int row = it / p.Kh, kap = it % p.Kh;
+        const uint8_t* ax = smem + pl.off_aux + (m & 1) * pl.aux_bytes;
         named_barrier_sync(1, kComputeThreads);  // previous item's readers of s_* are done
+        bounded_wait(&auxfull[m & 1], (m >> 1) & 1, broken);
 
         // ---- conv + silu of the item's channels; shift their history in place
+        const float* ah = reinterpret_cast<const float*>(ax);
+        const uint16_t* axx = reinterpret_cast<const uint16_t*>(ax + pl.aux_x);
+        const uint2* aw = reinterpret_cast<const uint2*>(ax + pl.aux_w);
 #pragma unroll
         for (int s = 0; s < kSlots; ++s) {
             const int idx = tid + s * kComputeThreads;
@@ -163,27 +245,25 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 const int ch = (grp == 0) ? kap * 128 + c
                              : (grp == 1) ? p.Kh * 128 + kap * 128 + c
                                           : 2 * p.Kh * 128 + (kap * G + grp - 2) * 128 + c;
-                float* hr = p.conv + (size_t)row * 3 * p.C + ch;
-                const float h0 = hr[0], h1 = hr[p.C], h2 = hr[2 * p.C];
-                const float x = bf16_bits_to_float(p.qkv[(size_t)row * p.C + ch]);
-                const uint2 wb = *reinterpret_cast<const uint2*>(p.conv_w + (size_t)ch * 4);
+                const float h0 = ah[idx], h1 = ah[nch + idx], h2 = ah[2 * nch + idx];
+                const float x = bf16_bits_to_float(axx[idx]);
+                const uint2 wb = aw[idx];
                 const float cv = __uint_as_float(wb.x << 16) * h0 + __uint_as_float(wb.x & 0xffff0000u) * h1 +
                                  __uint_as_float(wb.y << 16) * h2 + __uint_as_float(wb.y & 0xffff0000u) * x;
                 const float act = silu_f(cv);
                 if (grp == 0) s_q[c] = act;
                 else if (grp == 1) s_k[c] = act;
                 else s_v[(grp - 2) * 128 + c] = act;
+                float* hr = p.conv + (size_t)row * 3 * p.C + ch;
                 hr[0] = h1;
                 hr[p.C] = h2;
                 hr[2 * p.C] = x;
             }
         }
         if (tid < G) {
-            const int head = kap * G + tid;
-            const float av = bf16_bits_to_float(p.a[(size_t)row * p.Vh + head]);
-            const float bv = bf16_bits_to_float(p.b[(size_t)row * p.Vh + head]);
-            s_gate[2 * tid] = expf(-expf(p.A_log[head]) * softplus_f(av + p.dt_bias[head]));  // alpha
-            s_gate[2 * tid + 1] = sigmoid_f(bv);                                                // beta
+            s_gate[2 * tid] = expf(-expf(gA) * softplus_f(ga + gdt));  // alpha
+            s_gate[2 * tid + 1] = sigmoid_f(gb);                        // beta
+            if (m + 1 < nmine) gate_prefetch(m + 1);
         }
         named_barrier_sync(1, kComputeThreads);
         // ---- L2 norms: q in warps 0-3, k in warps 4-7
@@ -209,8 +289,8 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
             float* so = s_o + hh * 128;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half, ++u) {
-                const int st = u % kStages;
-                bounded_wait(&full[st], (u / kStages) & 1, broken);
+                const int st = u % nst;
+                bounded_wait(&full[st], (u / nst) & 1, broken);
                 const float* tile = reinterpret_cast<const float*>(smem + st * kTileBytes);
                 float4 s[8];
 #pragma unroll
@@ -252,15 +332,18 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         }
         named_barrier_sync(1, kComputeThreads);
         if (tid < 128) {
+            const uint16_t* az = reinterpret_cast<const uint16_t*>(ax + pl.aux_z);
             for (int hh = 0; hh < G; ++hh) {
                 const float* r4 = s_red + 8 + hh * 8;
                 const float ms = (r4[0] + r4[1] + r4[2] + r4[3]) * (1.0f / 128.0f);
                 const int head = kap * G + hh;
-                const float zv = bf16_bits_to_float(p.z[(size_t)row * p.Vh * 128 + head * 128 + tid]);
+                const float zv = bf16_bits_to_float(az[hh * 128 + tid]);
                 const float y = s_o[hh * 128 + tid] * rsqrtf(ms + kEps) * w_n * silu_f(zv);
                 p.out[(size_t)row * p.Vh * 128 + head * 128 + tid] = float_to_bf16_bits(y);
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&auxempty[m & 1]);  // this warp is done with the item's inputs
     }
 }
 
