@@ -71,7 +71,7 @@ constexpr uint32_t OFF_M = 212992;     // tril(Q K^T) * E f16 [64][64]
 constexpr uint32_t OFF_A = OFF_LO;     // A, then T, f32 [64][LDA]
 constexpr uint32_t OFF_Z = OFF_WT;
 constexpr uint32_t OFF_MISC = 221184;
-constexpr uint32_t MISC_BYTES = 2048;
+constexpr uint32_t MISC_BYTES = 3072;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(64 * LDA * 4 <= 32768, "A/T must fit in the residual tile");
 // TMEM columns (f32, 128 lanes)
@@ -86,11 +86,76 @@ constexpr uint32_t ID_NEG_BMN = idesc_f16_f32(128, 64, false, true, true);
 constexpr uint32_t ID_DS = idesc_f16_f32(128, 128, false, true, false);
 }  // namespace chunk
 
+// ---- warp-level TF32 tensor-core products for the triangular solve.
+// x = hi + lo with hi, lo representable in tf32; hi*hi + hi*lo + lo*hi
+// recovers an f32-accurate product (the lo*lo term is below f32 rounding).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// acc[nt] (a 16 x 8 tile each) += A[16 x 8*KT] * B[8*KT x 8*NT]; A, B f32 in
+// shared memory (row-major, strides lda / ldb); D fragment layout of m16n8.
+template <int NT, int KT>
+__device__ __forceinline__ void warp_gemm_tf32x3(float (&acc)[NT][4], const float* A, int lda, const float* B, int ldb,
+                                                 int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kt = 0; kt < KT; ++kt) {
+        const float af[4] = {A[g * lda + kt * 8 + t], A[(g + 8) * lda + kt * 8 + t], A[g * lda + kt * 8 + t + 4],
+                             A[(g + 8) * lda + kt * 8 + t + 4]};
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            ah[i] = to_tf32(af[i]);
+            al[i] = to_tf32(af[i] - __uint_as_float(ah[i]));
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float bf[2] = {B[(kt * 8 + t) * ldb + nt * 8 + g], B[(kt * 8 + t + 4) * ldb + nt * 8 + g]};
+            uint32_t bh[2], bl[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                bh[i] = to_tf32(bf[i]);
+                bl[i] = to_tf32(bf[i] - __uint_as_float(bh[i]));
+            }
+            mma_tf32(acc[nt], al, bh);
+            mma_tf32(acc[nt], ah, bl);
+            mma_tf32(acc[nt], ah, bh);
+        }
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void warp_store_tile(float* D, int ldd, const float (&acc)[NT][4], float scale, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        D[g * ldd + nt * 8 + 2 * t] = scale * acc[nt][0];
+        D[g * ldd + nt * 8 + 2 * t + 1] = scale * acc[nt][1];
+        D[(g + 8) * ldd + nt * 8 + 2 * t] = scale * acc[nt][2];
+        D[(g + 8) * ldd + nt * 8 + 2 * t + 1] = scale * acc[nt][3];
+    }
+}
+
 // (I + A)^-1 of a unit lower-triangular 64 x 64 system, in place in sA (row
-// stride LDA): 16 x 16 diagonal blocks by forward substitution, then block
-// rows 1..3 as T_i,<i = -T_ii (sum_m A_im T_m,<i).  Uses sP (16 x 48 f32).
+// stride LDA).  The four 16 x 16 diagonal blocks are inverted by forward
+// substitution on the CUDA cores; the off-diagonal blocks follow from the
+// block inverse [[Ta, 0], [Y, Tb]] with Y = -Tb * L_ba * Ta, first for the
+// 16-blocks (1,0) and (3,2), then for the 32-block (1,0), on the tensor cores
+// (f32-accurate TF32 products).  sP: 4 KiB of f32 scratch.
 __device__ __forceinline__ void chunk_tsolve(float* sA, float* sP, int tid) {
     using namespace chunk;
+    const int warp = tid >> 5, lane = tid & 31;
     float x[16];
     const int b = tid >> 4, c = tid & 15;
     if (tid < 64) {
@@ -110,26 +175,34 @@ __device__ __forceinline__ void chunk_tsolve(float* sA, float* sP, int tid) {
         for (int r = 0; r < 16; ++r) Ab[r * LDA + c] = x[r];
     }
     __syncthreads();
-    for (int i = 1; i < 4; ++i) {
-        const int ncol = 16 * i;
-        const int nout = 16 * ncol;
-        for (int o = tid; o < nout; o += kThreads) {
-            const int r = o / ncol, cc = o % ncol;
-            const float* Ar = sA + (16 * i + r) * LDA;
-            float s = 0.f;
-            for (int m = cc; m < ncol; ++m) s = fmaf(Ar[m], sA[m * LDA + cc], s);
-            sP[r * 48 + cc] = s;
-        }
-        __syncthreads();
-        for (int o = tid; o < nout; o += kThreads) {
-            const int r = o / ncol, cc = o % ncol;
-            const float* Tr = sA + (16 * i + r) * LDA + 16 * i;
-            float s = 0.f;
-            for (int m = 0; m <= r; ++m) s = fmaf(Tr[m], sP[m * 48 + cc], s);
-            sA[(16 * i + r) * LDA + cc] = -s;
-        }
-        __syncthreads();
+    // 16-block merges: warp 0 -> block (1,0), warp 1 -> block (3,2)
+    if (warp < 2) {
+        const int bb = 2 * warp;                 // upper-left block index of the pair
+        float* X = sP + warp * 16 * 20;          // 16 x 16 scratch, stride 20
+        float acc[2][4] = {};
+        warp_gemm_tf32x3<2, 2>(acc, sA + (16 * (bb + 1)) * LDA + 16 * bb, LDA, sA + (16 * bb) * LDA + 16 * bb, LDA,
+                               lane);
+        warp_store_tile<2>(X, 20, acc, 1.f, lane);
+        __syncwarp();
+        float acc2[2][4] = {};
+        warp_gemm_tf32x3<2, 2>(acc2, sA + (16 * (bb + 1)) * LDA + 16 * (bb + 1), LDA, X, 20, lane);
+        warp_store_tile<2>(sA + (16 * (bb + 1)) * LDA + 16 * bb, LDA, acc2, -1.f, lane);
     }
+    __syncthreads();
+    // 32-block merge: warps 0-3, one 16 x 16 quadrant each
+    if (warp < 4) {
+        const int mi = warp >> 1, ni = warp & 1;
+        float* X = sP;  // 32 x 32 scratch, stride 36
+        float acc[2][4] = {};
+        warp_gemm_tf32x3<2, 4>(acc, sA + (32 + 16 * mi) * LDA, LDA, sA + 16 * ni, LDA, lane);
+        warp_store_tile<2>(X + (16 * mi) * 36 + 16 * ni, 36, acc, 1.f, lane);
+        named_barrier_sync(2, 128);
+        float acc2[2][4] = {};
+        warp_gemm_tf32x3<2, 4>(acc2, sA + (32 + 16 * mi) * LDA + 32, LDA, X + 16 * ni, 36, lane);
+        named_barrier_sync(2, 128);  // every quadrant of X is read before L_ba is overwritten
+        warp_store_tile<2>(sA + (32 + 16 * mi) * LDA + 16 * ni, LDA, acc2, -1.f, lane);
+    }
+    __syncthreads();
 }
 
 // Lane l of the warp ends with sum over the 32 lanes of v[l] (31 shuffles).
@@ -199,6 +272,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     float* s_eG = s_G + 64;                                            // [64]
     float* s_beta = s_G + 128;                                         // [64]
     float* s_red = reinterpret_cast<float*>(smem + OFF_MISC + 1024);  // [4][64]
+    float* s_rstd = reinterpret_cast<float*>(smem + OFF_MISC + 2048); // [64]
     float* sA = reinterpret_cast<float*>(smem + OFF_A);
     float* sP = reinterpret_cast<float*>(smem + OFF_UT);
 
@@ -264,6 +338,12 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
     const float wn = 1.0f + __ldg(p.norm_w + row);  // (1 + w) of this thread's v channel
     bool failed = false;
+    // gate inputs of the next chunk, loaded one chunk ahead (threads tid < 64)
+    float g_next = 0.f, b_next = 0.f;
+    if (tid < 64 && nchunks > 0 && tid < min(C, len)) {
+        g_next = __ldg(p.Gs + (size_t)h * p.total + start + tid);
+        b_next = __ldg(p.Bs + (size_t)h * p.total + start + tid);
+    }
     uint32_t mma_phase = 0;
 
     for (int c = 0; c < nchunks; ++c) {
@@ -274,8 +354,10 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
         // ---- gates of the chunk: G = inclusive cumsum of g, e^G, beta
         if (tid < 64) {
-            const float g = (tid < nv) ? __ldg(p.Gs + (size_t)h * p.total + tok0 + tid) : 0.f;
-            const float bt = (tid < nv) ? __ldg(p.Bs + (size_t)h * p.total + tok0 + tid) : 0.f;
+            const float g = g_next, bt = b_next;
+            const int nv1 = min(C, len - (c + 1) * C);  // tokens of the next chunk (<= 0: none)
+            g_next = (tid < nv1) ? __ldg(p.Gs + (size_t)h * p.total + tok0 + C + tid) : 0.f;
+            b_next = (tid < nv1) ? __ldg(p.Bs + (size_t)h * p.total + tok0 + C + tid) : 0.f;
             float x = g;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -521,13 +603,17 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             const float part = warp_transpose_sum(sq, lane);
             s_red[q4 * 64 + 32 * hf + lane] = part;
             __syncthreads();
+            if (tid < 64) {
+                const float ms = (s_red[tid] + s_red[64 + tid] + s_red[128 + tid] + s_red[192 + tid]) * (1.0f / 128.0f);
+                s_rstd[tid] = rsqrtf(ms + kEps);
+            }
+            __syncthreads();
             uint16_t* zt = reinterpret_cast<uint16_t*>(smem + OFF_Z);
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
                 const int t = 32 * hf + jj;
-                const float ms = (s_red[t] + s_red[64 + t] + s_red[128 + t] + s_red[192 + t]) * (1.0f / 128.0f);
                 const float zv = bf16_bits_to_float(zt[t * 128 + row]);
-                const float y = o[jj] * rsqrtf(ms + kEps) * wn * silu_f(zv);
+                const float y = o[jj] * s_rstd[t] * wn * silu_f(zv);
                 zt[t * 128 + row] = float_to_bf16_bits(y);
             }
         }

@@ -226,7 +226,8 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
     return *reinterpret_cast<uint16_t*>(&h);
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// silu(x) = x * sigmoid(x); fast reciprocal (x / inf -> 0 for very negative x).
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x))); }
 

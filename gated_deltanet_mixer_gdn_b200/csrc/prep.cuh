@@ -69,7 +69,7 @@ struct PrepParams {
     float* Bs;
 };
 
-constexpr int kPrepTokens = 16;
+constexpr int kPrepTokens = 8;  // tokens per thread; the 3 rows before them are read too
 
 __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     const int tid = threadIdx.x;
@@ -84,7 +84,18 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     const bool is_q = slot < p.Kh;
     const bool is_v = slot >= 2 * p.Kh;
     const int vh = slot - 2 * p.Kh;
+    const int t_begin = blockIdx.x * kPrepTokens;
 
+    // Issue all loads first: the window of kPrepTokens + 3 input rows of this
+    // thread's 8 channels (16 bytes each), then the conv taps.
+    uint4 win[kPrepTokens + 3];
+#pragma unroll
+    for (int r = 0; r < kPrepTokens + 3; ++r) {
+        const int t = t_begin - 3 + r;
+        win[r] = (t >= 0 && t < p.total)
+                     ? __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)t * p.C + ch0))
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
     // conv taps of the 8 channels: w[e][j] at conv_w[(ch0+e)*4 + j]
     float w[8][4];
     {
@@ -108,7 +119,7 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
         gdt = __ldg(p.dt_bias + vh);
     }
 
-    const int t_begin = blockIdx.x * kPrepTokens;
+#pragma unroll
     for (int tt = 0; tt < kPrepTokens; ++tt) {
         const int t = t_begin + tt;
         if (t >= p.total) break;
@@ -123,7 +134,7 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
             const int xi = s + j;  // index into [history (3 rows); tokens of the row]
             float x[8];
             if (xi >= 3) {
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)(t + j - 3) * p.C + ch0));
+                const uint4 v = win[tt + j];
                 const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
