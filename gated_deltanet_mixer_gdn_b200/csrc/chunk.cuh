@@ -51,7 +51,7 @@ struct ChunkParams {
 
 namespace chunk {
 constexpr int C = 64;              // tokens per chunk
-constexpr int kPThreads = 128;     // prologue warpgroup
+constexpr int kPThreads = 256;     // prologue warpgroups
 constexpr int kSThreads = 256;     // state warpgroups
 constexpr int kThreads = kPThreads + kSThreads;
 constexpr int LDA = 68;            // f32 row stride of the A / T matrix (conflict-free float4 rows)
@@ -150,7 +150,7 @@ __device__ __forceinline__ void warp_store_tile(float* D, int ldd, const float (
 }
 
 // (I + A)^-1 of a unit lower-triangular 64 x 64 system, in place in sA (row
-// stride LDA), by the 128 threads of the prologue warpgroup (named barrier 1).
+// stride LDA), by the threads of the prologue warpgroups (named barrier 1).
 // The four 16 x 16 diagonal blocks are inverted by forward substitution on the
 // CUDA cores; the off-diagonal blocks follow from the block inverse
 // [[Ta, 0], [Y, Tb]] with Y = -Tb * L_ba * Ta, first for the 16-blocks (1,0)
@@ -192,14 +192,16 @@ __device__ __forceinline__ void chunk_tsolve(float* sA, float* sP, int p) {
         warp_store_tile<2>(sA + (16 * (bb + 1)) * LDA + 16 * bb, LDA, acc2, -1.f, lane);
     }
     named_barrier_sync(1, kPThreads);
-    // 32-block merge: one 16 x 16 quadrant per warp
-    {
-        const int mi = warp >> 1, ni = warp & 1;
-        float* X = sP;  // 32 x 32 scratch, stride 36
+    // 32-block merge: one 16 x 16 quadrant per warp (warps 0-3)
+    const int mi = (warp >> 1) & 1, ni = warp & 1;
+    float* X = sP;  // 32 x 32 scratch, stride 36
+    if (warp < 4) {
         float acc[2][4] = {};
         warp_gemm_tf32x3<2, 4>(acc, sA + (32 + 16 * mi) * LDA, LDA, sA + 16 * ni, LDA, lane);
         warp_store_tile<2>(X + (16 * mi) * 36 + 16 * ni, 36, acc, 1.f, lane);
-        named_barrier_sync(1, kPThreads);  // X complete; every read of L_ba is done
+    }
+    named_barrier_sync(1, kPThreads);  // X complete; every read of L_ba is done
+    if (warp < 4) {
         float acc2[2][4] = {};
         warp_gemm_tf32x3<2, 4>(acc2, sA + (32 + 16 * mi) * LDA + 32, LDA, X + 16 * ni, 36, lane);
         warp_store_tile<2>(sA + (32 + 16 * mi) * LDA + 16 * ni, LDA, acc2, -1.f, lane);
@@ -316,10 +318,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         __syncwarp();
     };
 
-    if (warp < 4) {
-        // =================================================================== prologue warpgroup
-        const int pt = tid;  // TMEM lane / matrix row of this thread
-        const uint32_t tlane = tbase + (static_cast<uint32_t>(32 * warp) << 16);
+    if (warp < kPThreads / 32) {
+        // =================================================================== prologue warpgroups
+        const int pt = tid;
+        const int pq = warp & 3;             // TMEM lane quarter
+        const int phf = warp >> 2;           // column half
+        const int prow = 32 * pq + lane;     // TMEM lane / matrix row of this thread
+        const uint32_t tlane = tbase + (static_cast<uint32_t>(32 * pq) << 16);
         float g_next = 0.f, b_next = 0.f;
         if (pt < 64 && nchunks > 0 && pt < min(C, len)) {
             g_next = __ldg(p.Gs + (size_t)h * p.total + start + pt);
@@ -400,34 +405,33 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             tc_fence_after();
 
             // ---- A (rows of K K^T) and M (rows of Q K^T), masked before the exp
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            {
                 float v[32];
-                tmem_ld32(tlane + T_KQ + 32 * half, v);
+                tmem_ld32(tlane + T_KQ + 32 * phf, v);
                 tmem_ld_wait();
-                if (pt < 64) {
-                    const int i = pt;
-                    const float bi = s_beta[i];
+                if (prow < 64) {
+                    const int i = prow;
+                    const float bi = s_beta[i], Gr = G[i];
                     float a[32];
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
-                        const int j = 32 * half + jj;
-                        a[jj] = (j < i) ? bi * __expf(Gi - G[j]) * v[jj] : 0.f;
+                        const int j = 32 * phf + jj;
+                        a[jj] = (j < i) ? bi * __expf(Gr - G[j]) * v[jj] : 0.f;
                     }
-                    float4* dst = reinterpret_cast<float4*>(sA + i * LDA + 32 * half);
+                    float4* dst = reinterpret_cast<float4*>(sA + i * LDA + 32 * phf);
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4)
                         dst[j4] = make_float4(a[4 * j4], a[4 * j4 + 1], a[4 * j4 + 2], a[4 * j4 + 3]);
                 } else {
-                    const int i = pt - 64;
+                    const int i = prow - 64;
                     const float Gq = G[i];
                     float m[32];
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
-                        const int j = 32 * half + jj;
+                        const int j = 32 * phf + jj;
                         m[jj] = (j <= i) ? v[jj] * __expf(Gq - G[j]) : 0.f;
                     }
-                    store_row_f16_sw128(sM, i, 4 * half, m, 1.f);
+                    store_row_f16_sw128(sM, i, 4 * phf, m, 1.f);
                 }
             }
             tc_fence_before();
@@ -436,17 +440,29 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             // ---- T = (I + A)^-1, then T diag(beta) and T diag(beta e^G) as f16 B operands
             chunk_tsolve(sA, sP, pt);
             {
-                const int t = pt >> 1, part = pt & 1;
-                const float* Tr = sA + t * LDA + 32 * part;
-                float t1[32], t2[32];
+                const int t = pt >> 2, part = pt & 3;
+                const float* Tr = sA + t * LDA + 16 * part;
+                float t1[16], t2[16];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int tp = 32 * part + e;
+                for (int e = 0; e < 16; ++e) {
+                    const int tp = 16 * part + e;
                     t1[e] = Tr[e] * s_beta[tp];
                     t2[e] = t1[e] * eG[tp];
                 }
-                store_row_f16_sw128(smem + OFF_T1, t, 4 * part, t1, 1.f);
-                store_row_f16_sw128(smem + OFF_T2, t, 4 * part, t2, 1.f);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    uint4 p1, p2;
+                    p1.x = pack_half2(t1[8 * j], t1[8 * j + 1]);
+                    p1.y = pack_half2(t1[8 * j + 2], t1[8 * j + 3]);
+                    p1.z = pack_half2(t1[8 * j + 4], t1[8 * j + 5]);
+                    p1.w = pack_half2(t1[8 * j + 6], t1[8 * j + 7]);
+                    p2.x = pack_half2(t2[8 * j], t2[8 * j + 1]);
+                    p2.y = pack_half2(t2[8 * j + 2], t2[8 * j + 3]);
+                    p2.z = pack_half2(t2[8 * j + 4], t2[8 * j + 5]);
+                    p2.w = pack_half2(t2[8 * j + 6], t2[8 * j + 7]);
+                    *reinterpret_cast<uint4*>(smem + OFF_T1 + sw128_chunk(t, 2 * part + j)) = p1;
+                    *reinterpret_cast<uint4*>(smem + OFF_T2 + sw128_chunk(t, 2 * part + j)) = p2;
+                }
             }
             fence_proxy_async_smem();
             named_barrier_sync(1, kPThreads);
@@ -478,12 +494,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             }
 
             // ---- W^T to shared memory (MN-major B operand: row k, 64 tokens)
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            {
                 float v[32];
-                tmem_ld32(tlane + T_WT + 32 * half, v);
+                tmem_ld32(tlane + T_WT + 32 * phf, v);
                 tmem_ld_wait();
-                store_row_f16_sw128(sWt, pt, 4 * half, v, 1.f);
+                store_row_f16_sw128(sWt, prow, 4 * phf, v, 1.f);
             }
             fence_proxy_async_smem();
             tc_fence_before();
