@@ -183,7 +183,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     }
     // 3. chunked recurrence on tensor cores, gated RMSNorm epilogue
     {
-        CUtensorMap mK, mQ, mKl, mQl, mV;
+        CUtensorMap mK, mQ, mKl, mQl, mV, mZ;
         if (!make_map(&mK, Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&mKl, Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
@@ -193,7 +193,9 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
             !make_map(&mQ, Qs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&mV, Vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Vh * 128, total, 64, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
             return GDN_ERR_CUDA;
         ChunkParams cp{};
         cp.Kh = Kh;
@@ -215,7 +217,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         });
         if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
         dim3 grid(Vh, N);
-        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mK, mQ, mKl, mQl, mV, cp);
+        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mK, mQ, mKl, mQl, mV, mZ, cp);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     return GDN_OK;

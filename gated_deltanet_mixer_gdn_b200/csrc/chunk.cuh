@@ -60,8 +60,8 @@ constexpr uint32_t OFF_KQ0 = 0;        // [K rows 0-63 | Q rows 64-127] x k 0-63
 constexpr uint32_t OFF_KQ1 = 32768;    // second buffer
 constexpr uint32_t OFF_LO = 65536;     // same layout, f16 residuals; then A / T f32 and the T-solve scratch
 constexpr uint32_t OFF_V = 98304;      // V [64 t][64 v] x 2 blocks
-constexpr uint32_t OFF_WT0 = 114688;   // W^T f16 [128 k][64 t], two buffers
-constexpr uint32_t OFF_WT1 = 131072;
+constexpr uint32_t OFF_WT = 114688;    // W^T f16 [128 k][64 t]
+constexpr uint32_t OFF_Z = 131072;     // z bf16 [64 t][128], plain row-major
 constexpr uint32_t OFF_S16 = 147456;   // S0 f16 [128 v][64 k] x 2 blocks
 constexpr uint32_t OFF_T1 = 180224;    // T diag(beta) f16 [64][64]
 constexpr uint32_t OFF_T2 = 188416;    // T diag(beta e^G) f16 [64][64]
@@ -79,13 +79,15 @@ static_assert(64 * LDA * 4 + 32 * 36 * 4 <= 32768, "A/T and scratch must fit in 
 constexpr uint32_t T_KQ = 0, T_WT = 64, T_U0 = 128, T_U1 = 192, T_OI = 256, T_OA = 320, T_S = 384;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t KQV_BYTES = 6 * 8192;
+constexpr uint32_t Z_BYTES = 64 * 128 * 2;
 constexpr uint32_t LO_BYTES = 4 * 8192;
 constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, false, false, false);
 constexpr uint32_t ID_AMN = idesc_f16_f32(128, 64, true, false, false);
 constexpr uint32_t ID_NEG_BMN = idesc_f16_f32(128, 64, false, true, true);
 constexpr uint32_t ID_DS = idesc_f16_f32(128, 128, false, true, false);
 // mbarrier slots
-constexpr int B_KQV = 0, B_LO = 1, B_P = 2, B_S = 3, B_PRO = 4, B_ST = 6, B_KQF = 8;
+constexpr int B_KQV = 0, B_LO = 1, B_P = 2, B_S = 3, B_PRO = 4, B_ST = 6, B_KQF = 8, B_Z = 10, B_WTF = 11;
+constexpr int kBars = 12;
 }  // namespace chunk
 
 // ---- warp-level TF32 tensor-core products for the triangular solve.
@@ -241,7 +243,8 @@ __device__ __forceinline__ void store_row_f16_sw128(uint8_t* tile, uint32_t row,
 __global__ void __launch_bounds__(chunk::kThreads, 1)
     gdn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmQl,
-                     const __grid_constant__ CUtensorMap tmV, const ChunkParams p) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZ,
+                     const ChunkParams p) {
     using namespace chunk;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -271,13 +274,14 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     const int nchunks = (len + C - 1) / C;
 
     if (tid == 0) {
-        for (int i = 0; i < 10; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kBars; ++i) mbar_init(&bars[i], 1);
         fence_barrier_init();
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmKl);
         prefetch_tensormap(&tmQl);
         prefetch_tensormap(&tmV);
+        prefetch_tensormap(&tmZ);
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, TMEM_COLS);
@@ -304,9 +308,14 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         tma_load_2d(smem + OFF_LO + 8192, &tmQl, kap * 128, y, &bars[B_LO]);
         tma_load_2d(smem + OFF_LO + 24576, &tmQl, kap * 128 + 64, y, &bars[B_LO]);
     };
+    auto load_z = [&](int y) {
+        mbar_arrive_expect_tx(&bars[B_Z], Z_BYTES);
+        tma_load_2d(smem + OFF_Z, &tmZ, h * 128, y, &bars[B_Z]);
+    };
     if (tid == 0 && nchunks > 0) {
         load_kqv(OFF_KQ0, start);
         load_lo(start);
+        load_z(start);
     }
     bool broken = false;
     // every thread of the warp calls this; the warp is converged again on return
@@ -340,7 +349,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             float* eG = s_eG + 64 * b;
             float* dec = s_dec + 64 * b;
             uint8_t* sM = smem + (b ? OFF_M1 : OFF_M0);
-            uint8_t* sWt = smem + (b ? OFF_WT1 : OFF_WT0);
+            uint8_t* sWt = smem + OFF_WT;
             const uint32_t T_U = b ? T_U1 : T_U0;
             // the state group must be done with chunk c-2's copies of these buffers
             if (c >= 2) wait(B_ST + b, ((c - 2) >> 1) & 1);
@@ -493,7 +502,9 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                 __syncwarp();
             }
 
-            // ---- W^T to shared memory (MN-major B operand: row k, 64 tokens)
+            // ---- W^T to shared memory (MN-major B operand: row k, 64 tokens), once the
+            //      state group's MMA4 of chunk c-1 has read the previous one
+            if (c >= 1) wait(B_WTF, (c - 1) & 1);
             {
                 float v[32];
                 tmem_ld32(tlane + T_WT + 32 * phf, v);
@@ -551,22 +562,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             const uint32_t aKQ = sbase + (b ? OFF_KQ1 : OFF_KQ0);
             const float* eG = s_eG + 64 * b;
             const float* dec = s_dec + 64 * b;
-            const uint32_t aWt = sbase + (b ? OFF_WT1 : OFF_WT0);
+            const uint32_t aWt = sbase + OFF_WT;
             const uint32_t aM = sbase + (b ? OFF_M1 : OFF_M0);
             const uint32_t T_U = b ? T_U1 : T_U0;
             wait(B_PRO + b, (c >> 1) & 1);
             tc_fence_after();
-
-            // z of this thread's channel for its 32 tokens (used by the epilogue)
-            uint32_t zz[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int t0 = 32 * hf + 2 * j;
-                const uint16_t* zp = p.z + (size_t)(tok0 + t0) * p.Vh * 128 + h * 128 + row;
-                const uint32_t lo = (t0 < nv) ? __ldg(zp) : 0u;
-                const uint32_t hi = (t0 + 1 < nv) ? __ldg(zp + (size_t)p.Vh * 128) : 0u;
-                zz[j] = lo | (hi << 16);
-            }
 
             // ---- MMA4: U^T = U~^T - S0 W^T ; MMA5: Oi^T = S0 Q^T
             if (st == 0) {
@@ -588,6 +588,8 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             wait(B_S, sphase);
             sphase ^= 1;
             tc_fence_after();
+            if (st == 0) mbar_arrive(&bars[B_WTF]);  // W^T of this chunk has been read
+            __syncwarp();
 
             // ---- U^T to f16 in TMEM (plain, and scaled by e^{G_C - G_t}); state scaled by e^{G_C}
             {
@@ -669,12 +671,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                     s_rstd[st] = rsqrtf(ms + kEps);
                 }
                 named_barrier_sync(2, kSThreads);
+                wait(B_Z, c & 1);
+                const uint16_t* zt = reinterpret_cast<const uint16_t*>(smem + OFF_Z);
                 uint16_t* op = p.out + (size_t)tok0 * p.Vh * 128 + h * 128 + row;
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
                     const int t = 32 * hf + jj;
-                    const uint32_t zb = (jj & 1) ? (zz[jj >> 1] >> 16) : (zz[jj >> 1] & 0xffffu);
-                    const float zv = bf16_bits_to_float(static_cast<uint16_t>(zb));
+                    const float zv = bf16_bits_to_float(zt[t * 128 + row]);
                     const float y = o[jj] * s_rstd[t] * wn * silu_f(zv);
                     if (t < nv) op[(size_t)t * p.Vh * 128] = float_to_bf16_bits(y);
                 }
@@ -682,6 +685,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             named_barrier_sync(2, kSThreads);
+            if (st == 0 && c + 1 < nchunks) load_z(tok0 + C);  // the z tile of the next chunk
             if (st == 0) mbar_arrive(&bars[B_ST + b]);  // chunk c's shared buffers are released
         }
 
