@@ -69,15 +69,29 @@ struct PrepParams {
     float* Bs;
 };
 
-// One CTA per token and 16 head slots (16 threads x 8 channels each): four
-// 16-byte tap loads per thread, no loop, so many CTAs per SM keep enough
-// loads in flight; the rows shared by neighbouring tokens hit in L2.
+constexpr int kPrepTokens = 16;  // consecutive tokens per thread
+constexpr int kPrepAhead = 4;    // rows loaded ahead of the token being computed
+
+__device__ __forceinline__ void unpack8(const uint4 v, float (&x)[8]) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        x[2 * m] = __uint_as_float(u[m] << 16);
+        x[2 * m + 1] = __uint_as_float(u[m] & 0xffff0000u);
+    }
+}
+
+// A CTA covers 16 head slots (16 threads x 8 channels each) for kPrepTokens
+// consecutive tokens.  Each thread keeps its taps unpacked and the last three
+// inputs of its channels in registers (a rolling window that restarts from
+// the row's history at every row start), and loads the next inputs
+// kPrepAhead tokens ahead, so a token costs one 16-byte load and ~130
+// instructions per thread.
 __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     const int tid = threadIdx.x;
     const int grp = tid >> 4;
     const int gl = tid & 15;
     const int nheads = 2 * p.Kh + p.Vh;
-    const int t = blockIdx.x;
     // Slots past the last head run along (clamped, no stores) so that every
     // lane of a warp reaches the shuffles.
     const bool active = blockIdx.y * 16 + grp < nheads;
@@ -86,102 +100,131 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     const bool is_q = slot < p.Kh;
     const bool is_v = slot >= 2 * p.Kh;
     const int vh = slot - 2 * p.Kh;
+    const int t0 = blockIdx.x * kPrepTokens;
+    const int nt = min(kPrepTokens, p.total - t0);
+    if (nt <= 0) return;  // whole CTA
 
-    int n, start, len;
-    p.seq.locate(t, n, start, len);
-    const int s = t - start;
-    // taps j = 0..3 read index s + j of [history (3 rows); tokens of the row]
-    uint4 xr[4];
-    float4 hx[4][2];
+    // next inputs, kPrepAhead tokens ahead
+    uint4 ahead[kPrepAhead];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int xi = s + j;
-        if (xi >= 3) {
-            xr[j] = __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)(t + j - 3) * p.C + ch0));
-        } else if (p.init_conv != nullptr) {
-            const float4* hp = reinterpret_cast<const float4*>(p.init_conv + ((size_t)n * 3 + xi) * p.C + ch0);
-            hx[j][0] = __ldg(hp);
-            hx[j][1] = __ldg(hp + 1);
-        } else {
-            hx[j][0] = make_float4(0.f, 0.f, 0.f, 0.f);
-            hx[j][1] = hx[j][0];
-        }
-    }
-    uint4 wq[4];
+    for (int i = 0; i < kPrepAhead; ++i)
+        ahead[i] = (i < nt) ? __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)(t0 + i) * p.C + ch0))
+                            : make_uint4(0u, 0u, 0u, 0u);
+    float w[4][8];  // w[j][e]: tap j of channel ch0 + e
     {
         const uint4* wp = reinterpret_cast<const uint4*>(p.conv_w + (size_t)ch0 * 4);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) wq[q] = __ldg(wp + q);
-    }
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float x[8];
-        if (s + j >= 3) {
-            const uint32_t u[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = __ldg(wp + q);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                x[2 * m] = __uint_as_float(u[m] << 16);
-                x[2 * m + 1] = __uint_as_float(u[m] & 0xffff0000u);
+                const int e = q * 2 + m / 2;  // two channels per uint4 (8 bf16 = 2 x 4 taps)
+                const int j = (m % 2) * 2;
+                w[j][e] = __uint_as_float(u[m] << 16);
+                w[j + 1][e] = __uint_as_float(u[m] & 0xffff0000u);
             }
-        } else {
-            x[0] = hx[j][0].x; x[1] = hx[j][0].y; x[2] = hx[j][0].z; x[3] = hx[j][0].w;
-            x[4] = hx[j][1].x; x[5] = hx[j][1].y; x[6] = hx[j][1].z; x[7] = hx[j][1].w;
         }
-        // tap j of channel e: bf16 at conv_w[(ch0 + e) * 4 + j]; two channels per uint4
+    }
+    const float gA = is_v ? expf(__ldg(p.A_log + vh)) : 0.f;
+    const float gdt = is_v ? __ldg(p.dt_bias + vh) : 0.f;
+
+    int n, start, len;
+    p.seq.locate(t0, n, start, len);
+    // window: w0 = index s, w1 = s + 1, w2 = s + 2 of [history (3 rows); tokens of the row]
+    float w0[8], w1[8], w2[8];
+    auto fetch_xbar = [&](int nn, int xi, int tok, float (&x)[8]) {
+        if (xi >= 3) {
+            unpack8(__ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)tok * p.C + ch0)), x);
+        } else if (p.init_conv != nullptr) {
+            const float4* hp = reinterpret_cast<const float4*>(p.init_conv + ((size_t)nn * 3 + xi) * p.C + ch0);
+            const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
+            x[0] = h0.x; x[1] = h0.y; x[2] = h0.z; x[3] = h0.w;
+            x[4] = h1.x; x[5] = h1.y; x[6] = h1.z; x[7] = h1.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        }
+    };
+    {
+        const int s = t0 - start;
+        fetch_xbar(n, s, t0 - 3, w0);
+        fetch_xbar(n, s + 1, t0 - 2, w1);
+        fetch_xbar(n, s + 2, t0 - 1, w2);
+    }
+
+#pragma unroll
+    for (int tt = 0; tt < kPrepTokens; ++tt) {
+        if (tt >= nt) break;
+        const int t = t0 + tt;
+        float xn[8];
+        unpack8(ahead[tt % kPrepAhead], xn);
+        if (tt + kPrepAhead < nt)
+            ahead[tt % kPrepAhead] =
+                __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)(t + kPrepAhead) * p.C + ch0));
+        if (t == start + len) {  // a new row starts here (skip empty rows): restart from its history
+            if (p.seq.cu == nullptr) {
+                ++n;
+                start += len;
+            } else {
+                do {
+                    ++n;
+                    start = __ldg(p.seq.cu + n);
+                    len = __ldg(p.seq.cu + n + 1) - start;
+                } while (len == 0);
+            }
+            fetch_xbar(n, 0, 0, w0);
+            fetch_xbar(n, 1, 0, w1);
+            fetch_xbar(n, 2, 0, w2);
+        }
+        float act[8];
+        float ss = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const uint4 wv = wq[e >> 1];
-            const uint32_t word = (e & 1) ? ((j < 2) ? wv.z : wv.w) : ((j < 2) ? wv.x : wv.y);
-            const float wj = (j & 1) ? __uint_as_float(word & 0xffff0000u) : __uint_as_float(word << 16);
-            acc[e] = fmaf(wj, x[e], acc[e]);
+            const float cv = fmaf(w[0][e], w0[e], fmaf(w[1][e], w1[e], fmaf(w[2][e], w2[e], w[3][e] * xn[e])));
+            act[e] = silu_f(cv);
+            ss = fmaf(act[e], act[e], ss);
+            w0[e] = w1[e];
+            w1[e] = w2[e];
+            w2[e] = xn[e];
         }
-    }
-    float act[8];
-    float ss = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        act[e] = silu_f(acc[e]);
-        ss = fmaf(act[e], act[e], ss);
-    }
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (!active) return;
-    float scale = 1.0f;
-    if (!is_v) {
-        scale = rsqrtf(ss + kEps);
-        if (is_q) scale *= rsqrtf((float)kD);
-    }
-    float xs[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) xs[e] = act[e] * scale;
-    uint4 pk;
-    pk.x = pack_half2(xs[0], xs[1]);
-    pk.y = pack_half2(xs[2], xs[3]);
-    pk.z = pack_half2(xs[4], xs[5]);
-    pk.w = pack_half2(xs[6], xs[7]);
-    if (is_v) {
-        *reinterpret_cast<uint4*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + gl * 8) = pk;
-        if (gl == 0) {
-            const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
-            const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);
-            p.Gs[(size_t)vh * p.total + t] = -expf(__ldg(p.A_log + vh)) * softplus_f(av + __ldg(p.dt_bias + vh));
-            p.Bs[(size_t)vh * p.total + t] = sigmoid_f(bv);
+        for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (!active) continue;
+        float scale = 1.0f;
+        if (!is_v) {
+            scale = rsqrtf(ss + kEps);
+            if (is_q) scale *= rsqrtf((float)kD);
         }
-    } else {
-        const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + gl * 8;
-        const __half2* hp = reinterpret_cast<const __half2*>(&pk);
-        uint4 lo;
-        uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+        float xs[8];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float2 hf = __half22float2(hp[m]);
-            lw[m] = pack_half2(xs[2 * m] - hf.x, xs[2 * m + 1] - hf.y);
+        for (int e = 0; e < 8; ++e) xs[e] = act[e] * scale;
+        uint4 pk;
+        pk.x = pack_half2(xs[0], xs[1]);
+        pk.y = pack_half2(xs[2], xs[3]);
+        pk.z = pack_half2(xs[4], xs[5]);
+        pk.w = pack_half2(xs[6], xs[7]);
+        if (is_v) {
+            *reinterpret_cast<uint4*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + gl * 8) = pk;
+            if (gl == 0) {
+                const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
+                const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);
+                p.Gs[(size_t)vh * p.total + t] = -gA * softplus_f(av + gdt);
+                p.Bs[(size_t)vh * p.total + t] = sigmoid_f(bv);
+            }
+        } else {
+            const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + gl * 8;
+            const __half2* hp = reinterpret_cast<const __half2*>(&pk);
+            uint4 lo;
+            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float2 hf = __half22float2(hp[m]);
+                lw[m] = pack_half2(xs[2 * m] - hf.x, xs[2 * m + 1] - hf.y);
+            }
+            *reinterpret_cast<uint4*>((is_q ? p.Qs : p.Ks) + off) = pk;
+            *reinterpret_cast<uint4*>((is_q ? p.Ql : p.Kl) + off) = lo;
         }
-        *reinterpret_cast<uint4*>((is_q ? p.Qs : p.Ks) + off) = pk;
-        *reinterpret_cast<uint4*>((is_q ? p.Ql : p.Kl) + off) = lo;
     }
 }
 
