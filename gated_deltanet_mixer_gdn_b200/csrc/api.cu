@@ -164,7 +164,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         pp.Vs = Vs;
         pp.Gs = Gs;
         pp.Bs = Bs;
-        dim3 grid((total + kPrepTokens - 1) / kPrepTokens, (2 * Kh + Vh + 15) / 16);
+        dim3 grid((total + kPrepTokens - 1) / kPrepTokens, (2 * Kh + Vh + kPrepSlots - 1) / kPrepSlots);
         gdn_prep_kernel<<<grid, 256, 0, stream>>>(pp);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }

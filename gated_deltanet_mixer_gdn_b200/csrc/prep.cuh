@@ -8,9 +8,9 @@
 //   Gs, Bs  f32 [Vh][total]       (g = log-decay, beta = write rate)
 // A second tiny kernel writes each row's final conv history.
 //
-// Mapping: a CTA of 256 threads is 16 groups of 16; a group owns one
-// 128-channel head slot, each thread 8 contiguous channels (16-byte loads and
-// stores), so the per-token L2 norm is a 16-lane shuffle reduction.
+// Mapping: a warp owns one 128-channel head slot, each lane 4 contiguous
+// channels (8-byte loads and stores), so the per-token L2 norm is one warp
+// shuffle reduction.
 #pragma once
 
 #include "common.cuh"
@@ -70,33 +70,28 @@ struct PrepParams {
 };
 
 constexpr int kPrepTokens = 16;  // consecutive tokens per thread
-constexpr int kPrepAhead = 4;    // rows loaded ahead of the token being computed
+constexpr int kPrepAhead = 8;    // rows loaded ahead of the token being computed
+constexpr int kPrepSlots = 8;    // head slots (warps) per CTA
 
-__device__ __forceinline__ void unpack8(const uint4 v, float (&x)[8]) {
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        x[2 * m] = __uint_as_float(u[m] << 16);
-        x[2 * m + 1] = __uint_as_float(u[m] & 0xffff0000u);
-    }
+__device__ __forceinline__ void unpack4(const uint2 v, float (&x)[4]) {
+    x[0] = __uint_as_float(v.x << 16);
+    x[1] = __uint_as_float(v.x & 0xffff0000u);
+    x[2] = __uint_as_float(v.y << 16);
+    x[3] = __uint_as_float(v.y & 0xffff0000u);
 }
 
-// A CTA covers 16 head slots (16 threads x 8 channels each) for kPrepTokens
-// consecutive tokens.  Each thread keeps its taps unpacked and the last three
-// inputs of its channels in registers (a rolling window that restarts from
-// the row's history at every row start), and loads the next inputs
-// kPrepAhead tokens ahead, so a token costs one 16-byte load and ~130
-// instructions per thread.
-__global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
-    const int tid = threadIdx.x;
-    const int grp = tid >> 4;
-    const int gl = tid & 15;
+// A CTA covers 8 head slots (one warp each, 4 channels per lane) for
+// kPrepTokens consecutive tokens.  Each thread keeps its taps unpacked and the
+// last three inputs of its channels in registers (a rolling window that
+// restarts from the row's history at every row start), and loads the next
+// inputs kPrepAhead tokens ahead: per token one 8-byte load and a short
+// instruction chain per thread, with many warps resident per SM.
+__global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
+    const int lane = threadIdx.x & 31;
     const int nheads = 2 * p.Kh + p.Vh;
-    // Slots past the last head run along (clamped, no stores) so that every
-    // lane of a warp reaches the shuffles.
-    const bool active = blockIdx.y * 16 + grp < nheads;
-    const int slot = active ? blockIdx.y * 16 + grp : nheads - 1;
-    const int ch0 = slot * kD + gl * 8;
+    const int slot = blockIdx.y * kPrepSlots + (threadIdx.x >> 5);
+    if (slot >= nheads) return;  // whole warp
+    const int ch0 = slot * kD + lane * 4;
     const bool is_q = slot < p.Kh;
     const bool is_v = slot >= 2 * p.Kh;
     const int vh = slot - 2 * p.Kh;
@@ -104,17 +99,16 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     const int nt = min(kPrepTokens, p.total - t0);
     if (nt <= 0) return;  // whole CTA
 
-    // next inputs, kPrepAhead tokens ahead
-    uint4 ahead[kPrepAhead];
+    uint2 ahead[kPrepAhead];
 #pragma unroll
     for (int i = 0; i < kPrepAhead; ++i)
-        ahead[i] = (i < nt) ? __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)(t0 + i) * p.C + ch0))
-                            : make_uint4(0u, 0u, 0u, 0u);
-    float w[4][8];  // w[j][e]: tap j of channel ch0 + e
+        ahead[i] = (i < nt) ? __ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)(t0 + i) * p.C + ch0))
+                            : make_uint2(0u, 0u);
+    float w[4][4];  // w[j][e]: tap j of channel ch0 + e
     {
         const uint4* wp = reinterpret_cast<const uint4*>(p.conv_w + (size_t)ch0 * 4);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
             const uint4 v = __ldg(wp + q);
             const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -132,18 +126,16 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     int n, start, len;
     p.seq.locate(t0, n, start, len);
     // window: w0 = index s, w1 = s + 1, w2 = s + 2 of [history (3 rows); tokens of the row]
-    float w0[8], w1[8], w2[8];
-    auto fetch_xbar = [&](int nn, int xi, int tok, float (&x)[8]) {
+    float w0[4], w1[4], w2[4];
+    auto fetch_xbar = [&](int nn, int xi, int tok, float (&x)[4]) {
         if (xi >= 3) {
-            unpack8(__ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)tok * p.C + ch0)), x);
+            unpack4(__ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)tok * p.C + ch0)), x);
         } else if (p.init_conv != nullptr) {
-            const float4* hp = reinterpret_cast<const float4*>(p.init_conv + ((size_t)nn * 3 + xi) * p.C + ch0);
-            const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
-            x[0] = h0.x; x[1] = h0.y; x[2] = h0.z; x[3] = h0.w;
-            x[4] = h1.x; x[5] = h1.y; x[6] = h1.z; x[7] = h1.w;
+            const float4 h = __ldg(reinterpret_cast<const float4*>(p.init_conv + ((size_t)nn * 3 + xi) * p.C + ch0));
+            x[0] = h.x; x[1] = h.y; x[2] = h.z; x[3] = h.w;
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+            for (int e = 0; e < 4; ++e) x[e] = 0.f;
         }
     };
     {
@@ -157,11 +149,11 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
     for (int tt = 0; tt < kPrepTokens; ++tt) {
         if (tt >= nt) break;
         const int t = t0 + tt;
-        float xn[8];
-        unpack8(ahead[tt % kPrepAhead], xn);
+        float xn[4];
+        unpack4(ahead[tt % kPrepAhead], xn);
         if (tt + kPrepAhead < nt)
             ahead[tt % kPrepAhead] =
-                __ldg(reinterpret_cast<const uint4*>(p.qkv + (size_t)(t + kPrepAhead) * p.C + ch0));
+                __ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)(t + kPrepAhead) * p.C + ch0));
         if (t == start + len) {  // a new row starts here (skip empty rows): restart from its history
             if (p.seq.cu == nullptr) {
                 ++n;
@@ -177,10 +169,10 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
             fetch_xbar(n, 1, 0, w1);
             fetch_xbar(n, 2, 0, w2);
         }
-        float act[8];
+        float act[4];
         float ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
             const float cv = fmaf(w[0][e], w0[e], fmaf(w[1][e], w1[e], fmaf(w[2][e], w2[e], w[3][e] * xn[e])));
             act[e] = silu_f(cv);
             ss = fmaf(act[e], act[e], ss);
@@ -188,42 +180,36 @@ __global__ void __launch_bounds__(256) gdn_prep_kernel(const PrepParams p) {
             w1[e] = w2[e];
             w2[e] = xn[e];
         }
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (!active) continue;
         float scale = 1.0f;
-        if (!is_v) {
+        if (!is_v) {  // warp-uniform
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
             scale = rsqrtf(ss + kEps);
             if (is_q) scale *= rsqrtf((float)kD);
         }
-        float xs[8];
+        float xs[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) xs[e] = act[e] * scale;
-        uint4 pk;
+        for (int e = 0; e < 4; ++e) xs[e] = act[e] * scale;
+        uint2 pk;
         pk.x = pack_half2(xs[0], xs[1]);
         pk.y = pack_half2(xs[2], xs[3]);
-        pk.z = pack_half2(xs[4], xs[5]);
-        pk.w = pack_half2(xs[6], xs[7]);
         if (is_v) {
-            *reinterpret_cast<uint4*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + gl * 8) = pk;
-            if (gl == 0) {
+            *reinterpret_cast<uint2*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + lane * 4) = pk;
+            if (lane == 0) {
                 const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
                 const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);
                 p.Gs[(size_t)vh * p.total + t] = -gA * softplus_f(av + gdt);
                 p.Bs[(size_t)vh * p.total + t] = sigmoid_f(bv);
             }
         } else {
-            const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + gl * 8;
-            const __half2* hp = reinterpret_cast<const __half2*>(&pk);
-            uint4 lo;
-            uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float2 hf = __half22float2(hp[m]);
-                lw[m] = pack_half2(xs[2 * m] - hf.x, xs[2 * m + 1] - hf.y);
-            }
-            *reinterpret_cast<uint4*>((is_q ? p.Qs : p.Ks) + off) = pk;
-            *reinterpret_cast<uint4*>((is_q ? p.Ql : p.Kl) + off) = lo;
+            const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + lane * 4;
+            const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&pk.x));
+            const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&pk.y));
+            uint2 lo;
+            lo.x = pack_half2(xs[0] - h0.x, xs[1] - h0.y);
+            lo.y = pack_half2(xs[2] - h1.x, xs[3] - h1.y);
+            *reinterpret_cast<uint2*>((is_q ? p.Qs : p.Ks) + off) = pk;
+            *reinterpret_cast<uint2*>((is_q ? p.Ql : p.Kl) + off) = lo;
         }
     }
 }
