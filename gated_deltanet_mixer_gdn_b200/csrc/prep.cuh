@@ -120,8 +120,13 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
             }
         }
     }
-    const float gA = is_v ? expf(__ldg(p.A_log + vh)) : 0.f;
-    const float gdt = is_v ? __ldg(p.dt_bias + vh) : 0.f;
+    if (is_v && lane < nt) {  // gates of this value head: one token per lane
+        const int t = t0 + lane;
+        const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
+        const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);
+        p.Gs[(size_t)vh * p.total + t] = -expf(__ldg(p.A_log + vh)) * softplus_f(av + __ldg(p.dt_bias + vh));
+        p.Bs[(size_t)vh * p.total + t] = sigmoid_f(bv);
+    }
 
     int n, start, len;
     p.seq.locate(t0, n, start, len);
@@ -195,12 +200,6 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
         pk.y = pack_half2(xs[2], xs[3]);
         if (is_v) {
             *reinterpret_cast<uint2*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + lane * 4) = pk;
-            if (lane == 0) {
-                const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
-                const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);
-                p.Gs[(size_t)vh * p.total + t] = -gA * softplus_f(av + gdt);
-                p.Bs[(size_t)vh * p.total + t] = sigmoid_f(bv);
-            }
         } else {
             const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + lane * 4;
             const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&pk.x));
