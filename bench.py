@@ -4,8 +4,9 @@ Default workload (N=1): the decode batch — 64 rows x 128 successive single-tok
 steps with the 27B model's GDN shapes, each row with its own f32 state
 [48,128,128] ~ N(0,0.05) and conv history ~ N(0,1).  One bench step = that
 whole pass (128 decode launches, 8192 row-tokens).  Metric: row-tokens/s.
-A second measured object, "prefill", times the chunked prefill of one row of
-8192 tokens (zero initial state) in tokens/s against the tensor roofline.
+A second measured object, "prefill", times the chunked prefill (one row of
+8192 tokens from zero state, and the 8-row varlen workload) in tokens/s
+against the tensor roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -37,6 +38,21 @@ STATE_BYTES_PER_ROW_TOKEN = 2 * 48 * 128 * 128 * 4          # f32 state read + w
 PREFILL_T = 8192
 PREFILL_FLOP_PER_TOKEN = 7602176                               # chunk-64 contraction FLOPs, 48 heads
 PREFILL_BYTES_PER_TOKEN = 10240 * 2 + 6144 * 2 + 2 * 48 * 2 + 6144 * 2
+
+
+def decode_traffic():
+    """DRAM bytes per decode launch from the committed ncu record, if it was taken
+    on the decode kernel's current source; else None."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", "gdn_decode_kernel_traffic.json")
+    src = os.path.join(ROOT, "gated_deltanet_mixer_gdn_b200", "csrc", "decode.cuh")
+    if not os.path.exists(rec):
+        return None
+    with open(rec) as f:
+        d = json.load(f)
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    return d.get("bytes_per_launch") if d.get("decode_cuh_sha256") == h else None
 
 
 def load_peaks():
@@ -282,7 +298,7 @@ def run_ours(args, world, rank, local):
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (402.7 MB of state per step)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": decode_traffic(),
                          "kernel": "gdn_decode_kernel", "peak_source": peaks["source"],
                          "algorithmic_bytes_per_launch": ROWS * STATE_BYTES_PER_ROW_TOKEN},
             "e2e": {"value": e2e_value, "unit": "row-tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -292,43 +308,68 @@ def run_ours(args, world, rank, local):
     return line, case
 
 
-def bench_prefill(args, world, rank, local, T):
-    """Chunked prefill of one row of T tokens (zero initial state), L2 flushed before each call."""
-    import gated_deltanet_mixer_gdn_b200 as gdn
-    dev = torch.device("cuda", local)
-    peaks = load_peaks()
-    stream = torch.cuda.Stream(dev)
-    PREFILL_T = T
-    pcase = synth.config(2) if T == 8192 else synth.dense_case(1236, 1, T)
-    pw = gdn.weights_to(pcase["weights"], dev)
-    pin_acts = {k: pcase[k].to(dev) for k in ("qkv", "z", "a", "b")}
-    pout = torch.empty((1, PREFILL_T, 6144), dtype=torch.bfloat16, device=dev)
-    pst = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
-    pcv = torch.empty((1, 3, 10240), dtype=torch.float32, device=dev)
+def _time_prefill(call, dev, stream, warmup, reps):
+    """Median seconds of `call` (CUDA events on `stream`), L2 flushed before each timed call."""
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > L2, written between iterations
     with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
-            gdn.prefill(pin_acts["qkv"], pin_acts["z"], pin_acts["a"], pin_acts["b"], pw, out=pout,
-                        final_state=pst, final_conv=pcv)
+        for _ in range(warmup):
+            call()
         torch.cuda.synchronize(dev)
         pt = []
-        for _ in range(max(5, args.steps)):
+        for _ in range(reps):
             flush.fill_(1)
             s0 = torch.cuda.Event(enable_timing=True)
             s1 = torch.cuda.Event(enable_timing=True)
             s0.record(stream)
-            gdn.prefill(pin_acts["qkv"], pin_acts["z"], pin_acts["a"], pin_acts["b"], pw, out=pout,
-                        final_state=pst, final_conv=pcv)
+            call()
             s1.record(stream)
             s1.synchronize()
             pt.append(s0.elapsed_time(s1) / 1000.0)
-    p_med = statistics.median(pt)
-    return {"workload": f"prefill B=1 T={T}, zero initial state (3 kernels: load stage, history, chunk)",
-            "value": PREFILL_T / p_med, "unit": "tokens/s", "ms": p_med * 1000.0,
-            "tflops": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12,
-            "frac_of_bf16_peak": PREFILL_T * PREFILL_FLOP_PER_TOKEN / p_med / 1e12 / peaks["bf16_tflops"],
-            "peak_source": peaks["source"], "l2": "flushed (256 MiB write) before each timed call",
-            "gpu_launches": 3 * len(pt)}
+    return statistics.median(pt), len(pt)
+
+
+def bench_prefill(args, world, rank, local, T):
+    """Chunked prefill: one row of T tokens from zero state, and the 8-row varlen
+    workload (lengths U[512,16384] from the seed, random initial state and history)."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(dev)
+    pcase = synth.config(2) if T == 8192 else synth.dense_case(1236, 1, T)
+    pw = gdn.weights_to(pcase["weights"], dev)
+    a1 = {k: pcase[k].to(dev) for k in ("qkv", "z", "a", "b")}
+    pout = torch.empty((1, T, 6144), dtype=torch.bfloat16, device=dev)
+    pst = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
+    pcv = torch.empty((1, 3, 10240), dtype=torch.float32, device=dev)
+    t1, n1 = _time_prefill(lambda: gdn.prefill(a1["qkv"], a1["z"], a1["a"], a1["b"], pw, out=pout, final_state=pst,
+                                               final_conv=pcv), dev, stream, max(3, args.warmup), max(5, args.steps))
+
+    def line(tokens, sec, workload, launches):
+        tf = tokens * PREFILL_FLOP_PER_TOKEN / sec / 1e12
+        return {"workload": workload, "value": tokens / sec, "unit": "tokens/s", "ms": sec * 1000.0,
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"],
+                             "algorithmic_flop_per_token": PREFILL_FLOP_PER_TOKEN},
+                "l2": "flushed (256 MiB write) before each timed call", "gpu_launches": launches}
+
+    out = {"b1": line(T, t1, f"prefill B=1 T={T}, zero initial state", 3 * n1)}
+    if T == 8192:
+        vcase = synth.config(3)
+        vw = gdn.weights_to(vcase["weights"], dev)
+        av = {k: vcase[k].to(dev) for k in ("qkv", "z", "a", "b")}
+        cu, cud = vcase["cu_seqlens"], vcase["cu_seqlens"].to(dev)
+        st0, cv0 = vcase["init_state"].to(dev), vcase["init_conv"].to(dev)
+        total = int(cu[-1])
+        vout = torch.empty((total, 6144), dtype=torch.bfloat16, device=dev)
+        vst = torch.empty_like(st0)
+        vcv = torch.empty_like(cv0)
+        t2, n2 = _time_prefill(lambda: gdn.prefill_varlen(cu, av["qkv"], av["z"], av["a"], av["b"], vw, st0, cv0,
+                                                          out=vout, final_state=vst, final_conv=vcv,
+                                                          cu_seqlens_dev=cud),
+                               dev, stream, max(3, args.warmup), max(5, args.steps))
+        out["varlen8"] = line(total, t2, f"varlen prefill 8 rows ({total} tokens, lengths U[512,16384]), "
+                                         "random initial state and history", 3 * n2)
+    return out
 
 
 def main():
@@ -351,7 +392,7 @@ def main():
         if args.workload == "prefill":
             pre = bench_prefill(args, world, rank, local, args.prefill_T)
             if rank == 0:
-                print(json.dumps({"metric": "GDN prefill tokens/s", **pre}))
+                print(json.dumps({"metric": "GDN prefill tokens/s", **pre["b1"], "varlen8": pre.get("varlen8")}))
             return 0
         line, case = run_ours(args, world, rank, local)
         pre = bench_prefill(args, world, rank, local, args.prefill_T)

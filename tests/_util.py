@@ -94,3 +94,33 @@ def to_dev(case, device="cuda"):
     st = None if case["init_state"] is None else case["init_state"].to(device)
     cv = None if case["init_conv"] is None else case["init_conv"].to(device)
     return w, acts, st, cv
+
+
+def group_case(case, kappa):
+    """The sub-problem of q/k head `kappa`: its q and k channels, the channels,
+    z, gates and parameters of its value heads, as a case with one q/k head.
+    The mixer computes each value head from exactly these inputs, so the
+    oracle on this case gives those heads' outputs and states (and the
+    history of these channels) at a fraction of the cost."""
+    d = case["dims"]
+    G, D = d.num_v_heads // d.num_k_heads, d.head_dim
+    heads = list(range(kappa * G, (kappa + 1) * G))
+    ch = list(range(kappa * D, (kappa + 1) * D)) + list(range(d.num_k_heads * D + kappa * D,
+                                                              d.num_k_heads * D + (kappa + 1) * D))
+    ch += [2 * d.num_k_heads * D + h * D + c for h in heads for c in range(D)]
+    ch = torch.tensor(ch)
+    zc = torch.tensor([h * D + c for h in heads for c in range(D)])
+    hs = torch.tensor(heads)
+    sub = dict(case)
+    sub["dims"] = synth.Dims(num_k_heads=1, num_v_heads=G, head_dim=D, conv_width=d.conv_width)
+    w = case["weights"]
+    sub["weights"] = {"conv_w": w["conv_w"][ch], "A_log": w["A_log"][hs], "dt_bias": w["dt_bias"][hs],
+                      "norm_w": w["norm_w"]}
+    for k, idx in (("qkv", ch), ("z", zc), ("a", hs), ("b", hs)):
+        sub[k] = case[k].index_select(-1, idx).contiguous()
+    if case.get("init_state") is not None:
+        sub["init_state"] = case["init_state"][:, hs].contiguous()
+    if case.get("init_conv") is not None:
+        sub["init_conv"] = case["init_conv"].index_select(-1, ch).contiguous()
+    sub["channels"], sub["z_channels"], sub["heads"] = ch, zc, hs
+    return sub

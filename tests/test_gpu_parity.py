@@ -15,8 +15,8 @@ import torch
 import gated_deltanet_mixer_gdn_b200 as gdn
 from gated_deltanet_mixer_gdn_b200 import synth
 
-from _util import (OUT_RMS_TOL, OUT_TOL, STATE_TOL, conv_exact, oracle_prefill, out_err, out_rms_err,
-                   state_err, to_dev)
+from _util import (OUT_RMS_TOL, OUT_TOL, STATE_TOL, conv_exact, group_case, oracle_prefill, out_err,
+                   out_rms_err, state_err, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -208,14 +208,50 @@ def test_chunked_prefill_8192_and_split():
     _check_prefill(case, (torch.cat([o1, o2], 1), s2, c2), ref)
 
 
-def test_varlen_benchmark_rows_sampled_heads():
-    """The 8-row varlen workload (lengths U[512,16384]); oracle on 3 value heads."""
+def test_varlen_benchmark_rows_sampled_group():
+    """The 8-row varlen workload (lengths U[512,16384]); oracle on the 3 value
+    heads of q/k head 7."""
     case = synth.config(3)
-    heads = (21, 24)
-    ref = oracle_prefill(case, heads=heads)
+    sub = group_case(case, 7)
+    ref = oracle_prefill(sub)
     w, acts, st, cv = to_dev(case)
     out, fs, fc = gdn.prefill_varlen(case["cu_seqlens"], acts["qkv"], acts["z"], acts["a"], acts["b"], w, st, cv)
     torch.cuda.synchronize()
-    assert out_err(out[:, heads[0] * 128:heads[1] * 128], ref["out"]) <= OUT_TOL
-    assert state_err(fs[:, heads[0]:heads[1]], ref["state"]) <= STATE_TOL
-    assert conv_exact(fc, ref["conv"])
+    zc, hs, ch = sub["z_channels"].cuda(), sub["heads"].cuda(), sub["channels"].cuda()
+    assert out_err(out.index_select(1, zc), ref["out"]) <= OUT_TOL
+    assert out_rms_err(out.index_select(1, zc), ref["out"]) <= OUT_RMS_TOL
+    assert state_err(fs.index_select(1, hs), ref["state"]) <= STATE_TOL
+    assert conv_exact(fc.index_select(2, ch), ref["conv"])
+
+
+def test_long_context_two_rows_then_decode_sampled_group():
+    """Two rows of 65,536 tokens from zero state, returning final states, then
+    256 decode steps per row from those states; oracle on the 3 value heads of
+    q/k head 15 (and the history of their channels)."""
+    case = synth.config(4)
+    sub = group_case(case, 15)
+    w, acts, _, _ = to_dev(case)
+    out, fs, fc = gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w)
+    torch.cuda.synchronize()
+    ref = oracle_prefill(sub)
+    zc, hs, ch = sub["z_channels"].cuda(), sub["heads"].cuda(), sub["channels"].cuda()
+    o2 = out.reshape(2 * 65536, -1).index_select(1, zc)
+    assert out_err(o2, ref["out"]) <= OUT_TOL
+    assert out_rms_err(o2, ref["out"]) <= OUT_RMS_TOL
+    assert state_err(fs.index_select(1, hs), ref["state"]) <= STATE_TOL
+    assert conv_exact(fc.index_select(2, ch), ref["conv"])
+    # 256 decode steps from the GPU's final state; the oracle continues from its own
+    dec = case["decode"]
+    outs = [gdn.decode(*(dec[k][s].cuda() for k in ("qkv", "z", "a", "b")), w, fs, fc) for s in range(256)]
+    torch.cuda.synchronize()
+    st_ref, cv_ref = ref["state"], ref["conv"]
+    errs = []
+    for s in range(256):
+        step = {"qkv": dec["qkv"][s].index_select(-1, sub["channels"]), "z": dec["z"][s].index_select(-1, sub["z_channels"]),
+                "a": dec["a"][s].index_select(-1, sub["heads"]), "b": dec["b"][s].index_select(-1, sub["heads"])}
+        r = oracle_prefill(sub, cu=np.arange(3), init_state=st_ref, init_conv=cv_ref, acts=step)
+        errs.append(out_err(outs[s].index_select(1, zc), r["out"]))
+        st_ref, cv_ref = r["state"], r["conv"]
+    assert max(errs) <= OUT_TOL
+    assert state_err(fs.index_select(1, hs), st_ref) <= STATE_TOL
+    assert conv_exact(fc.index_select(2, ch), cv_ref)

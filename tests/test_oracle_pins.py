@@ -323,3 +323,18 @@ def test_mixer_head_subset():
     D = TINY.head_dim
     assert np.array_equal(part["out"], full["out"][:, 2 * D:5 * D])
     assert np.array_equal(part["state"], full["state"][:, 2:5])
+
+
+def test_group_case_reproduces_full_mixer_heads():
+    """The one-q/k-head sub-problem used by the full-size parity tests gives
+    exactly the full mixer's outputs, states and history for that group."""
+    from _util import group_case
+    case = synth.prefill_case(13, [9, 4], TINY, init=True)
+    full = _mixer(case)
+    sub = group_case(case, 1)
+    part = _mixer(sub)
+    D = TINY.head_dim
+    hs = sub["heads"].numpy()
+    assert np.array_equal(part["out"], full["out"][:, hs[0] * D:(hs[-1] + 1) * D])
+    assert np.array_equal(part["state"], full["state"][:, hs])
+    assert np.array_equal(part["conv"], full["conv"][:, :, sub["channels"].numpy()])
