@@ -85,10 +85,14 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t
 }
 
 struct Workspace {
-    size_t off_q, off_k, off_ql, off_kl, off_v, off_g, off_b, bytes;
+    size_t off_q, off_k, off_ql, off_kl, off_v, off_g, off_b, off_cb, off_rec, bytes;
 };
 
-Workspace plan_workspace(const gdn_dims* d, int64_t total) {
+// Chunks over all rows: exact for uniform rows, and an upper bound for N rows
+// of `total` tokens in all (each row adds at most one partial chunk).
+int64_t chunk_bound(int64_t N, int64_t total) { return (total + 63 * N) / 64; }
+
+Workspace plan_workspace(const gdn_dims* d, int64_t total, int64_t N, int64_t nchunks) {
     Workspace w{};
     const size_t qk = (size_t)total * d->num_k_heads * 128 * 2;
     const size_t vv = (size_t)total * d->num_v_heads * 128 * 2;
@@ -100,12 +104,14 @@ Workspace plan_workspace(const gdn_dims* d, int64_t total) {
     w.off_v = w.off_kl + align_up(qk);
     w.off_g = w.off_v + align_up(vv);
     w.off_b = w.off_g + align_up(gb);
-    w.bytes = w.off_b + align_up(gb);
+    w.off_cb = w.off_b + align_up(gb);
+    w.off_rec = w.off_cb + align_up((size_t)(N + 1) * 4);
+    w.bytes = w.off_rec + align_up((size_t)nchunks * d->num_v_heads * wy::REC_BYTES);
     return w;
 }
 
 int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32_t* cu_dev, int32_t uniform_T,
-                 int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                 int32_t total, int64_t nchunks, int64_t nchunks_planned, const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
                  const float* init_state, const float* init_conv, uint16_t* out, float* final_state,
                  float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
@@ -130,7 +136,8 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         return GDN_OK;
     }
 
-    const Workspace ws = plan_workspace(d, total);
+    const Workspace ws = plan_workspace(d, total, N, nchunks_planned);
+    if (nchunks > nchunks_planned || nchunks > INT32_MAX / d->num_v_heads) return GDN_ERR_INVALID_ARG;
     if (workspace == nullptr || workspace_bytes < ws.bytes) return GDN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
@@ -141,6 +148,8 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     __half* Vs = reinterpret_cast<__half*>(wsb + ws.off_v);
     float* Gs = reinterpret_cast<float*>(wsb + ws.off_g);
     float* Bs = reinterpret_cast<float*>(wsb + ws.off_b);
+    int* chunk_base = cu_dev ? reinterpret_cast<int*>(wsb + ws.off_cb) : nullptr;
+    uint8_t* rec = wsb + ws.off_rec;
 
     // 1. load stage: conv + silu, L2 norms, gates
     {
@@ -181,33 +190,68 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         gdn_conv_out_kernel<<<grid, 256, 0, stream>>>(cp);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
-    // 3. chunked recurrence on tensor cores, gated RMSNorm epilogue
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    CUtensorMap mK, mQ, mKl, mQl, mV, mZ, mO;
+    if (!make_map(&mK, Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mKl, Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mQl, Ql, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mQ, Qs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mV, Vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Vh * 128, total, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&mO, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+        return GDN_ERR_CUDA;
+    // 3. first chunk of every row (packed rows only)
+    if (chunk_base != nullptr) {
+        gdn_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu_dev, N, chunk_base);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    // 4. per-chunk WY records, all chunks in parallel
+    if (nchunks > 0) {
+        WyParams wp{};
+        wp.Kh = Kh;
+        wp.Vh = Vh;
+        wp.total = total;
+        wp.seq = seq;
+        wp.chunk_base = chunk_base;
+        wp.nchunks = (int)nchunks;
+        wp.Gs = Gs;
+        wp.Bs = Bs;
+        wp.rec = rec;
+        static std::once_flag wy_once;
+        static cudaError_t wy_err = cudaSuccess;
+        std::call_once(wy_once, [] {
+            wy_err = cudaFuncSetAttribute(gdn_wy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)wy::SMEM_BYTES);
+        });
+        if (wy_err != cudaSuccess) return GDN_ERR_CUDA;
+        const int ratio = Vh / Kh;
+        const int64_t ntasks = nchunks * Kh * ((ratio + wy::kHeads - 1) / wy::kHeads);
+        const int grid = (int)(ntasks < nsm ? ntasks : nsm);
+        gdn_wy_kernel<<<grid, wy::kThreads, wy::SMEM_BYTES, stream>>>(mK, mQ, mKl, mQl, wp);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    // 5. the state recurrence, gated RMSNorm epilogue
     {
-        CUtensorMap mK, mQ, mKl, mQl, mV, mZ;
-        if (!make_map(&mK, Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&mKl, Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&mQl, Ql, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&mQ, Qs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&mV, Vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Vh * 128, total, 64, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
-            return GDN_ERR_CUDA;
         ChunkParams cp{};
         cp.Kh = Kh;
         cp.Vh = Vh;
         cp.total = total;
         cp.seq = seq;
-        cp.Gs = Gs;
-        cp.Bs = Bs;
+        cp.chunk_base = chunk_base;
+        cp.rec = rec;
         cp.init_state = init_state;
         cp.final_state = final_state;
         cp.norm_w = w->norm_w;
-        cp.z = z;
         cp.out = out;
         static std::once_flag attr_once;
         static cudaError_t attr_err = cudaSuccess;
@@ -217,7 +261,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         });
         if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
         dim3 grid(Vh, N);
-        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mK, mQ, mKl, mQl, mV, mZ, cp);
+        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mK, mQ, mV, mZ, mO, cp);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     return GDN_OK;
@@ -269,12 +313,12 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
     if (check_dims(dims) != GDN_OK || B < 0 || T < 0) return 0;
     const int64_t total = (int64_t)B * T;
     if (total > INT32_MAX) return 0;
-    return plan_workspace(dims, total).bytes;
+    return plan_workspace(dims, total, B, (int64_t)B * ((T + 63) / 64)).bytes;
 }
 
 size_t gdn_prefill_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T) {
     if (check_dims(dims) != GDN_OK || N < 0 || total_T < 0) return 0;
-    return plan_workspace(dims, total_T).bytes;
+    return plan_workspace(dims, total_T, N, chunk_bound(N, total_T)).bytes;
 }
 
 int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, const uint16_t* qkv,
@@ -290,8 +334,9 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
     if ((st = check_io((int32_t)total, qkv, z, a, b, out, init_state, init_conv, final_state, final_conv)) != GDN_OK)
         return st;
     if ((st = check_device()) != GDN_OK) return st;
-    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, qkv, z, a, b, init_state, init_conv, out, final_state,
-                        final_conv, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    const int64_t nch = (int64_t)B * ((T + 63) / 64);
+    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, a, b, init_state, init_conv, out,
+                        final_state, final_conv, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_host,
@@ -311,8 +356,11 @@ int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, co
     if ((st = check_io(total_T, qkv, z, a, b, out, init_state, init_conv, final_state, final_conv)) != GDN_OK)
         return st;
     if ((st = check_device()) != GDN_OK) return st;
-    return prefill_impl(dims, w, N, cu_dev, 0, total_T, qkv, z, a, b, init_state, init_conv, out, final_state,
-                        final_conv, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    int64_t nch = 0;
+    for (int32_t i = 0; i < N; ++i) nch += (cu_host[i + 1] - cu_host[i] + 63) / 64;
+    return prefill_impl(dims, w, N, cu_dev, 0, total_T, nch, chunk_bound(N, total_T), qkv, z, a, b, init_state,
+                        init_conv, out, final_state, final_conv, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const uint16_t* qkv, const uint16_t* z,
@@ -377,12 +425,14 @@ int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, i
     if (total > INT32_MAX) return GDN_ERR_INVALID_ARG;
     if ((st = check_io((int32_t)total, qkv, z, a, b, out, init_state, init_conv, final_state, final_conv)) != GDN_OK)
         return st;
-    if (plan_workspace(dims, total).bytes > (size_t)GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
+    const int64_t nch = (int64_t)B * ((T + 63) / 64);
+    if (plan_workspace(dims, total, B, nch).bytes > (size_t)GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
     if ((st = check_device()) != GDN_OK) return st;
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != GDN_OK) return st;
-    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, qkv, z, a, b, init_state, init_conv, out, final_state,
-                        final_conv, scratch, (size_t)GDN_NOALLOC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
+    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, a, b, init_state, init_conv, out,
+                        final_state, final_conv, scratch, (size_t)GDN_NOALLOC_SCRATCH_BYTES,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int gdn_last_device_error(void) {

@@ -84,6 +84,14 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// Tiled TMA store of a box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(smem_src))
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -254,6 +262,21 @@ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t r, uint32_t c) { return
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 32 values -> 4 chunks of 8 f16 of row `row` of a 128-byte-swizzled tile,
+// starting at 16-byte chunk index chunk0 (shared or global memory).
+__device__ __forceinline__ void store_row_f16_sw128(uint8_t* tile, uint32_t row, uint32_t chunk0, const float* vals,
+                                                    float scale_all) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 pk;
+        pk.x = pack_half2(vals[8 * j + 0] * scale_all, vals[8 * j + 1] * scale_all);
+        pk.y = pack_half2(vals[8 * j + 2] * scale_all, vals[8 * j + 3] * scale_all);
+        pk.z = pack_half2(vals[8 * j + 4] * scale_all, vals[8 * j + 5] * scale_all);
+        pk.w = pack_half2(vals[8 * j + 6] * scale_all, vals[8 * j + 7] * scale_all);
+        *reinterpret_cast<uint4*>(tile + sw128_chunk(row, chunk0 + j)) = pk;
+    }
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }

@@ -143,11 +143,13 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
  *
  * Same arguments, layouts, aliasing and results as gdn_prefill, minus
  * workspace / workspace_bytes.  The scratch lives in one file-scope device
- * array of GDN_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads this
+ * array of GDN_NOALLOC_SCRATCH_BYTES (64 MiB) that every GPU which loads this
  * library holds until the process exits.  A request whose scratch exceeds it
- * is rejected with GDN_ERR_WORKSPACE before anything is enqueued; for the
- * 27B model's dims (16/48 heads) that is B*T > 1154 tokens (29,056 bytes per
- * token plus alignment).  The call itself allocates nothing.
+ * (gdn_prefill_workspace_size(dims, B, T) > GDN_NOALLOC_SCRATCH_BYTES) is
+ * rejected with GDN_ERR_WORKSPACE before anything is enqueued; for the 27B
+ * model's dims (16/48 heads) that is about 1,200 tokens per call (one row of
+ * up to 1216 tokens; 29,056 bytes per token plus 1,597,440 bytes per 64-token
+ * chunk of a row).  The call itself allocates nothing.
  *
  * The first call on each device resolves the device address of the array
  * (cudaGetSymbolAddress, with that device current); make that first call
@@ -157,7 +159,7 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
  * overlaps on the GPU (different streams, or different host threads without
  * ordering) race on the array: order them on one stream.
  */
-#define GDN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+#define GDN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T,
                         const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
                         const float* init_state, const float* init_conv,

@@ -46,8 +46,13 @@ def test_workspace_sizes(lib):
     d = _dims()
     one = lib.gdn_prefill_workspace_size(ctypes.byref(d), 1, 1)
     big = lib.gdn_prefill_workspace_size(ctypes.byref(d), 2, 1000)
-    assert one > 0 and big >= 2000 * (4 * 16 * 128 * 2 + 48 * 128 * 2 + 2 * 48 * 4)
-    assert lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 3, 2000) == big
+    # per token: q, k and their residual parts (f16), v (f16), gates; per 64-token chunk
+    # and value head a 33,280-byte record of the chunked form
+    assert one > 0 and big >= 2000 * (4 * 16 * 128 * 2 + 48 * 128 * 2 + 2 * 48 * 4) + 2 * 16 * 48 * 33280
+    # packed rows are planned for the most chunks N rows of 2000 tokens can have
+    assert lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 2, 2000) >= big
+    assert lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 3, 2000) >= \
+        lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 2, 2000)
     assert lib.gdn_prefill_workspace_size(ctypes.byref(_dims(d=64)), 1, 10) == 0
     assert lib.gdn_prefill_workspace_size(ctypes.byref(d), -1, 10) == 0
 
