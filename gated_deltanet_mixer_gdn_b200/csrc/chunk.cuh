@@ -385,18 +385,28 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             wait(B_Z, c & 1);
             // a full chunk is written over its z tile and leaves by one TMA store; a ragged
             // last chunk is stored directly (the rows past it belong to the next sequence)
+            // (the branch stays outside the loops so that their elements can overlap)
             const bool full = (nv == C);
-            uint16_t* zt = reinterpret_cast<uint16_t*>(smem + OFF_Z);
-            uint16_t* op = p.out + (size_t)tok0 * p.Vh * 128 + h * 128 + row;
+            uint16_t* zt = reinterpret_cast<uint16_t*>(smem + OFF_Z) + 32 * hf * 128 + row;
+            const float* rs = s_rstd + 32 * hf;
+            if (full) {
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-                const int t = 32 * hf + jj;
-                const float zv = bf16_bits_to_float(zt[t * 128 + row]);
-                const uint16_t y = float_to_bf16_bits(o[jj] * s_rstd[t] * wn * silu_f(zv));
-                if (full) zt[t * 128 + row] = y;
-                else if (t < nv) op[(size_t)t * p.Vh * 128] = y;
+                for (int jj = 0; jj < 32; ++jj) {
+                    const float zv = bf16_bits_to_float(zt[jj * 128]);
+                    zt[jj * 128] = float_to_bf16_bits(o[jj] * rs[jj] * wn * silu_f(zv));
+                }
+                fence_proxy_async_smem();
+            } else {
+                uint16_t* op = p.out + (size_t)(tok0 + 32 * hf) * p.Vh * 128 + h * 128 + row;
+                const int nt = nv - 32 * hf;  // tokens of this half inside the row
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    if (jj < nt) {
+                        const float zv = bf16_bits_to_float(zt[jj * 128]);
+                        op[(size_t)jj * p.Vh * 128] = float_to_bf16_bits(o[jj] * rs[jj] * wn * silu_f(zv));
+                    }
+                }
             }
-            if (full) fence_proxy_async_smem();
             named_barrier_sync(3, kEThreads);
             if (et == 0) {
                 if (full) {

@@ -438,7 +438,8 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             {
                 const bool is_a = row < 64;
                 const int i = is_a ? row : row - 64;
-                const float Gr = sG[i], bi = sbeta[i];
+                const int last = is_a ? i - 1 : i;  // last unmasked column
+                const float Gr = sG[i], scale = is_a ? sbeta[i] : 1.f;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
@@ -448,8 +449,8 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = 32 * hh + jj;
-                        e[jj] = is_a ? ((j < i) ? bi * __expf(Gr - sG[j]) * v[jj] : 0.f)
-                                     : ((j <= i) ? v[jj] * __expf(Gr - sG[j]) : 0.f);
+                        const float d = __expf(Gr - sG[j]);  // (masked below; the branch-free form overlaps)
+                        e[jj] = (j <= last) ? scale * d * v[jj] : 0.f;
                     }
                     if (is_a) {
                         float4* dst = reinterpret_cast<float4*>(sA + i * LDA + 32 * hh);
