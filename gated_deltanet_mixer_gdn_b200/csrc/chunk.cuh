@@ -5,25 +5,27 @@
 // head with state S [128 v][128 k]:
 //     S_t = exp(g_t) S_{t-1} + u_t k_t^T,   u_t = beta_t (v_t - exp(g_t) S_{t-1} k_t),
 //     o_t = S_t q_t.
-// Over a chunk of 64 tokens, with the per-chunk record of wy.cuh (T1, W, M
-// and the decays, none of which depends on the state):
+// Over a chunk of 64 tokens, with the per-chunk record of wy.cuh (T1, W, Qs,
+// K', M and e^{G_C}, none of which depends on the state):
 //     U   = T1 V - W S0^T                                   (U~ = T1 V)
-//     O   = diag(e^G) Q S0^T + M U
-//     S_C = e^{G_C} S0 + U^T diag(e^{G_C - G}) K.
+//     O   = Qs S0^T + M U                                   (Qs = diag(e^G) Q)
+//     S_C = e^{G_C} S0 + U^T K'                             (K' = diag(e^{G_C - G}) K).
 //
-// One CTA owns one (row, value head) and walks its chunks in order.  Two
-// warp-specialised groups run side by side:
-//   * the chain (8 warps) carries the state: MMA4 U^T = U~^T - S0 W^T and
-//     MMA5 Oi^T = S0 Q^T with S0 as f16 in shared memory; U^T to f16 in TMEM
-//     (plain, and scaled by e^{G_C - G}); MMA6 S += (U^T diag e^{G_C-G}) K and
-//     MMA7 Oa^T = U^T M^T with A read from TMEM; then the f16 copy of the new
-//     state and its scaling by the next chunk's e^{G_C}.  Its thread 0 also
-//     issues the loads of chunk c+2 and MMA2 U~^T = V^T T1^T of chunk c+1;
-//   * the epilogue (8 warps) turns Oi, Oa of chunk c into o = e^G Oi + Oa,
-//     the gated RMSNorm and the bf16 output while the chain is on chunk c+1
-//     (double-buffered accumulators).
-// Every contraction is a tcgen05.mma with M = 128 and an f32 accumulator in
-// TMEM.
+// One CTA owns one (row, value head) and walks its chunks in order.  Per chunk
+// the tensor cores run four products, all tcgen05.mma kind::f16 with M = 128
+// and f32 accumulators in TMEM:
+//     MMA-P  U~^T        = V^T T1^T                 (state-free, issued a chunk ahead)
+//     MMA-A  [U^T | O^T] += S0 [-W ; Qs]^T           (one N = 128 pass; S0 as f16 in TMEM)
+//     MMA-S  S           += U^T K'                   (U^T as f16 in TMEM)
+//     MMA7   O^T         += U^T M^T
+// Only MMA-A, the f16 conversion of U^T, MMA-S and the f16 copy of the new
+// state are on the sequential path from one chunk to the next; a single
+// issuing thread keeps the tensor pipe fed while
+//   * the converters (8 warps) turn U^T and the state into f16 operands, then
+//     scale the f32 state by the next chunk's e^{G_C} while MMA-A runs, and
+//   * the epilogue (16 warps, 16 tokens each) turns O^T of chunk c into the
+//     gated RMSNorm and the bf16 output while the chain is on chunk c+1 (two
+//     accumulators).
 #pragma once
 
 #include "common.cuh"
@@ -45,65 +47,62 @@ struct ChunkParams {
 
 namespace chunk {
 constexpr int C = 64;              // tokens per chunk
-constexpr int kCThreads = 256;     // state chain, warps 0-7
-constexpr int kEThreads = 256;     // epilogue, warps 8-15
-constexpr int kThreads = kCThreads + kEThreads;
-// one input buffer: K, Q, V f16 [64 t][64] x 2 column blocks (TMA, 128B swizzle), then the record
-constexpr uint32_t BUF_K = 0, BUF_Q = 16384, BUF_V = 32768, BUF_REC = 49152;
-constexpr uint32_t BUF_BYTES = BUF_REC + 33792;  // record rounded up to 1 KB
+constexpr int kCThreads = 256;     // converters, warps 0-7
+constexpr int kEThreads = 512;     // epilogue, warps 8-23
+constexpr int kIssuerWarp = 24;    // tensor-core issue
+constexpr int kLoaderWarp = 25;    // TMA loads of the chunk inputs
+constexpr int kThreads = kCThreads + kEThreads + 64;
+// one input buffer: V f16 [64 t][64] x 2 column blocks (TMA, 128B swizzle), then the record
+constexpr uint32_t BUF_V = 0, BUF_REC = 16384;
+constexpr uint32_t BUF_BYTES = 82944;  // rounded up to 1 KB
+static_assert(BUF_REC + wy::REC_BYTES <= BUF_BYTES, "input buffer");
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_BUF0 = 0;
 constexpr uint32_t OFF_BUF1 = BUF_BYTES;
-constexpr uint32_t OFF_S16 = 2 * BUF_BYTES;      // S0 f16 [128 v][64 k] x 2 blocks
-constexpr uint32_t OFF_Z = OFF_S16 + 32768;      // z bf16 [64 t][128], plain row-major; the output tile
-constexpr uint32_t OFF_MISC = OFF_Z + 16384;
-constexpr uint32_t MISC_BYTES = 3072;
+constexpr uint32_t OFF_Z = 2 * BUF_BYTES;  // 2 x z bf16 [64 t][128], plain row-major; the output tiles
+constexpr uint32_t OFF_MISC = OFF_Z + 2 * 16384;
+constexpr uint32_t MISC_BYTES = 2048;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-// misc: 0 barriers, 128 TMEM slot, 256 e^G [4][64] (by chunk mod 4), 1280 reductions [4][64], 2304 rstd[64]
-// TMEM columns (f32, 128 lanes)
-constexpr uint32_t T_U0 = 0, T_U1 = 64, T_S = 128, T_O0 = 256, T_O1 = 384;  // O: Oi at +0, Oa at +64
+// misc: 0 barriers, 128 TMEM slot, 256 reductions [4][64], 1280 rstd [64]
+// TMEM columns (32-bit, 128 lanes = v rows)
+constexpr uint32_t T_S = 0;                  // state f32 [128 v][128 k]
+constexpr uint32_t T_D0 = 128, T_D1 = 256;   // per buffer: U^T f32 [128][64] at +0, O^T at +64
+constexpr uint32_t T_S16 = 384;              // state f16, k pairs (A of MMA-A)
+constexpr uint32_t T_U16 = 448;              // U^T f16, t pairs (A of MMA-S and MMA7)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t LD_BYTES = 3 * 16384 + wy::REC_BYTES;
+constexpr uint32_t LD_BYTES = 16384 + wy::REC_BYTES;
 constexpr uint32_t Z_BYTES = 64 * 128 * 2;
-constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, false, false, false);
-constexpr uint32_t ID_AMN = idesc_f16_f32(128, 64, true, false, false);
-constexpr uint32_t ID_NEG_BMN = idesc_f16_f32(128, 64, false, true, true);
-constexpr uint32_t ID_DS = idesc_f16_f32(128, 128, false, true, false);
+constexpr uint32_t ID_P = idesc_f16_f32(128, 64, true, false, false);   // V^T (MN-major) x T1 (K-major)
+constexpr uint32_t ID_A = idesc_f16_f32(128, 128, false, false, false); // S16 x [-W ; Qs] (K-major)
+constexpr uint32_t ID_S = idesc_f16_f32(128, 128, false, true, false);  // U16 x K' (MN-major)
+constexpr uint32_t ID_7 = idesc_f16_f32(128, 64, false, false, false);  // Up x M (K-major)
 // mbarrier slots
-constexpr int B_LD = 0, B_S = 2, B_O = 3, B_E = 5, B_Z = 7;  // B_LD, B_O, B_E: + buffer
-constexpr int kBars = 8;
+constexpr int B_LD = 0;     // + buffer: inputs landed
+constexpr int B_A = 2;      // MMA-A complete
+constexpr int B_UC = 3;     // U^T converted (one arrive per converter warp)
+constexpr int B_SM = 4;     // MMA-S complete
+constexpr int B_SC = 5;     // state converted (one arrive per converter warp)
+constexpr int B_O = 6;      // + buffer: MMA7 complete, O^T final
+constexpr int B_E = 8;      // + buffer: the epilogue has read and cleared O^T
+constexpr int B_FREE = 10;  // + buffer: every MMA that reads the buffer is complete
+constexpr int B_Z = 12;     // + z buffer: z tile landed
+constexpr int B_SS = 14;    // f32 state scaled by e^{G_C} (one arrive per converter warp)
+constexpr int kBars = 15;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace chunk
 
-// Lane l of the warp ends with sum over the 32 lanes of v[l] (31 shuffles).
-__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < off; ++i) {
-            const float send = upper ? v[i] : v[i + off];
-            const float keep = upper ? v[i + off] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-    }
-    return v[0];
-}
-
 __global__ void __launch_bounds__(chunk::kThreads, 1)
-    gdn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZ,
-                     const __grid_constant__ CUtensorMap tmO, const ChunkParams p) {
+    gdn_chunk_kernel(const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmO,
+                     const ChunkParams p) {
     using namespace chunk;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_u32(smem);
 
     const int h = blockIdx.x;
     const int n = blockIdx.y;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int kap = h / (p.Vh / p.Kh);
     const int q4 = warp & 3;                  // TMEM lane quarter
     const int hf = (warp >> 2) & 1;           // column half within the group
     const int row = 32 * q4 + lane;           // v row of the state / output channel
@@ -112,9 +111,8 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     uint8_t* misc = smem + OFF_MISC;
     uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc + 128);
-    float* s_eG = reinterpret_cast<float*>(misc + 256);     // [4][64]
-    float* s_red = reinterpret_cast<float*>(misc + 1280);   // [4][64]
-    float* s_rstd = reinterpret_cast<float*>(misc + 2304);  // [64]
+    float* s_red = reinterpret_cast<float*>(misc + 256);    // [4][64]
+    float* s_rstd = reinterpret_cast<float*>(misc + 1280);  // [64]
 
     int start, len;
     p.seq.bounds(n, start, len);
@@ -122,17 +120,9 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     const int cbase = p.chunk_base ? __ldg(p.chunk_base + n) : n * ((p.seq.uniform_T + C - 1) / C);
 
     if (tid == 0) {
-        mbar_init(&bars[B_LD], 1);
-        mbar_init(&bars[B_LD + 1], 1);
-        mbar_init(&bars[B_S], 1);
-        mbar_init(&bars[B_O], 2);  // the chain's arrive (e^G published) + the commit of MMA7
-        mbar_init(&bars[B_O + 1], 2);
-        mbar_init(&bars[B_E], 1);
-        mbar_init(&bars[B_E + 1], 1);
-        mbar_init(&bars[B_Z], 1);
+        for (int i = 0; i < kBars; ++i)
+            mbar_init(&bars[i], (i == B_UC || i == B_SC || i == B_SS) ? kCThreads / 32 : 1);
         fence_barrier_init();
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmV);
         prefetch_tensormap(&tmZ);
         prefetch_tensormap(&tmO);
@@ -147,37 +137,28 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     const uint32_t tbase = *s_tmem;
 
     auto buf = [&](int c) { return smem + ((c & 1) ? OFF_BUF1 : OFF_BUF0); };
+    auto dacc = [&](int c) { return tbase + ((c & 1) ? T_D1 : T_D0); };
+    auto rec_of = [&](int c) { return p.rec + ((size_t)(cbase + c) * p.Vh + h) * wy::REC_BYTES; };
     auto load_chunk = [&](int c) {
         uint8_t* B = buf(c);
         uint64_t* bar = &bars[B_LD + (c & 1)];
         const int y = start + c * C;
         mbar_arrive_expect_tx(bar, LD_BYTES);
-        tma_load_2d(B + BUF_K, &tmK, kap * 128, y, bar);
-        tma_load_2d(B + BUF_K + 8192, &tmK, kap * 128 + 64, y, bar);
-        tma_load_2d(B + BUF_Q, &tmQ, kap * 128, y, bar);
-        tma_load_2d(B + BUF_Q + 8192, &tmQ, kap * 128 + 64, y, bar);
         tma_load_2d(B + BUF_V, &tmV, h * 128, y, bar);
         tma_load_2d(B + BUF_V + 8192, &tmV, h * 128 + 64, y, bar);
-        bulk_load(B + BUF_REC, p.rec + ((size_t)(cbase + c) * p.Vh + h) * wy::REC_BYTES, wy::REC_BYTES, bar);
+        bulk_load(B + BUF_REC, rec_of(c), wy::REC_BYTES, bar);
+    };
+    auto prefetch_chunk = [&](int c) {
+        const int y = start + c * C;
+        prefetch_tma_2d(&tmV, h * 128, y);
+        prefetch_tma_2d(&tmV, h * 128 + 64, y);
+        prefetch_l2(rec_of(c), wy::REC_BYTES);
     };
     auto load_z = [&](int c) {
-        mbar_arrive_expect_tx(&bars[B_Z], Z_BYTES);
-        tma_load_2d(smem + OFF_Z, &tmZ, h * 128, start + c * C, &bars[B_Z]);
+        uint64_t* bar = &bars[B_Z + (c & 1)];
+        mbar_arrive_expect_tx(bar, Z_BYTES);
+        tma_load_2d(smem + OFF_Z + (c & 1) * 16384, &tmZ, h * 128, start + c * C, bar);
     };
-    // MMA2: U~^T = V^T T1^T of chunk c into its U buffer
-    auto mma2 = [&](int c) {
-        const uint32_t B = smem_u32(buf(c));
-        const uint32_t tU = tbase + ((c & 1) ? T_U1 : T_U0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            mma_f16(tU, sw128_desc(B + BUF_V + s * 2048, 8192, 1024),
-                    sw128_desc(B + BUF_REC + wy::REC_T1 + s * 32, 16, 1024), ID_AMN, s > 0);
-    };
-    if (tid == 0 && nchunks > 0) {
-        load_chunk(0);
-        if (nchunks > 1) load_chunk(1);
-        load_z(0);
-    }
     bool broken = false;
     // every thread of the warp calls this; the warp is converged again on return
     auto wait = [&](int slot, uint32_t parity) {
@@ -195,15 +176,87 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         }
     };
 
-    if (tid < kCThreads) {
-        // =================================================================== state chain
-        const int ct = tid;
-        // initial state: f16 copy in shared memory, f32 in TMEM scaled by the first chunk's e^{G_C}
+    if (warp == kIssuerWarp) {
+        // =================================================================== issue
+        if (lane == 0 && nchunks > 0) {
+            // MMA-P: U~^T of chunk c into the U^T half of its accumulator
+            auto mma_P = [&](int c) {
+                const uint32_t B = smem_u32(buf(c));
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_f16(dacc(c), sw128_desc(B + BUF_V + s * 2048, 8192, 1024),
+                            sw128_desc(B + BUF_REC + wy::REC_T1 + s * 32, 16, 1024), ID_P, s > 0);
+            };
+            wait1(B_LD, 0);
+            tc_fence_after();
+            mma_P(0);
+            for (int c = 0; c < nchunks; ++c) {
+                const int b = c & 1;
+                const uint32_t B = smem_u32(buf(c));
+                const uint32_t d = dacc(c);
+                wait1(B_E + b, (c >> 1) & 1);  // O^T[b] cleared
+                wait1(B_SC, c & 1);            // state of chunk c in f16 and scaled
+                tc_fence_after();
+                // MMA-A: [U^T | O^T] += S0 [-W ; Qs]^T
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_f16_ta(d, tbase + T_S16 + 8 * s,
+                               sw128_desc(B + BUF_REC + wy::REC_WQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), ID_A,
+                               1);
+                mma_commit(&bars[B_A]);
+                // U~ of the next chunk now if its inputs are in, else after MMA7
+                bool p_next = c + 1 < nchunks;
+                if (p_next && mbar_try_wait(smem_u32(&bars[B_LD + (b ^ 1)]), ((c + 1) >> 1) & 1)) {
+                    tc_fence_after();
+                    mma_P(c + 1);
+                    p_next = false;
+                }
+                wait1(B_UC, c & 1);
+                wait1(B_SS, c & 1);  // f32 state scaled by e^{G_C} of chunk c
+                tc_fence_after();
+                // MMA-S: S += U^T K'
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_f16_ta(tbase + T_S, tbase + T_U16 + 8 * s,
+                               sw128_desc(B + BUF_REC + wy::REC_KP + s * 2048, 8192, 1024), ID_S, 1);
+                mma_commit(&bars[B_SM]);
+                // MMA7: O^T += U^T M^T
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_f16_ta(d + 64, tbase + T_U16 + 8 * s,
+                               sw128_desc(B + BUF_REC + wy::REC_M + s * 32, 16, 1024), ID_7, 1);
+                mma_commit(&bars[B_O + b]);
+                mma_commit(&bars[B_FREE + b]);
+                if (p_next) {
+                    wait1(B_LD + (b ^ 1), ((c + 1) >> 1) & 1);
+                    tc_fence_after();
+                    mma_P(c + 1);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kLoaderWarp) {
+        // =================================================================== loads
+        if (lane == 0 && nchunks > 0) {
+            load_chunk(0);
+            if (nchunks > 1) load_chunk(1);
+            for (int c = 2; c < nchunks && c < 4; ++c) prefetch_chunk(c);
+            // a buffer takes chunk c+2 once every MMA that reads chunk c is done
+            for (int c = 0; c + 2 < nchunks; ++c) {
+                wait1(B_FREE + (c & 1), (c >> 1) & 1);
+                load_chunk(c + 2);
+                if (c + 4 < nchunks) prefetch_chunk(c + 4);
+            }
+        }
+        __syncwarp();
+    } else if (tid < kCThreads) {
+        // =================================================================== converters
+        // initial state: f16 copy for MMA-A, f32 scaled by the first chunk's e^{G_C}
         {
             float gC = 1.f;
             if (nchunks > 0) {
                 wait(B_LD, 0);
-                gC = reinterpret_cast<const float*>(buf(0) + BUF_REC + wy::REC_GATE)[63];
+                gC = *reinterpret_cast<const float*>(buf(0) + BUF_REC + wy::REC_GC);
             }
             const float* src =
                 p.init_state ? p.init_state + (((size_t)n * p.Vh + h) * 128 + row) * 128 + 64 * hf : nullptr;
@@ -219,121 +272,76 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                     v[4 * j + 2] = f.z;
                     v[4 * j + 3] = f.w;
                 }
-                store_row_f16_sw128(smem + OFF_S16 + 16384 * hf, row, 4 * half, v, 1.f);
-                uint32_t r[32];
+                uint32_t hpk[16], r[32];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) hpk[j] = pack_half2(v[2 * j], v[2 * j + 1]);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(gC * v[j]);
+                tmem_st16(tbase + tlane + T_S16 + 32 * hf + 16 * half, hpk);
                 tmem_st32(tbase + tlane + T_S + 64 * hf + 32 * half, r);
             }
             tmem_st_wait();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
-        named_barrier_sync(2, kCThreads);
-        if (ct == 0 && nchunks > 0) {
-            tc_fence_after();
-            mma2(0);
-        }
         __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&bars[B_SC]);
+            mbar_arrive(&bars[B_SS]);
+        }
 
-        uint32_t sphase = 0;
         for (int c = 0; c < nchunks; ++c) {
-            const int b = c & 1;
-            const uint32_t aB = smem_u32(buf(c));
-            const float* gate = reinterpret_cast<const float*>(buf(c) + BUF_REC + wy::REC_GATE);
-            const uint32_t tU = tbase + (b ? T_U1 : T_U0);
-            const uint32_t tO = tbase + (b ? T_O1 : T_O0);
-
-            // ---- MMA4: U^T = U~^T - S0 W^T ; MMA5: Oi^T = S0 Q^T
-            if (ct == 0) {
-                if (c >= 2) wait1(B_E + b, ((c - 2) >> 1) & 1);  // the epilogue is done with O[b]
-                tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint64_t a = sw128_desc(sbase + OFF_S16 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-                    mma_f16(tU, a, sw128_desc(aB + BUF_REC + wy::REC_WT + s * 2048, 8192, 1024), ID_NEG_BMN, 1);
-                }
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint64_t a = sw128_desc(sbase + OFF_S16 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-                    mma_f16(tO, a, sw128_desc(aB + BUF_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_KK, s > 0);
-                }
-                mma_commit(&bars[B_S]);
-            }
-            __syncwarp();
-            wait(B_S, sphase);
-            sphase ^= 1;
+            // ---- U^T to f16 (A of MMA-S and MMA7)
+            wait(B_A, c & 1);
             tc_fence_after();
-
-            // ---- U^T to f16 in TMEM (plain, and scaled by e^{G_C - G_t})
             {
                 float u[32];
-                tmem_ld32(tU + tlane + 32 * hf, u);
+                tmem_ld32(dacc(c) + tlane + 32 * hf, u);
                 tmem_ld_wait();
-                named_barrier_sync(2, kCThreads);  // every f32 U^T column is read before the f16 copies land
-                const float* dec = gate + 64;
-                uint32_t uh[16], us[16];
+                uint32_t up[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = 32 * hf + 2 * j;
-                    uh[j] = pack_half2(u[2 * j], u[2 * j + 1]);
-                    us[j] = pack_half2(u[2 * j] * dec[t], u[2 * j + 1] * dec[t + 1]);
-                }
-                tmem_st16(tU + tlane + 16 * hf, uh);
-                tmem_st16(tU + tlane + 32 + 16 * hf, us);
+                for (int j = 0; j < 16; ++j) up[j] = pack_half2(u[2 * j], u[2 * j + 1]);
+                tmem_st16(tbase + tlane + T_U16 + 16 * hf, up);
                 tmem_st_wait();
-                if (ct < 64) s_eG[(c & 3) * 64 + ct] = gate[ct];
             }
             tc_fence_before();
-            named_barrier_sync(2, kCThreads);
-
-            // ---- MMA6: S += (U^T diag e^{G_C-G}) K ; MMA7: Oa^T = U^T M^T  (A from TMEM)
-            if (ct == 0) {
-                mbar_arrive(&bars[B_O + b]);  // e^G of chunk c is published
-                tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_f16_ta(tbase + T_S, tU + 32 + 8 * s, sw128_desc(aB + BUF_K + s * 2048, 8192, 1024), ID_DS, 1);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_f16_ta(tO + 64, tU + 8 * s, sw128_desc(aB + BUF_REC + wy::REC_M + s * 32, 16, 1024), ID_KK,
-                               s > 0);
-                mma_commit(&bars[B_S]);
-                mma_commit(&bars[B_O + b]);
-                // the other U buffer is free again: U~ of the next chunk
-                if (c + 1 < nchunks) {
-                    wait1(B_LD + (b ^ 1), ((c + 1) >> 1) & 1);
-                    tc_fence_after();
-                    mma2(c + 1);
-                }
-            }
             __syncwarp();
-            wait(B_S, sphase);
-            sphase ^= 1;
+            if (lane == 0) mbar_arrive(&bars[B_UC]);
+
+            // ---- the new state: f16 copy for the next MMA-A first, then the f32 state
+            // scaled by the next e^{G_C} (needed only by the next MMA-S)
+            wait(B_SM, c & 1);
             tc_fence_after();
-            // every input of chunk c has been read: its buffer takes chunk c+2
-            if (ct == 0 && c + 2 < nchunks) load_chunk(c + 2);
-            __syncwarp();
-
-            // ---- f16 copy of the new state for MMA4/5 of chunk c+1; the f32 state scaled by its e^{G_C}
             if (c + 1 < nchunks) {
-                wait(B_LD + (b ^ 1), ((c + 1) >> 1) & 1);
-                const float gC = reinterpret_cast<const float*>(buf(c + 1) + BUF_REC + wy::REC_GATE)[63];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float v[32];
                     tmem_ld32(tbase + tlane + T_S + 64 * hf + 32 * half, v);
                     tmem_ld_wait();
-                    store_row_f16_sw128(smem + OFF_S16 + 16384 * hf, row, 4 * half, v, 1.f);
+                    uint32_t hpk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) hpk[j] = pack_half2(v[2 * j], v[2 * j + 1]);
+                    tmem_st16(tbase + tlane + T_S16 + 32 * hf + 16 * half, hpk);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_SC]);
+                wait(B_LD + ((c + 1) & 1), ((c + 1) >> 1) & 1);
+                const float gC = *reinterpret_cast<const float*>(buf(c + 1) + BUF_REC + wy::REC_GC);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tmem_ld32(tbase + tlane + T_S + 64 * hf + 32 * half, v);
+                    tmem_ld_wait();
                     uint32_t r[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(gC * v[j]);
                     tmem_st32(tbase + tlane + T_S + 64 * hf + 32 * half, r);
                 }
                 tmem_st_wait();
-                fence_proxy_async_smem();
                 tc_fence_before();
-                named_barrier_sync(2, kCThreads);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_SS]);
             }
         }
 
@@ -353,74 +361,94 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     } else {
         // =================================================================== epilogue
         const int et = tid - kCThreads;
+        const int qt = (warp - 8) >> 2;                 // token quarter of this warp
         const float wn = 1.0f + __ldg(p.norm_w + row);  // (1 + w) of this thread's v channel
+        const uint32_t zero[16] = {};
+        // both O^T accumulators start cleared
+        tmem_st16(tbase + tlane + T_D0 + 64 + 16 * qt, zero);
+        tmem_st16(tbase + tlane + T_D1 + 64 + 16 * qt, zero);
+        tmem_st_wait();
+        tc_fence_before();
+        named_barrier_sync(3, kEThreads);
+        if (et == 0) {
+            mbar_arrive(&bars[B_E]);
+            mbar_arrive(&bars[B_E + 1]);
+        }
+        if (et == 32 && nchunks > 0) load_z(0);
+        __syncwarp();
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             const int tok0 = start + c * C;
             const int nv = min(C, len - c * C);
-            const uint32_t tO = tbase + (b ? T_O1 : T_O0);
+            const uint32_t tO = dacc(c) + 64 + tlane + 16 * qt;
+            // z of chunk c+1 into the other tile, once the output of chunk c-1 has left it
+            // (thread 32 of the epilogue owns the output stores and z loads)
+            if (et == 32 && c + 1 < nchunks) {
+                bulk_wait_read_all();
+                load_z(c + 1);
+            }
+            __syncwarp();
             wait(B_O + b, (c >> 1) & 1);
             tc_fence_after();
-            float o[32];
+            float o[16];
+            tmem_ld16(tO, o);
+            tmem_ld_wait();
+            tmem_st16(tO, zero);  // cleared for chunk c+2
+            tmem_st_wait();
+            tc_fence_before();
             {
-                float oa[32];
-                tmem_ld32(tO + tlane + 32 * hf, o);
-                tmem_ld32(tO + tlane + 64 + 32 * hf, oa);
-                tmem_ld_wait();
-                tc_fence_before();
-                const float* eG = s_eG + (c & 3) * 64 + 32 * hf;
+                float sq[16];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    o[jj] = fmaf(eG[jj], o[jj], oa[jj]);
-                    oa[jj] = o[jj] * o[jj];
-                }
-                s_red[q4 * 64 + 32 * hf + lane] = warp_transpose_sum(oa, lane);
+                for (int jj = 0; jj < 16; ++jj) sq[jj] = o[jj] * o[jj];
+                const float part = warp_transpose_sum16(sq, lane);  // token lane >> 1
+                if ((lane & 1) == 0) s_red[q4 * 64 + 16 * qt + (lane >> 1)] = part;
             }
             named_barrier_sync(3, kEThreads);
-            if (et == 0) mbar_arrive(&bars[B_E + b]);  // O[b] may take chunk c+2
+            if (et == 0) mbar_arrive(&bars[B_E + b]);  // O^T[b] may take chunk c+2
             if (et < 64)
                 s_rstd[et] = rsqrtf((s_red[et] + s_red[64 + et] + s_red[128 + et] + s_red[192 + et]) * (1.0f / 128.0f) +
                                     kEps);
             named_barrier_sync(3, kEThreads);
-            wait(B_Z, c & 1);
+            wait(B_Z + b, (c >> 1) & 1);
             // a full chunk is written over its z tile and leaves by one TMA store; a ragged
             // last chunk is stored directly (the rows past it belong to the next sequence)
-            // (the branch stays outside the loops so that their elements can overlap)
+            uint16_t* zt = reinterpret_cast<uint16_t*>(smem + OFF_Z + b * 16384) + 16 * qt * 128 + row;
+            const float* rs = s_rstd + 16 * qt;
+            {
+                float zv[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) zv[jj] = bf16_bits_to_float(zt[jj * 128]);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) o[jj] = o[jj] * rs[jj] * wn * silu_tanh(zv[jj]);
+            }
+            // bf16 rounding two tokens at a time (one paired conversion)
+            uint32_t yb[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) yb[j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
             const bool full = (nv == C);
-            uint16_t* zt = reinterpret_cast<uint16_t*>(smem + OFF_Z) + 32 * hf * 128 + row;
-            const float* rs = s_rstd + 32 * hf;
             if (full) {
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const float zv = bf16_bits_to_float(zt[jj * 128]);
-                    zt[jj * 128] = float_to_bf16_bits(o[jj] * rs[jj] * wn * silu_f(zv));
+                for (int j = 0; j < 8; ++j) {
+                    zt[(2 * j) * 128] = static_cast<uint16_t>(yb[j]);
+                    zt[(2 * j + 1) * 128] = static_cast<uint16_t>(yb[j] >> 16);
                 }
                 fence_proxy_async_smem();
             } else {
-                uint16_t* op = p.out + (size_t)(tok0 + 32 * hf) * p.Vh * 128 + h * 128 + row;
-                const int nt = nv - 32 * hf;  // tokens of this half inside the row
+                uint16_t* op = p.out + (size_t)(tok0 + 16 * qt) * p.Vh * 128 + h * 128 + row;
+                const int nt = nv - 16 * qt;  // tokens of this quarter inside the row
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    if (jj < nt) {
-                        const float zv = bf16_bits_to_float(zt[jj * 128]);
-                        op[(size_t)jj * p.Vh * 128] = float_to_bf16_bits(o[jj] * rs[jj] * wn * silu_f(zv));
-                    }
-                }
+                for (int jj = 0; jj < 16; ++jj)
+                    if (jj < nt)
+                        op[(size_t)jj * p.Vh * 128] = static_cast<uint16_t>((jj & 1) ? (yb[jj >> 1] >> 16) : yb[jj >> 1]);
             }
             named_barrier_sync(3, kEThreads);
-            if (et == 0) {
-                if (full) {
-                    tma_store_2d(&tmO, smem + OFF_Z, h * 128, tok0);
-                    bulk_commit();
-                }
-                if (c + 1 < nchunks) {
-                    bulk_wait_read_all();  // the output tile has left shared memory
-                    load_z(c + 1);
-                }
+            if (et == 32 && full) {
+                tma_store_2d(&tmO, smem + OFF_Z + b * 16384, h * 128, tok0);
+                bulk_commit();
             }
             __syncwarp();
         }
-        if (et == 0) bulk_wait_all();
+        if (et == 32) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();

@@ -92,21 +92,6 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// 16 values per lane -> lane l holds the warp-wide sum of value (l >> 1).
-__device__ __forceinline__ float warp_transpose_sum16(float (&v)[16], int lane) {
-#pragma unroll
-    for (int off = 16, n = 8; off >= 2; off >>= 1, n >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < n; ++i) {
-            const float send = upper ? v[i] : v[i + n];
-            const float keep = upper ? v[i + n] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-    }
-    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
-}
-
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, bool& broken) {
     if (broken) return false;
     if (!mbar_wait(bar, parity)) {
