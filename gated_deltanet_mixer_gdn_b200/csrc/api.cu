@@ -261,7 +261,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         });
         if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
         dim3 grid(Vh, N);
-        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mV, mZ, mO, cp);
+        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mV, mQ, mK, mZ, mO, cp);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     return GDN_OK;

@@ -5,8 +5,8 @@
 // head with state S [128 v][128 k]:
 //     S_t = exp(g_t) S_{t-1} + u_t k_t^T,   u_t = beta_t (v_t - exp(g_t) S_{t-1} k_t),
 //     o_t = S_t q_t.
-// Over a chunk of 64 tokens, with the per-chunk record of wy.cuh (T1, W, Qs,
-// K', M and e^{G_C}, none of which depends on the state):
+// Over a chunk of 64 tokens, with the per-chunk record of wy.cuh (T1, W, M and
+// the decays, none of which depends on the state):
 //     U   = T1 V - W S0^T                                   (U~ = T1 V)
 //     O   = Qs S0^T + M U                                   (Qs = diag(e^G) Q)
 //     S_C = e^{G_C} S0 + U^T K'                             (K' = diag(e^{G_C - G}) K).
@@ -22,7 +22,9 @@
 // state are on the sequential path from one chunk to the next; a single
 // issuing thread keeps the tensor pipe fed while
 //   * the converters (8 warps) turn U^T and the state into f16 operands, then
-//     scale the f32 state by the next chunk's e^{G_C} while MMA-A runs, and
+//     scale the f32 state by the next chunk's e^{G_C} while MMA-A runs,
+//   * the preparers (4 warps) scale the Q and K tiles of the next chunk in
+//     shared memory into Qs and K' (the decays come with the record), and
 //   * the epilogue (16 warps, 16 tokens each) turns O^T of chunk c into the
 //     gated RMSNorm and the bf16 output while the chain is on chunk c+1 (two
 //     accumulators).
@@ -49,13 +51,19 @@ namespace chunk {
 constexpr int C = 64;              // tokens per chunk
 constexpr int kCThreads = 256;     // converters, warps 0-7
 constexpr int kEThreads = 512;     // epilogue, warps 8-23
-constexpr int kIssuerWarp = 24;    // tensor-core issue
-constexpr int kLoaderWarp = 25;    // TMA loads of the chunk inputs
-constexpr int kThreads = kCThreads + kEThreads + 64;
-// one input buffer: V f16 [64 t][64] x 2 column blocks (TMA, 128B swizzle), then the record
-constexpr uint32_t BUF_V = 0, BUF_REC = 16384;
+constexpr int kPThreads = 128;     // preparers, warps 24-27
+constexpr int kIssuerWarp = 28;    // tensor-core issue
+constexpr int kLoaderWarp = 29;    // TMA loads of the chunk inputs
+constexpr int kThreads = kCThreads + kEThreads + kPThreads + 64;
+// one input buffer; every tile is f16 [64 rows][64] with 128-byte rows in the TMA 128B swizzle
+constexpr uint32_t BUF_V = 0;        // V [t][v], 2 column blocks (TMA)
+constexpr uint32_t BUF_T1 = 16384;   // T1 (record)
+constexpr uint32_t BUF_WQ = 24576;   // per k block b at 16384 b: -W (record), then Q (TMA) scaled in place to Qs
+constexpr uint32_t BUF_M = 57344;    // M (record)
+constexpr uint32_t BUF_KP = 65536;   // K (TMA), 2 column blocks, scaled in place to K'
+constexpr uint32_t BUF_DEC = 81920;  // f32 e^{G_C - G_t} [64], e^{G_t} [64], e^{G_C} (record)
 constexpr uint32_t BUF_BYTES = 82944;  // rounded up to 1 KB
-static_assert(BUF_REC + wy::REC_BYTES <= BUF_BYTES, "input buffer");
+static_assert(BUF_DEC + wy::REC_DEC_BYTES <= BUF_BYTES, "input buffer");
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_BUF0 = 0;
 constexpr uint32_t OFF_BUF1 = BUF_BYTES;
@@ -63,14 +71,14 @@ constexpr uint32_t OFF_Z = 2 * BUF_BYTES;  // 2 x z bf16 [64 t][128], plain row-
 constexpr uint32_t OFF_MISC = OFF_Z + 2 * 16384;
 constexpr uint32_t MISC_BYTES = 2048;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-// misc: 0 barriers, 128 TMEM slot, 256 reductions [4][64], 1280 rstd [64]
+// misc: 0 barriers, 256 TMEM slot, 512 reductions [4][64], 1536 rstd [64]
 // TMEM columns (32-bit, 128 lanes = v rows)
 constexpr uint32_t T_S = 0;                  // state f32 [128 v][128 k]
 constexpr uint32_t T_D0 = 128, T_D1 = 256;   // per buffer: U^T f32 [128][64] at +0, O^T at +64
 constexpr uint32_t T_S16 = 384;              // state f16, k pairs (A of MMA-A)
 constexpr uint32_t T_U16 = 448;              // U^T f16, t pairs (A of MMA-S and MMA7)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t LD_BYTES = 16384 + wy::REC_BYTES;
+constexpr uint32_t LD_BYTES = 3 * 16384 + 4 * 8192 + wy::REC_DEC_BYTES;
 constexpr uint32_t Z_BYTES = 64 * 128 * 2;
 constexpr uint32_t ID_P = idesc_f16_f32(128, 64, true, false, false);   // V^T (MN-major) x T1 (K-major)
 constexpr uint32_t ID_A = idesc_f16_f32(128, 128, false, false, false); // S16 x [-W ; Qs] (K-major)
@@ -87,12 +95,14 @@ constexpr int B_E = 8;      // + buffer: the epilogue has read and cleared O^T
 constexpr int B_FREE = 10;  // + buffer: every MMA that reads the buffer is complete
 constexpr int B_Z = 12;     // + z buffer: z tile landed
 constexpr int B_SS = 14;    // f32 state scaled by e^{G_C} (one arrive per converter warp)
-constexpr int kBars = 15;
+constexpr int B_PREP = 15;  // + buffer: Qs and K' ready (one arrive per preparer warp)
+constexpr int kBars = 17;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace chunk
 
 __global__ void __launch_bounds__(chunk::kThreads, 1)
-    gdn_chunk_kernel(const __grid_constant__ CUtensorMap tmV,
+    gdn_chunk_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmO,
                      const ChunkParams p) {
     using namespace chunk;
@@ -103,6 +113,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     const int n = blockIdx.y;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const int kap = h / (p.Vh / p.Kh);
     const int q4 = warp & 3;                  // TMEM lane quarter
     const int hf = (warp >> 2) & 1;           // column half within the group
     const int row = 32 * q4 + lane;           // v row of the state / output channel
@@ -110,9 +121,9 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
     uint8_t* misc = smem + OFF_MISC;
     uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc + 128);
-    float* s_red = reinterpret_cast<float*>(misc + 256);    // [4][64]
-    float* s_rstd = reinterpret_cast<float*>(misc + 1280);  // [64]
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc + 256);
+    float* s_red = reinterpret_cast<float*>(misc + 512);    // [4][64]
+    float* s_rstd = reinterpret_cast<float*>(misc + 1536);  // [64]
 
     int start, len;
     p.seq.bounds(n, start, len);
@@ -121,9 +132,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
     if (tid == 0) {
         for (int i = 0; i < kBars; ++i)
-            mbar_init(&bars[i], (i == B_UC || i == B_SC || i == B_SS) ? kCThreads / 32 : 1);
+            mbar_init(&bars[i], (i == B_UC || i == B_SC || i == B_SS) ? kCThreads / 32
+                                : (i == B_PREP || i == B_PREP + 1) ? kPThreads / 32
+                                                                   : 1);
         fence_barrier_init();
         prefetch_tensormap(&tmV);
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmZ);
         prefetch_tensormap(&tmO);
     }
@@ -146,12 +161,25 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         mbar_arrive_expect_tx(bar, LD_BYTES);
         tma_load_2d(B + BUF_V, &tmV, h * 128, y, bar);
         tma_load_2d(B + BUF_V + 8192, &tmV, h * 128 + 64, y, bar);
-        bulk_load(B + BUF_REC, rec_of(c), wy::REC_BYTES, bar);
+        tma_load_2d(B + BUF_WQ + 8192, &tmQ, kap * 128, y, bar);
+        tma_load_2d(B + BUF_WQ + 24576, &tmQ, kap * 128 + 64, y, bar);
+        tma_load_2d(B + BUF_KP, &tmK, kap * 128, y, bar);
+        tma_load_2d(B + BUF_KP + 8192, &tmK, kap * 128 + 64, y, bar);
+        const uint8_t* r = rec_of(c);
+        bulk_load(B + BUF_T1, r + wy::REC_T1, 8192, bar);
+        bulk_load(B + BUF_WQ, r + wy::REC_MW, 8192, bar);
+        bulk_load(B + BUF_WQ + 16384, r + wy::REC_MW + 8192, 8192, bar);
+        bulk_load(B + BUF_M, r + wy::REC_M, 8192, bar);
+        bulk_load(B + BUF_DEC, r + wy::REC_DEC, wy::REC_DEC_BYTES, bar);
     };
     auto prefetch_chunk = [&](int c) {
         const int y = start + c * C;
         prefetch_tma_2d(&tmV, h * 128, y);
         prefetch_tma_2d(&tmV, h * 128 + 64, y);
+        prefetch_tma_2d(&tmQ, kap * 128, y);
+        prefetch_tma_2d(&tmQ, kap * 128 + 64, y);
+        prefetch_tma_2d(&tmK, kap * 128, y);
+        prefetch_tma_2d(&tmK, kap * 128 + 64, y);
         prefetch_l2(rec_of(c), wy::REC_BYTES);
     };
     auto load_z = [&](int c) {
@@ -185,7 +213,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_f16(dacc(c), sw128_desc(B + BUF_V + s * 2048, 8192, 1024),
-                            sw128_desc(B + BUF_REC + wy::REC_T1 + s * 32, 16, 1024), ID_P, s > 0);
+                            sw128_desc(B + BUF_T1 + s * 32, 16, 1024), ID_P, s > 0);
             };
             wait1(B_LD, 0);
             tc_fence_after();
@@ -195,13 +223,14 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                 const uint32_t B = smem_u32(buf(c));
                 const uint32_t d = dacc(c);
                 wait1(B_E + b, (c >> 1) & 1);  // O^T[b] cleared
-                wait1(B_SC, c & 1);            // state of chunk c in f16 and scaled
+                wait1(B_SC, c & 1);            // state of chunk c in f16
+                wait1(B_PREP + b, (c >> 1) & 1);  // Qs and K' of chunk c
                 tc_fence_after();
                 // MMA-A: [U^T | O^T] += S0 [-W ; Qs]^T
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_f16_ta(d, tbase + T_S16 + 8 * s,
-                               sw128_desc(B + BUF_REC + wy::REC_WQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), ID_A,
+                               sw128_desc(B + BUF_WQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), ID_A,
                                1);
                 mma_commit(&bars[B_A]);
                 // U~ of the next chunk now if its inputs are in, else after MMA7
@@ -218,13 +247,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_f16_ta(tbase + T_S, tbase + T_U16 + 8 * s,
-                               sw128_desc(B + BUF_REC + wy::REC_KP + s * 2048, 8192, 1024), ID_S, 1);
+                               sw128_desc(B + BUF_KP + s * 2048, 8192, 1024), ID_S, 1);
                 mma_commit(&bars[B_SM]);
                 // MMA7: O^T += U^T M^T
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_f16_ta(d + 64, tbase + T_U16 + 8 * s,
-                               sw128_desc(B + BUF_REC + wy::REC_M + s * 32, 16, 1024), ID_7, 1);
+                               sw128_desc(B + BUF_M + s * 32, 16, 1024), ID_7, 1);
                 mma_commit(&bars[B_O + b]);
                 mma_commit(&bars[B_FREE + b]);
                 if (p_next) {
@@ -256,7 +285,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             float gC = 1.f;
             if (nchunks > 0) {
                 wait(B_LD, 0);
-                gC = *reinterpret_cast<const float*>(buf(0) + BUF_REC + wy::REC_GC);
+                gC = reinterpret_cast<const float*>(buf(0) + BUF_DEC)[128];
             }
             const float* src =
                 p.init_state ? p.init_state + (((size_t)n * p.Vh + h) * 128 + row) * 128 + 64 * hf : nullptr;
@@ -327,7 +356,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_SC]);
                 wait(B_LD + ((c + 1) & 1), ((c + 1) >> 1) & 1);
-                const float gC = *reinterpret_cast<const float*>(buf(c + 1) + BUF_REC + wy::REC_GC);
+                const float gC = reinterpret_cast<const float*>(buf(c + 1) + BUF_DEC)[128];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float v[32];
@@ -358,7 +387,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                         make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             }
         }
-    } else {
+    } else if (tid < kCThreads + kEThreads) {
         // =================================================================== epilogue
         const int et = tid - kCThreads;
         const int qt = (warp - 8) >> 2;                 // token quarter of this warp
@@ -449,6 +478,37 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             __syncwarp();
         }
         if (et == 32) bulk_wait_all();
+    } else {
+        // =================================================================== preparers
+        // Qs = diag(e^G) Q and K' = diag(e^{G_C - G}) K, in place; one row of 64 k per thread per block
+        const int pt = tid - (kCThreads + kEThreads);
+        const int which = pt >> 6;  // 0: Q rows, 1: K rows
+        const int t = pt & 63;
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            wait(B_LD + b, (c >> 1) & 1);
+            uint8_t* B = buf(c);
+            const float sc = reinterpret_cast<const float*>(B + BUF_DEC)[which ? t : 64 + t];
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+                uint8_t* tile = which ? B + BUF_KP + blk * 8192 : B + BUF_WQ + 8192 + blk * 16384;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint4* q = reinterpret_cast<uint4*>(tile + sw128_chunk(t, cc));
+                    uint4 v = *q;
+                    uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[e]));
+                        u[e] = pack_half2(f.x * sc, f.y * sc);
+                    }
+                    *q = v;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_PREP + b]);
+        }
     }
     tc_fence_before();
     __syncthreads();

@@ -9,10 +9,9 @@
 // T = (I + A)^-1, everything that does not involve the incoming state is
 //     T1 = T diag(beta)                 (U~ = T1 V)
 //     W  = T diag(beta e^G) K           (U = U~ - W S0^T)
-//     Qs = diag(e^G) Q                  (O = Qs S0^T + M U)
-//     K' = diag(e^{G_C - G}) K          (S_C = e^{G_C} S0 + U^T K')
 //     M  = tril_incl(Q K^T) * E,  E_ij = exp(G_i - G_j)
-// plus the chunk decay e^{G_C}.  None of it depends on the state,
+// plus the decays e^{G_t}, e^{G_C - G_t} and e^{G_C} (the recurrence kernel
+// scales Q and K by them: Qs = diag(e^G) Q, K' = diag(e^{G_C - G}) K).  None of it depends on the state,
 // so this kernel computes it for all (chunk, value head) pairs in parallel and
 // leaves a record per pair for the recurrence kernel (chunk.cuh).
 //
@@ -48,11 +47,11 @@ constexpr int LDA = 68;                   // f32 row stride of A / T
 // image of a 128-byte-swizzled shared-memory tile (row r, 16-byte chunk c at
 // r * 128 + ((c ^ (r & 7)) << 4)), so the reader moves them with plain bulk copies
 constexpr uint32_t REC_T1 = 0;            // T diag(beta)            f16 [64 t][64 j]
-constexpr uint32_t REC_WQ = 8192;         // per 64-k block b (at 16384 b): -W f16 [64 t][64 k], then Qs [64 t][64 k]
-constexpr uint32_t REC_M = 40960;         // tril_incl(Q K^T) * E    f16 [64 t][64 j]
-constexpr uint32_t REC_KP = 49152;        // K' f16 [64 t][64 k] x 2 blocks (k 0-63, then 64-127)
-constexpr uint32_t REC_GC = 65536;        // f32 e^{G_C} (16 bytes reserved)
-constexpr uint32_t REC_BYTES = 65552;
+constexpr uint32_t REC_MW = 8192;         // -W f16 [64 t][64 k] x 2 blocks (k 0-63, then 64-127)
+constexpr uint32_t REC_M = 24576;         // tril_incl(Q K^T) * E    f16 [64 t][64 j]
+constexpr uint32_t REC_DEC = 32768;       // f32 e^{G_C - G_t} [64], e^{G_t} [64], e^{G_C} (+ 12 bytes)
+constexpr uint32_t REC_DEC_BYTES = 528;
+constexpr uint32_t REC_BYTES = REC_DEC + REC_DEC_BYTES;
 // shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;            // [K t0-63 | Q t0-63] x k 0-63, then x k 64-127: f16 hi parts
 constexpr uint32_t OFF_LO = 32768;        // same layout, lo parts; then T diag(beta e^G) f16 per warpgroup
@@ -396,9 +395,13 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             }
             const float Gi = chunk_cumsum(gv, sG, wt, lane, wbar, 128);
             if (wt < 64) {
-                seG[wt] = expf(Gi);
+                const float e = expf(Gi);
+                seG[wt] = e;
                 sbeta[wt] = bv;
-                if (wt == 63) *reinterpret_cast<float*>(rec + REC_GC) = expf(Gi);
+                float* dec = reinterpret_cast<float*>(rec + REC_DEC);
+                dec[wt] = expf(sG[63] - Gi);
+                dec[64 + wt] = e;
+                if (wt == 63) dec[128] = e;
             }
             named_barrier_sync(wbar, 128);
         }
@@ -433,7 +436,6 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             // nothing to do for this slot; the input buffer is not read by it
             if (wt == 0) mbar_arrive(&bars[B_FREE]);
             __syncwarp();
-            named_barrier_sync(4, kThreads);
         } else {
             // ---- A (rows of K K^T) and M (rows of Q K^T), masked before the exp
             {
@@ -465,40 +467,9 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             }
             named_barrier_sync(wbar, 128);
 
-            // ---- Qs = diag(e^G) (Q hi + Q lo) and K' = diag(e^{G_C - G}) (K hi + K lo) to the record
-            {
-                const int t = wt >> 1, hh = wt & 1;
-                const float eg = seG[t], ek = expf(sG[63] - sG[t]);
-#pragma unroll
-                for (int which = 0; which < 2; ++which) {  // 0: Q rows, 1: K rows
-                    const uint32_t src = (which ? 0 : 8192) + hh * 16384;
-                    const uint8_t* xh = smem + OFF_KQ + src;
-                    const uint8_t* xl = smem + OFF_LO + src;
-                    uint8_t* dst = which ? rec + REC_KP + hh * 8192 : rec + REC_WQ + hh * 16384 + 8192;
-                    const float sc = which ? ek : eg;
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const uint32_t off = sw128_chunk(t, cc);
-                        const uint4 h4 = *reinterpret_cast<const uint4*>(xh + off);
-                        const uint4 l4 = *reinterpret_cast<const uint4*>(xl + off);
-                        const __half2* hp = reinterpret_cast<const __half2*>(&h4);
-                        const __half2* lp = reinterpret_cast<const __half2*>(&l4);
-                        uint4 o4;
-                        uint32_t* op = reinterpret_cast<uint32_t*>(&o4);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 fh = __half22float2(hp[e]), fl = __half22float2(lp[e]);
-                            op[e] = pack_half2((fh.x + fl.x) * sc, (fh.y + fl.y) * sc);
-                        }
-                        *reinterpret_cast<uint4*>(dst + off) = o4;
-                    }
-                }
-            }
-
             // ---- T = (I + A)^-1; T diag(beta) to the record, T diag(beta e^G) to shared memory
-            // (over the lo tiles, which every slot has read once barrier 4 is passed)
+            // (over the lo tiles, which only MMA1 reads)
             wy_tsolve(sA, sP, wt, wbar);
-            named_barrier_sync(4, kThreads);
             {
                 const int t = wt >> 1, hh = wt & 1;
                 const float* Tr = sA + t * LDA + 32 * hh;
@@ -541,7 +512,7 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         if (active) {
             wait(B_W + wg, ph);
             tc_fence_after();
-            uint8_t* dst = rec + REC_WQ + (row >> 6) * 16384 + (row & 7) * 2;
+            uint8_t* dst = rec + REC_MW + (row >> 6) * 8192 + (row & 7) * 2;
             const uint32_t kc = (row & 63) >> 3;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {

@@ -147,8 +147,8 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
  * library holds until the process exits.  A request whose scratch exceeds it
  * (gdn_prefill_workspace_size(dims, B, T) > GDN_NOALLOC_SCRATCH_BYTES) is
  * rejected with GDN_ERR_WORKSPACE before anything is enqueued; for the 27B
- * model's dims (16/48 heads) that is about 800 tokens per call (one row of
- * up to 832 tokens; 29,056 bytes per token plus 3,146,496 bytes per 64-token
+ * model's dims (16/48 heads) that is about 1,200 tokens per call (one row of
+ * up to 1216 tokens; 29,056 bytes per token plus 1,598,208 bytes per 64-token
  * chunk of a row).  The call itself allocates nothing.
  *
  * The first call on each device resolves the device address of the array

@@ -77,12 +77,12 @@ def test_noalloc_rejects_requests_beyond_its_scratch(dev):
     out = torch.empty((1, 4, 6144), dtype=torch.bfloat16, device=dev)
     fs = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
     fc = torch.empty((1, 3, 10240), dtype=torch.float32, device=dev)
-    # 1 row of 833 tokens needs more than the 64 MiB of fixed scratch (832 is the most
+    # 1 row of 1217 tokens needs more than the 64 MiB of fixed scratch (1216 is the most
     # one row gets); refused before any launch
     lib = gdn.load_library()
     size = lib.gdn_prefill_workspace_size
     size.restype = ctypes.c_size_t
     dc = gdn._dims_c(synth.MODEL)
-    assert size(ctypes.byref(dc), 1, 832) <= 64 * 1024 * 1024 < size(ctypes.byref(dc), 1, 833)
-    status = _call_noalloc(fn, 1, 833, w, acts, None, None, out, fs, fc)
+    assert size(ctypes.byref(dc), 1, 1216) <= 64 * 1024 * 1024 < size(ctypes.byref(dc), 1, 1217)
+    status = _call_noalloc(fn, 1, 1217, w, acts, None, None, out, fs, fc)
     assert status == GDN_ERR_WORKSPACE
