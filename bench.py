@@ -352,7 +352,8 @@ def bench_prefill(args, world, rank, local, T):
                              "algorithmic_flop_per_token": PREFILL_FLOP_PER_TOKEN},
                 "l2": "flushed (256 MiB write) before each timed call", "gpu_launches": launches}
 
-    out = {"b1": line(T, t1, f"prefill B=1 T={T}, zero initial state", 3 * n1)}
+    # launches per call: load stage, history out, WY records, recurrence (+ chunk offsets for packed rows)
+    out = {"b1": line(T, t1, f"prefill B=1 T={T}, zero initial state", 4 * n1)}
     if T == 8192:
         vcase = synth.config(3)
         vw = gdn.weights_to(vcase["weights"], dev)
@@ -368,7 +369,7 @@ def bench_prefill(args, world, rank, local, T):
                                                           cu_seqlens_dev=cud),
                                dev, stream, max(3, args.warmup), max(5, args.steps))
         out["varlen8"] = line(total, t2, f"varlen prefill 8 rows ({total} tokens, lengths U[512,16384]), "
-                                         "random initial state and history", 3 * n2)
+                                         "random initial state and history", 5 * n2)
     return out
 
 

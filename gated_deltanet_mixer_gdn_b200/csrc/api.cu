@@ -110,10 +110,158 @@ Workspace plan_workspace(const gdn_dims* d, int64_t total, int64_t N, int64_t nc
     return w;
 }
 
+// Internal streams of the overlapped dense prefill, one set per device: the
+// recurrence runs on a high-priority stream while the load stage and the WY
+// records of the next segment run on a low-priority one.  Created on the
+// first overlapped call on the device.
+constexpr int kMaxSegments = 8;
+struct SideStreams {
+    bool ready = false;
+    cudaStream_t prod = nullptr, chain = nullptr;
+    cudaEvent_t fork = nullptr, prod_done = nullptr, chain_done = nullptr;
+    cudaEvent_t seg[kMaxSegments] = {};
+};
+std::mutex g_side_mu;
+SideStreams g_side[kMaxDevices];
+
+int side_streams(int dev, SideStreams** out) {
+    if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+    SideStreams& st = g_side[dev];
+    if (!st.ready) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GDN_ERR_CUDA;
+        if (cudaStreamCreateWithPriority(&st.prod, cudaStreamNonBlocking, least) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&st.chain, cudaStreamNonBlocking, greatest) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        cudaEvent_t* evs[3] = {&st.fork, &st.prod_done, &st.chain_done};
+        for (cudaEvent_t* e : evs)
+            if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
+        for (auto& e : st.seg)
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
+        st.ready = true;
+    }
+    *out = &st;
+    return GDN_OK;
+}
+
+// Everything one prefill call launches, with the workspace carved and the
+// tensor maps built once.
+struct PrefillPlan {
+    int Kh, Vh, C, N, uniform_T, total, nsm;
+    SeqIndex seq;
+    const gdn_weights* w;
+    const uint16_t *qkv, *a, *b;
+    const float* init_conv;
+    float* final_conv;
+    uint16_t* out;
+    const float* norm_w;
+    __half *Qs, *Ks, *Ql, *Kl, *Vs;
+    float *Gs, *Bs;
+    int* chunk_base;
+    uint8_t* rec;
+    CUtensorMap mK, mQ, mKl, mQl, mV, mZ, mO;
+
+    int prep(int tok_begin, int tok_end, cudaStream_t st) const {
+        if (tok_end <= tok_begin) return GDN_OK;
+        PrepParams pp{};
+        pp.Kh = Kh;
+        pp.Vh = Vh;
+        pp.C = C;
+        pp.total = total;
+        pp.tok_begin = tok_begin;
+        pp.tok_end = tok_end;
+        pp.seq = seq;
+        pp.qkv = qkv;
+        pp.a = a;
+        pp.b = b;
+        pp.conv_w = w->conv_w;
+        pp.A_log = w->A_log;
+        pp.dt_bias = w->dt_bias;
+        pp.init_conv = init_conv;
+        pp.Qs = Qs;
+        pp.Ks = Ks;
+        pp.Ql = Ql;
+        pp.Kl = Kl;
+        pp.Vs = Vs;
+        pp.Gs = Gs;
+        pp.Bs = Bs;
+        dim3 grid((tok_end - tok_begin + kPrepTokens - 1) / kPrepTokens, (2 * Kh + Vh + kPrepSlots - 1) / kPrepSlots);
+        gdn_prep_kernel<<<grid, 256, 0, st>>>(pp);
+        return cuda_status(cudaGetLastError());
+    }
+    int conv_out(cudaStream_t st) const {
+        if (final_conv == nullptr) return GDN_OK;
+        ConvOutParams cp{};
+        cp.C = C;
+        cp.N = N;
+        cp.seq = seq;
+        cp.qkv = qkv;
+        cp.init_conv = init_conv;
+        cp.final_conv = final_conv;
+        dim3 grid((C + 255) / 256, N);
+        gdn_conv_out_kernel<<<grid, 256, 0, st>>>(cp);
+        return cuda_status(cudaGetLastError());
+    }
+    // WY records of nch chunks: all of them (win 0), or the window [c0, c0 + win) of every uniform row
+    int wy_records(int64_t nch, int c0, int win, int grid_cap, cudaStream_t st) const {
+        if (nch <= 0) return GDN_OK;
+        WyParams wp{};
+        wp.Kh = Kh;
+        wp.Vh = Vh;
+        wp.total = total;
+        wp.seq = seq;
+        wp.chunk_base = chunk_base;
+        wp.nchunks = (int)nch;
+        wp.c0 = c0;
+        wp.win = win;
+        wp.Gs = Gs;
+        wp.Bs = Bs;
+        wp.rec = rec;
+        static std::once_flag once;
+        static cudaError_t err = cudaSuccess;
+        std::call_once(once, [] {
+            err = cudaFuncSetAttribute(gdn_wy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wy::SMEM_BYTES);
+        });
+        if (err != cudaSuccess) return GDN_ERR_CUDA;
+        const int ratio = Vh / Kh;
+        const int64_t ntasks = nch * Kh * ((ratio + wy::kHeads - 1) / wy::kHeads);
+        const int grid = (int)(ntasks < grid_cap ? ntasks : grid_cap);
+        gdn_wy_kernel<<<grid, wy::kThreads, wy::SMEM_BYTES, st>>>(mK, mQ, mKl, mQl, wp);
+        return cuda_status(cudaGetLastError());
+    }
+    // the recurrence over the chunk window [c0, c1) of every row (c1 < 0: to the end)
+    int recurrence(int c0, int c1, const float* init_state, float* final_state, cudaStream_t st) const {
+        ChunkParams cp{};
+        cp.Kh = Kh;
+        cp.Vh = Vh;
+        cp.total = total;
+        cp.seq = seq;
+        cp.chunk_base = chunk_base;
+        cp.rec = rec;
+        cp.init_state = init_state;
+        cp.final_state = final_state;
+        cp.norm_w = norm_w;
+        cp.out = out;
+        cp.c0 = c0;
+        cp.c1 = c1;
+        static std::once_flag once;
+        static cudaError_t err = cudaSuccess;
+        std::call_once(once, [] {
+            err = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)chunk::SMEM_BYTES);
+        });
+        if (err != cudaSuccess) return GDN_ERR_CUDA;
+        dim3 grid(Vh, N);
+        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, st>>>(mV, mQ, mK, mZ, mO, cp);
+        return cuda_status(cudaGetLastError());
+    }
+};
+
 int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32_t* cu_dev, int32_t uniform_T,
-                 int32_t total, int64_t nchunks, int64_t nchunks_planned, const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
-                 const float* init_state, const float* init_conv, uint16_t* out, float* final_state,
-                 float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                 int32_t total, int64_t nchunks, int64_t nchunks_planned, const uint16_t* qkv, const uint16_t* z,
+                 const uint16_t* a, const uint16_t* b, const float* init_state, const float* init_conv, uint16_t* out,
+                 float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                 bool may_overlap) {
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
     const int C = (2 * Kh + Vh) * 128;
     const size_t state_bytes = (size_t)N * Vh * 128 * 128 * 4;
@@ -141,130 +289,109 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     if (workspace == nullptr || workspace_bytes < ws.bytes) return GDN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
-    __half* Qs = reinterpret_cast<__half*>(wsb + ws.off_q);
-    __half* Ks = reinterpret_cast<__half*>(wsb + ws.off_k);
-    __half* Ql = reinterpret_cast<__half*>(wsb + ws.off_ql);
-    __half* Kl = reinterpret_cast<__half*>(wsb + ws.off_kl);
-    __half* Vs = reinterpret_cast<__half*>(wsb + ws.off_v);
-    float* Gs = reinterpret_cast<float*>(wsb + ws.off_g);
-    float* Bs = reinterpret_cast<float*>(wsb + ws.off_b);
-    int* chunk_base = cu_dev ? reinterpret_cast<int*>(wsb + ws.off_cb) : nullptr;
-    uint8_t* rec = wsb + ws.off_rec;
-
-    // 1. load stage: conv + silu, L2 norms, gates
-    {
-        PrepParams pp{};
-        pp.Kh = Kh;
-        pp.Vh = Vh;
-        pp.C = C;
-        pp.total = total;
-        pp.seq = seq;
-        pp.qkv = qkv;
-        pp.a = a;
-        pp.b = b;
-        pp.conv_w = w->conv_w;
-        pp.A_log = w->A_log;
-        pp.dt_bias = w->dt_bias;
-        pp.init_conv = init_conv;
-        pp.Qs = Qs;
-        pp.Ks = Ks;
-        pp.Ql = Ql;
-        pp.Kl = Kl;
-        pp.Vs = Vs;
-        pp.Gs = Gs;
-        pp.Bs = Bs;
-        dim3 grid((total + kPrepTokens - 1) / kPrepTokens, (2 * Kh + Vh + kPrepSlots - 1) / kPrepSlots);
-        gdn_prep_kernel<<<grid, 256, 0, stream>>>(pp);
-        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    }
-    // 2. final conv history (after the load stage has read the initial one)
-    if (final_conv != nullptr) {
-        ConvOutParams cp{};
-        cp.C = C;
-        cp.N = N;
-        cp.seq = seq;
-        cp.qkv = qkv;
-        cp.init_conv = init_conv;
-        cp.final_conv = final_conv;
-        dim3 grid((C + 255) / 256, N);
-        gdn_conv_out_kernel<<<grid, 256, 0, stream>>>(cp);
-        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    }
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
-    CUtensorMap mK, mQ, mKl, mQl, mV, mZ, mO;
-    if (!make_map(&mK, Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+
+    PrefillPlan P{};
+    P.Kh = Kh;
+    P.Vh = Vh;
+    P.C = C;
+    P.N = N;
+    P.uniform_T = uniform_T;
+    P.total = total;
+    P.nsm = nsm;
+    P.seq = seq;
+    P.w = w;
+    P.qkv = qkv;
+    P.a = a;
+    P.b = b;
+    P.init_conv = init_conv;
+    P.final_conv = final_conv;
+    P.out = out;
+    P.norm_w = w->norm_w;
+    P.Qs = reinterpret_cast<__half*>(wsb + ws.off_q);
+    P.Ks = reinterpret_cast<__half*>(wsb + ws.off_k);
+    P.Ql = reinterpret_cast<__half*>(wsb + ws.off_ql);
+    P.Kl = reinterpret_cast<__half*>(wsb + ws.off_kl);
+    P.Vs = reinterpret_cast<__half*>(wsb + ws.off_v);
+    P.Gs = reinterpret_cast<float*>(wsb + ws.off_g);
+    P.Bs = reinterpret_cast<float*>(wsb + ws.off_b);
+    P.chunk_base = cu_dev ? reinterpret_cast<int*>(wsb + ws.off_cb) : nullptr;
+    P.rec = wsb + ws.off_rec;
+    if (!make_map(&P.mK, P.Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mKl, Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+        !make_map(&P.mKl, P.Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mQl, Ql, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+        !make_map(&P.mQl, P.Ql, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mQ, Qs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
+        !make_map(&P.mQ, P.Qs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mV, Vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Vh * 128, total, 64, 64,
+        !make_map(&P.mV, P.Vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Vh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
+        !make_map(&P.mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mO, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
+        !make_map(&P.mO, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return GDN_ERR_CUDA;
-    // 3. first chunk of every row (packed rows only)
-    if (chunk_base != nullptr) {
-        gdn_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu_dev, N, chunk_base);
+
+    // Overlapped schedule (dense rows that leave most SMs idle during the recurrence):
+    // the rows' chunks are cut into S segments; the load stage and the WY records of
+    // segment s+1 run on the low-priority stream while the recurrence of segment s runs
+    // on the high-priority one, each segment's recurrence starting from the state the
+    // previous one left in final_state.
+    const int per = cu_dev ? 0 : (uniform_T + 63) / 64;
+    const int chain_ctas = N * Vh;
+    int S = 1;
+    if (may_overlap && cu_dev == nullptr && final_state != nullptr && chain_ctas + 32 <= nsm && per >= 16)
+        S = per >= 4 * kMaxSegments ? 4 : 2;
+    if (S > 1) {
+        std::lock_guard<std::mutex> lock(g_side_mu);
+        SideStreams* ss = nullptr;
+        int st = side_streams(dev, &ss);
+        if (st != GDN_OK) return st;
+        if (cudaEventRecord(ss->fork, stream) != cudaSuccess || cudaStreamWaitEvent(ss->prod, ss->fork, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(ss->chain, ss->fork, 0) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        int cs[kMaxSegments + 1];
+        for (int k = 0; k <= S; ++k) cs[k] = (int)((int64_t)k * per / S);
+        for (int k = 0; k < S; ++k) {
+            // load stage of the segment's tokens in every row
+            for (int n = 0; n < N; ++n) {
+                const int t0 = n * uniform_T + cs[k] * 64;
+                const int t1 = n * uniform_T + (cs[k + 1] * 64 < uniform_T ? cs[k + 1] * 64 : uniform_T);
+                if ((st = P.prep(t0, t1, ss->prod)) != GDN_OK) return st;
+            }
+            const int win = cs[k + 1] - cs[k];
+            const int cap = k == 0 ? nsm : nsm - chain_ctas;  // leave the recurrence its SMs
+            if ((st = P.wy_records((int64_t)N * win, cs[k], win, cap, ss->prod)) != GDN_OK) return st;
+            if (cudaEventRecord(ss->seg[k], ss->prod) != cudaSuccess ||
+                cudaStreamWaitEvent(ss->chain, ss->seg[k], 0) != cudaSuccess)
+                return GDN_ERR_CUDA;
+            if ((st = P.recurrence(cs[k], k + 1 < S ? cs[k + 1] : -1, k == 0 ? init_state : final_state, final_state,
+                                   ss->chain)) != GDN_OK)
+                return st;
+        }
+        if ((st = P.conv_out(ss->prod)) != GDN_OK) return st;  // after every load-stage launch read the history
+        if (cudaEventRecord(ss->prod_done, ss->prod) != cudaSuccess ||
+            cudaEventRecord(ss->chain_done, ss->chain) != cudaSuccess ||
+            cudaStreamWaitEvent(stream, ss->prod_done, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(stream, ss->chain_done, 0) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        return GDN_OK;
+    }
+
+    // Plain schedule on the caller's stream.
+    int st = P.prep(0, total, stream);  // 1. load stage: conv + silu, L2 norms, gates
+    if (st != GDN_OK) return st;
+    if ((st = P.conv_out(stream)) != GDN_OK) return st;  // 2. final history (after the load stage read it)
+    if (P.chunk_base != nullptr) {                        // 3. first chunk of every packed row
+        gdn_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu_dev, N, P.chunk_base);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
-    // 4. per-chunk WY records, all chunks in parallel
-    if (nchunks > 0) {
-        WyParams wp{};
-        wp.Kh = Kh;
-        wp.Vh = Vh;
-        wp.total = total;
-        wp.seq = seq;
-        wp.chunk_base = chunk_base;
-        wp.nchunks = (int)nchunks;
-        wp.Gs = Gs;
-        wp.Bs = Bs;
-        wp.rec = rec;
-        static std::once_flag wy_once;
-        static cudaError_t wy_err = cudaSuccess;
-        std::call_once(wy_once, [] {
-            wy_err = cudaFuncSetAttribute(gdn_wy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)wy::SMEM_BYTES);
-        });
-        if (wy_err != cudaSuccess) return GDN_ERR_CUDA;
-        const int ratio = Vh / Kh;
-        const int64_t ntasks = nchunks * Kh * ((ratio + wy::kHeads - 1) / wy::kHeads);
-        const int grid = (int)(ntasks < nsm ? ntasks : nsm);
-        gdn_wy_kernel<<<grid, wy::kThreads, wy::SMEM_BYTES, stream>>>(mK, mQ, mKl, mQl, wp);
-        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    }
-    // 5. the state recurrence, gated RMSNorm epilogue
-    {
-        ChunkParams cp{};
-        cp.Kh = Kh;
-        cp.Vh = Vh;
-        cp.total = total;
-        cp.seq = seq;
-        cp.chunk_base = chunk_base;
-        cp.rec = rec;
-        cp.init_state = init_state;
-        cp.final_state = final_state;
-        cp.norm_w = w->norm_w;
-        cp.out = out;
-        static std::once_flag attr_once;
-        static cudaError_t attr_err = cudaSuccess;
-        std::call_once(attr_once, [] {
-            attr_err = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)chunk::SMEM_BYTES);
-        });
-        if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
-        dim3 grid(Vh, N);
-        gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, stream>>>(mV, mQ, mK, mZ, mO, cp);
-        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    }
-    return GDN_OK;
+    if ((st = P.wy_records(nchunks, 0, 0, nsm, stream)) != GDN_OK) return st;  // 4. WY records, all chunks
+    return P.recurrence(0, -1, init_state, final_state, stream);              // 5. recurrence + gated norm
 }
 
 int check_io(int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
@@ -336,7 +463,7 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
     if ((st = check_device()) != GDN_OK) return st;
     const int64_t nch = (int64_t)B * ((T + 63) / 64);
     return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, a, b, init_state, init_conv, out,
-                        final_state, final_conv, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+                        final_state, final_conv, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), true);
 }
 
 int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_host,
@@ -360,7 +487,7 @@ int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, co
     for (int32_t i = 0; i < N; ++i) nch += (cu_host[i + 1] - cu_host[i] + 63) / 64;
     return prefill_impl(dims, w, N, cu_dev, 0, total_T, nch, chunk_bound(N, total_T), qkv, z, a, b, init_state,
                         init_conv, out, final_state, final_conv, workspace, workspace_bytes,
-                        static_cast<cudaStream_t>(stream));
+                        static_cast<cudaStream_t>(stream), false);
 }
 
 int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const uint16_t* qkv, const uint16_t* z,
@@ -432,7 +559,7 @@ int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, i
     if ((st = noalloc_scratch(&scratch)) != GDN_OK) return st;
     return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, a, b, init_state, init_conv, out,
                         final_state, final_conv, scratch, (size_t)GDN_NOALLOC_SCRATCH_BYTES,
-                        static_cast<cudaStream_t>(stream));
+                        static_cast<cudaStream_t>(stream), false);
 }
 
 int gdn_last_device_error(void) {

@@ -45,6 +45,7 @@ struct ChunkParams {
     float* final_state;       // f32 [N][Vh][128][128] or nullptr (may alias init_state)
     const float* norm_w;      // f32 [128]
     uint16_t* out;            // bf16 [total][Vh*128]
+    int c0, c1;               // chunk window [c0, c1) of every row (c1 < 0: to the end of the row)
 };
 
 namespace chunk {
@@ -127,8 +128,12 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
     int start, len;
     p.seq.bounds(n, start, len);
-    const int nchunks = (len + C - 1) / C;
-    const int cbase = p.chunk_base ? __ldg(p.chunk_base + n) : n * ((p.seq.uniform_T + C - 1) / C);
+    // the chunks [cw, cw + nchunks) of the row; loop indices below count from cw
+    const int cw = min(p.c0, (len + C - 1) / C);
+    const int nchunks = max(0, (p.c1 < 0 ? (len + C - 1) / C : min(p.c1, (len + C - 1) / C)) - cw);
+    const int cbase = (p.chunk_base ? __ldg(p.chunk_base + n) : n * ((p.seq.uniform_T + C - 1) / C)) + cw;
+    start += cw * C;
+    len -= cw * C;
 
     if (tid == 0) {
         for (int i = 0; i < kBars; ++i)

@@ -52,6 +52,7 @@ struct SeqIndex {
 
 struct PrepParams {
     int Kh, Vh, C, total;
+    int tok_begin, tok_end;   // tokens processed by this launch
     SeqIndex seq;
     const uint16_t* qkv;      // bf16 [total][C]
     const uint16_t* a;        // bf16 [total][Vh]
@@ -95,8 +96,8 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
     const bool is_q = slot < p.Kh;
     const bool is_v = slot >= 2 * p.Kh;
     const int vh = slot - 2 * p.Kh;
-    const int t0 = blockIdx.x * kPrepTokens;
-    const int nt = min(kPrepTokens, p.total - t0);
+    const int t0 = p.tok_begin + blockIdx.x * kPrepTokens;
+    const int nt = min(kPrepTokens, p.tok_end - t0);
     if (nt <= 0) return;  // whole CTA
 
     uint2 ahead[kPrepAhead];

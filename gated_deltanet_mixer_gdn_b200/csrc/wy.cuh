@@ -32,7 +32,8 @@ struct WyParams {
     int Kh, Vh, total;
     SeqIndex seq;
     const int* chunk_base;  // [N+1] first chunk of each row (varlen), or nullptr for uniform rows
-    int nchunks;            // chunks over all rows
+    int nchunks;            // chunks to process (all rows, or N * win for a window)
+    int c0, win;            // uniform rows only: the chunk window [c0, c0 + win) of every row (win 0: all)
     const float* Gs;        // f32 [Vh][total] log-decay
     const float* Bs;        // f32 [Vh][total] write rate
     uint8_t* rec;           // records [nchunks][Vh] of wy::REC_BYTES
@@ -335,6 +336,10 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         const int r = task / nsub;
         kap = r % p.Kh;
         g = r / p.Kh;
+        if (p.win > 0) {  // window chunk -> chunk of the row
+            const int per = (p.seq.uniform_T + C - 1) / C;
+            g = (g / p.win) * per + p.c0 + g % p.win;
+        }
     };
     auto issue_loads = [&](int task) {
         int g, kap, sub, n, c;
