@@ -61,7 +61,7 @@ constexpr uint32_t WG_BYTES = 64 * LDA * 4 + 32 * 36 * 4;
 constexpr uint32_t OFF_MISC = OFF_WG + kHeads * WG_BYTES;
 constexpr uint32_t MISC_BYTES = 4096;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
-// misc: 0 barriers, 128 TMEM slot, 256 + 768 * wg: G[64], e^G[64], beta[64]
+// misc: 0 barriers, 128 TMEM slot, 256 + 1024 * wg: G[64], e^G[64], beta[64], column decays[64]
 constexpr uint32_t T_KQ = 0;              // [K;Q] K^T, 64 columns; then W^T of warpgroup w at 64 (w + 1)
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t IN_BYTES = 8 * 8192;
@@ -298,9 +298,10 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
     uint8_t* misc = smem + OFF_MISC;
     uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(misc + 128);
-    float* sG = reinterpret_cast<float*>(misc + 256 + 768 * wg);
+    float* sG = reinterpret_cast<float*>(misc + 256 + 1024 * wg);
     float* seG = sG + 64;
     float* sbeta = sG + 128;
+    float* scol = sG + 192;  // e^{G_r - G_j}, r the last token of j's 16-token block
     float* sA = reinterpret_cast<float*>(smem + OFF_WG + wg * WG_BYTES);
     float* sP = sA + 64 * LDA;
     uint8_t* sT2 = smem + OFF_LO + 8192 * wg;
@@ -376,6 +377,27 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         }
     };
 
+    // gate inputs of a task (value head slot of this warpgroup, token wt), loaded a task ahead
+    auto load_gates = [&](int task, float& gv, float& bv) {
+        gv = 0.f;
+        bv = 0.f;
+        if (task >= ntasks || wt >= C) return;
+        int g, kap, sub, n, c;
+        task_coords(task, g, kap, sub);
+        chunk_row(p, g, n, c);
+        const int hslot = sub * kHeads + wg;
+        if (hslot >= ratio) return;
+        int start, len;
+        p.seq.bounds(n, start, len);
+        if (wt < min(C, len - c * C)) {
+            const size_t off = (size_t)(kap * ratio + hslot) * p.total + start + c * C + wt;
+            gv = __ldg(p.Gs + off);
+            bv = __ldg(p.Bs + off);
+        }
+    };
+    float gv_next, bv_next;
+    load_gates(blockIdx.x, gv_next, bv_next);
+
     uint32_t it = 0;
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x, ++it) {
         const uint32_t ph = it & 1;
@@ -391,27 +413,12 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         const int h = kap * ratio + hslot;
         uint8_t* rec = p.rec + ((size_t)g * p.Vh + h) * REC_BYTES;
 
-        // ---- gates: G, e^G, beta; the decay part of the record
-        if (active) {
-            float gv = 0.f, bv = 0.f;
-            if (wt < nv) {
-                gv = __ldg(p.Gs + (size_t)h * p.total + tok0 + wt);
-                bv = __ldg(p.Bs + (size_t)h * p.total + tok0 + wt);
-            }
-            const float Gi = chunk_cumsum(gv, sG, wt, lane, wbar, 128);
-            if (wt < 64) {
-                const float e = expf(Gi);
-                seG[wt] = e;
-                sbeta[wt] = bv;
-                float* dec = reinterpret_cast<float*>(rec + REC_DEC);
-                dec[wt] = expf(sG[63] - Gi);
-                dec[64 + wt] = e;
-                if (wt == 63) dec[128] = e;
-            }
-            named_barrier_sync(wbar, 128);
-        }
+        const float gv = gv_next, bv = bv_next;
+        load_gates(task + gridDim.x, gv_next, bv_next);
+        (void)tok0;
+        (void)nv;
 
-        // ---- MMA1: [K;Q] K^T from hi/lo f16 parts
+        // ---- MMA1: [K;Q] K^T from hi/lo f16 parts (runs while the gates are formed)
         if (tid == 0) {
             wait1(B_IN, ph);
             tc_fence_after();
@@ -434,6 +441,22 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             mma_commit(&bars[B_MMA1]);
         }
         __syncwarp();
+
+        // ---- gates: G, e^G, beta, the column decays; the decay part of the record
+        if (active) {
+            const float Gi = chunk_cumsum(gv, sG, wt, lane, wbar, 128);
+            if (wt < 64) {
+                const float e = expf(Gi);
+                seG[wt] = e;
+                sbeta[wt] = bv;
+                scol[wt] = expf(sG[wt | 15] - Gi);
+                float* dec = reinterpret_cast<float*>(rec + REC_DEC);
+                dec[wt] = expf(sG[63] - Gi);
+                dec[64 + wt] = e;
+                if (wt == 63) dec[128] = e;
+            }
+            named_barrier_sync(wbar, 128);
+        }
         wait(B_MMA1, ph);
         tc_fence_after();
 
@@ -447,7 +470,18 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
                 const bool is_a = row < 64;
                 const int i = is_a ? row : row - 64;
                 const int last = is_a ? i - 1 : i;  // last unmasked column
+                const int I = i >> 4;               // 16-token block of the row
                 const float Gr = sG[i], scale = is_a ? sbeta[i] : 1.f;
+                // e^{G_i - G_j} = e^{G_i - G_r} e^{G_r - G_j} for j in an earlier block (r its last
+                // token, both factors <= 1); direct exponentials inside the row's own block
+                float rowf[3], diag[16];
+#pragma unroll
+                for (int J = 0; J < 3; ++J) rowf[J] = (J < I) ? scale * __expf(Gr - sG[16 * J + 15]) : 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const int j = 16 * I + m;
+                    diag[m] = (j <= last) ? scale * __expf(Gr - sG[j]) : 0.f;
+                }
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
@@ -457,8 +491,9 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = 32 * hh + jj;
-                        const float d = __expf(Gr - sG[j]);  // (masked below; the branch-free form overlaps)
-                        e[jj] = (j <= last) ? scale * d * v[jj] : 0.f;
+                        const int J = j >> 4;
+                        const float f = (J < 3 && J < I) ? rowf[J < 3 ? J : 0] * scol[j] : 0.f;
+                        e[jj] = ((J == I) ? diag[j & 15] : f) * v[jj];
                     }
                     if (is_a) {
                         float4* dst = reinterpret_cast<float4*>(sA + i * LDA + 32 * hh);
