@@ -72,13 +72,11 @@ constexpr int kBars = B_W + kHeads;
 }  // namespace wy
 
 // ---- warp-level TF32 tensor-core products for the triangular solve.
-// x = hi + lo with hi, lo representable in tf32; hi*hi + hi*lo + lo*hi
-// recovers an f32-accurate product (the lo*lo term is below f32 rounding).
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+// x = hi + lo with hi = x truncated to the 19 bits a tf32 operand carries (a
+// bit mask on the integer pipe) and lo = x - hi (exact in f32; the tensor core
+// keeps its top 19 bits); hi*hi + hi*lo + lo*hi recovers the product to about
+// 2^-21 relative (the lo*lo term and lo's own truncation are below that).
+__device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xffffe000u; }
 
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
     asm volatile(
@@ -102,8 +100,8 @@ __device__ __forceinline__ void warp_gemm_tf32x3(float (&acc)[NT][4], const floa
         uint32_t ah[4], al[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            ah[i] = to_tf32(af[i]);
-            al[i] = to_tf32(af[i] - __uint_as_float(ah[i]));
+            ah[i] = tf32_hi(af[i]);
+            al[i] = __float_as_uint(af[i] - __uint_as_float(ah[i]));
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -111,8 +109,8 @@ __device__ __forceinline__ void warp_gemm_tf32x3(float (&acc)[NT][4], const floa
             uint32_t bh[2], bl[2];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                bh[i] = to_tf32(bf[i]);
-                bl[i] = to_tf32(bf[i] - __uint_as_float(bh[i]));
+                bh[i] = tf32_hi(bf[i]);
+                bl[i] = __float_as_uint(bf[i] - __uint_as_float(bh[i]));
             }
             mma_tf32(cor[nt], al, bh);
             mma_tf32(cor[nt], ah, bl);
