@@ -558,8 +558,11 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
                 tmem_ld32(tlane + 64 * (wg + 1) + 32 * hh, v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    *reinterpret_cast<__half*>(dst + sw128_chunk(32 * hh + j, kc)) = __float2half_rn(-v[j]);
+                for (int j = 0; j < 32; j += 2) {  // one paired conversion for tokens j, j + 1
+                    const uint32_t pr = pack_half2(-v[j], -v[j + 1]);
+                    *reinterpret_cast<uint16_t*>(dst + sw128_chunk(32 * hh + j, kc)) = static_cast<uint16_t>(pr);
+                    *reinterpret_cast<uint16_t*>(dst + sw128_chunk(32 * hh + j + 1, kc)) = static_cast<uint16_t>(pr >> 16);
+                }
             }
             tc_fence_before();
         }
