@@ -337,10 +337,11 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         return GDN_ERR_CUDA;
 
     // Overlapped schedule (dense rows that leave most SMs idle during the recurrence):
-    // the rows' chunks are cut into S segments; the load stage and the WY records of
-    // segment s+1 run on the low-priority stream while the recurrence of segment s runs
-    // on the high-priority one, each segment's recurrence starting from the state the
-    // previous one left in final_state.
+    // the load stage runs over all tokens first; then the rows' chunks are cut into S
+    // segments and the WY records of segment s+1 run on the low-priority stream (a
+    // persistent grid that leaves the recurrence its SMs) while the recurrence of
+    // segment s runs on the high-priority one, each segment's recurrence starting from
+    // the state the previous one left in final_state.
     const int per = cu_dev ? 0 : (uniform_T + 63) / 64;
     const int chain_ctas = N * Vh;
     int S = 1;
@@ -356,13 +357,9 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
             return GDN_ERR_CUDA;
         int cs[kMaxSegments + 1];
         for (int k = 0; k <= S; ++k) cs[k] = (int)((int64_t)k * per / S);
+        if ((st = P.prep(0, total, ss->prod)) != GDN_OK) return st;
+        if ((st = P.conv_out(ss->prod)) != GDN_OK) return st;  // after the load stage read the history
         for (int k = 0; k < S; ++k) {
-            // load stage of the segment's tokens in every row
-            for (int n = 0; n < N; ++n) {
-                const int t0 = n * uniform_T + cs[k] * 64;
-                const int t1 = n * uniform_T + (cs[k + 1] * 64 < uniform_T ? cs[k + 1] * 64 : uniform_T);
-                if ((st = P.prep(t0, t1, ss->prod)) != GDN_OK) return st;
-            }
             const int win = cs[k + 1] - cs[k];
             const int cap = k == 0 ? nsm : nsm - chain_ctas;  // leave the recurrence its SMs
             if ((st = P.wy_records((int64_t)N * win, cs[k], win, cap, ss->prod)) != GDN_OK) return st;
@@ -373,7 +370,6 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                                    ss->chain)) != GDN_OK)
                 return st;
         }
-        if ((st = P.conv_out(ss->prod)) != GDN_OK) return st;  // after every load-stage launch read the history
         if (cudaEventRecord(ss->prod_done, ss->prod) != cudaSuccess ||
             cudaEventRecord(ss->chain_done, ss->chain) != cudaSuccess ||
             cudaStreamWaitEvent(stream, ss->prod_done, 0) != cudaSuccess ||
