@@ -26,8 +26,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen_workspace_size",
-           "gdn_prefill_varlen", "gdn_decode", "gdn_prefill_noalloc", "gdn_last_device_error",
-           "gdn_status_string", "gdn_version")
+           "gdn_prefill_varlen", "gdn_decode", "gdn_decode_slots", "gdn_prefill_varlen_slots",
+           "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string", "gdn_version")
 
 GDN_OK = 0
 
@@ -71,6 +71,11 @@ def load_library() -> ctypes.CDLL:
         L.gdn_prefill_varlen.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_decode.argtypes = [dp, wp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.gdn_decode_slots.restype = ctypes.c_int
+        L.gdn_decode_slots.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.gdn_prefill_varlen_slots.restype = ctypes.c_int
+        L.gdn_prefill_varlen_slots.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp,
+                                               vp, sz, vp]
         L.gdn_last_device_error.restype = ctypes.c_int
         L.gdn_last_device_error.argtypes = []
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -226,6 +231,71 @@ def decode(qkv, z, a, b, weights, state, conv, *, out=None, dims: Dims = MODEL):
     return out
 
 
+def _slot_tables(slots, n, dev):
+    if isinstance(slots, torch.Tensor):
+        host = slots.detach().to("cpu", torch.int32).contiguous()
+    else:
+        host = torch.tensor(list(slots), dtype=torch.int32)
+    if host.numel() != n:
+        raise ValueError("one slot per row")
+    return host, host.to(dev)
+
+
+def decode_slots(slots, qkv, z, a, b, weights, state_pool, conv_pool, *, out=None, dims: Dims = MODEL):
+    """One token for each of `rows` rows, row r on pool row slots[r] (int32, host or CUDA
+    tensor or list).  state_pool f32 [P,Vh,D,D] and conv_pool f32 [P,W-1,C] are updated in
+    place.  Returns out [rows,Vh*D]."""
+    dev = _device_of(qkv)
+    L = load_library()
+    rows = int(qkv.shape[0])
+    for t, dt, nm in ((qkv, torch.bfloat16, "qkv"), (z, torch.bfloat16, "z"), (a, torch.bfloat16, "a"),
+                      (b, torch.bfloat16, "b"), (state_pool, torch.float32, "state_pool"),
+                      (conv_pool, torch.float32, "conv_pool")):
+        _need(t, dt, nm, dev)
+    host, devs = _slot_tables(slots, rows, dev)
+    if out is None:
+        out = torch.empty((rows, dims.value_width), dtype=torch.bfloat16, device=dev)
+    dc = _dims_c(dims)
+    st = L.gdn_decode_slots(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), rows,
+                            ctypes.c_void_p(host.data_ptr()), _ptr(devs), int(state_pool.shape[0]),
+                            _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(state_pool), _ptr(conv_pool), _ptr(out),
+                            _stream(dev))
+    _check(st, "gdn_decode_slots")
+    return out
+
+
+def prefill_varlen_slots(cu_seqlens, slots, qkv, z, a, b, weights, state_pool, conv_pool, *, out=None,
+                         dims: Dims = MODEL):
+    """Packed prefill of N rows, row n starting from and updating pool row slots[n] in place.
+    Returns out [total,Vh*D]."""
+    dev = _device_of(qkv)
+    L = load_library()
+    if isinstance(cu_seqlens, torch.Tensor):
+        cu_host = cu_seqlens.detach().to("cpu", torch.int32).contiguous()
+    else:
+        cu_host = torch.tensor(list(cu_seqlens), dtype=torch.int32)
+    N = int(cu_host.numel()) - 1
+    total = int(qkv.shape[0])
+    for t, dt, nm in ((qkv, torch.bfloat16, "qkv"), (z, torch.bfloat16, "z"), (a, torch.bfloat16, "a"),
+                      (b, torch.bfloat16, "b"), (state_pool, torch.float32, "state_pool"),
+                      (conv_pool, torch.float32, "conv_pool")):
+        _need(t, dt, nm, dev)
+    host, devs = _slot_tables(slots, N, dev)
+    cu_dev = cu_host.to(dev)
+    if out is None:
+        out = torch.empty((total, dims.value_width), dtype=torch.bfloat16, device=dev)
+    dc = _dims_c(dims)
+    ws_bytes = L.gdn_prefill_varlen_workspace_size(ctypes.byref(dc), N, total)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    st = L.gdn_prefill_varlen_slots(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), N,
+                                    ctypes.c_void_p(cu_host.data_ptr()), _ptr(cu_dev), total,
+                                    ctypes.c_void_p(host.data_ptr()), _ptr(devs), int(state_pool.shape[0]),
+                                    _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(state_pool), _ptr(conv_pool),
+                                    _ptr(out), _ptr(ws), ws_bytes, _stream(dev))
+    _check(st, "gdn_prefill_varlen_slots")
+    return out
+
+
 def last_device_error() -> int:
     return load_library().gdn_last_device_error()
 
@@ -234,5 +304,5 @@ def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tens
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_varlen", "decode", "last_device_error", "status_string", "load_library",
+__all__ = ["prefill", "prefill_varlen", "decode", "decode_slots", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/gdn.h"
 #include "chunk.cuh"
@@ -155,6 +156,7 @@ struct PrefillPlan {
     float* final_conv;
     uint16_t* out;
     const float* norm_w;
+    const int* slots;  // state / history row of each packed row, or nullptr
     __half *Qs, *Ks, *Ql, *Kl, *Vs;
     float *Gs, *Bs;
     int* chunk_base;
@@ -178,6 +180,7 @@ struct PrefillPlan {
         pp.A_log = w->A_log;
         pp.dt_bias = w->dt_bias;
         pp.init_conv = init_conv;
+        pp.slots = slots;
         pp.Qs = Qs;
         pp.Ks = Ks;
         pp.Ql = Ql;
@@ -198,6 +201,7 @@ struct PrefillPlan {
         cp.qkv = qkv;
         cp.init_conv = init_conv;
         cp.final_conv = final_conv;
+        cp.slots = slots;
         dim3 grid((C + 255) / 256, N);
         gdn_conv_out_kernel<<<grid, 256, 0, st>>>(cp);
         return cuda_status(cudaGetLastError());
@@ -244,6 +248,7 @@ struct PrefillPlan {
         cp.out = out;
         cp.c0 = c0;
         cp.c1 = c1;
+        cp.slots = slots;
         static std::once_flag once;
         static cudaError_t err = cudaSuccess;
         std::call_once(once, [] {
@@ -261,7 +266,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                  int32_t total, int64_t nchunks, int64_t nchunks_planned, const uint16_t* qkv, const uint16_t* z,
                  const uint16_t* a, const uint16_t* b, const float* init_state, const float* init_conv, uint16_t* out,
                  float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-                 bool may_overlap) {
+                 bool may_overlap, const int32_t* slots_dev = nullptr) {
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
     const int C = (2 * Kh + Vh) * 128;
     const size_t state_bytes = (size_t)N * Vh * 128 * 128 * 4;
@@ -311,6 +316,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     P.final_conv = final_conv;
     P.out = out;
     P.norm_w = w->norm_w;
+    P.slots = slots_dev;
     P.Qs = reinterpret_cast<__half*>(wsb + ws.off_q);
     P.Ks = reinterpret_cast<__half*>(wsb + ws.off_k);
     P.Ql = reinterpret_cast<__half*>(wsb + ws.off_ql);
@@ -428,6 +434,69 @@ int noalloc_scratch(void** out) {
     return GDN_OK;
 }
 
+// Host check of a slot table: 0 <= slots[r] < pool_rows, no slot twice.
+int check_slots(const int32_t* slots_host, int32_t rows, int32_t pool_rows) {
+    if (slots_host == nullptr || pool_rows <= 0) return GDN_ERR_INVALID_ARG;
+    std::vector<unsigned char> seen((size_t)pool_rows, 0);
+    for (int32_t r = 0; r < rows; ++r) {
+        const int32_t sl = slots_host[r];
+        if (sl < 0 || sl >= pool_rows || seen[(size_t)sl]) return GDN_ERR_INVALID_ARG;
+        seen[(size_t)sl] = 1;
+    }
+    return GDN_OK;
+}
+
+// The decode launch: rows batch rows, state / history rows through slots (or nullptr).
+int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const uint16_t* qkv, const uint16_t* z,
+                const uint16_t* a, const uint16_t* b, float* state, float* conv, uint16_t* out, const int32_t* slots,
+                void* stream) {
+    int st = GDN_OK;
+    if (!state || !conv || !aligned16(state) || !aligned16(conv)) return GDN_ERR_INVALID_ARG;
+    if ((st = check_io(rows, qkv, z, a, b, out, nullptr, nullptr, nullptr, nullptr)) != GDN_OK) return st;
+    if ((st = check_device()) != GDN_OK) return st;
+    DecodeParams p{};
+    p.Kh = dims->num_k_heads;
+    p.Vh = dims->num_v_heads;
+    p.C = (2 * p.Kh + p.Vh) * 128;
+    p.rows = rows;
+    p.qkv = qkv;
+    p.z = z;
+    p.a = a;
+    p.b = b;
+    p.conv_w = w->conv_w;
+    p.A_log = w->A_log;
+    p.dt_bias = w->dt_bias;
+    p.norm_w = w->norm_w;
+    p.state = state;
+    p.conv = conv;
+    p.out = out;
+    p.slots = slots;
+    static std::once_flag dec_once;
+    static cudaError_t dec_err = cudaSuccess;
+    std::call_once(dec_once, [] {
+        dec_err = cudaFuncSetAttribute(gdn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)dec::kSmemLimit);
+    });
+    if (dec_err != cudaSuccess) return GDN_ERR_CUDA;
+    const dec::Plan dplan = dec::plan(p.Vh / p.Kh);
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    // persistent grid: one CTA per SM walking (row, q/k head) items round-robin
+    p.nitems = rows * p.Kh;
+    const int grid = p.nitems < nsm ? p.nitems : nsm;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(dec::kThreads);
+    cfg.dynamicSmemBytes = dplan.smem_bytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cuda_status(cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p));
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -493,48 +562,51 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
     if ((st = check_weights(w)) != GDN_OK) return st;
     if (rows < 0 || rows > 65535) return GDN_ERR_INVALID_ARG;
     if (rows == 0) return GDN_OK;
-    if (!state || !conv || !aligned16(state) || !aligned16(conv)) return GDN_ERR_INVALID_ARG;
-    if ((st = check_io(rows, qkv, z, a, b, out, nullptr, nullptr, nullptr, nullptr)) != GDN_OK) return st;
+    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, stream);
+}
+
+
+int gdn_decode_slots(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const int32_t* slots_host,
+                     const int32_t* slots_dev, int32_t pool_rows, const uint16_t* qkv, const uint16_t* z,
+                     const uint16_t* a, const uint16_t* b, float* state_pool, float* conv_pool, uint16_t* out,
+                     void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (rows < 0 || rows > 65535) return GDN_ERR_INVALID_ARG;
+    if (rows == 0) return GDN_OK;
+    if ((st = check_slots(slots_host, rows, pool_rows)) != GDN_OK) return st;
+    if (slots_dev == nullptr || (reinterpret_cast<uintptr_t>(slots_dev) & 3u)) return GDN_ERR_INVALID_ARG;
+    return decode_impl(dims, w, rows, qkv, z, a, b, state_pool, conv_pool, out, slots_dev, stream);
+}
+
+int gdn_prefill_varlen_slots(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_host,
+                             const int32_t* cu_dev, int32_t total_T, const int32_t* slots_host,
+                             const int32_t* slots_dev, int32_t pool_rows, const uint16_t* qkv, const uint16_t* z,
+                             const uint16_t* a, const uint16_t* b, float* state_pool, float* conv_pool,
+                             uint16_t* out, void* workspace, size_t workspace_bytes, void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (N < 0 || N > 65535 || total_T < 0) return GDN_ERR_INVALID_ARG;
+    if (cu_host == nullptr || (N > 0 && cu_dev == nullptr)) return GDN_ERR_INVALID_ARG;
+    if (cu_host[0] != 0 || cu_host[N] != total_T) return GDN_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < N; ++i)
+        if (cu_host[i + 1] < cu_host[i]) return GDN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_dev) & 3u) != 0) return GDN_ERR_INVALID_ARG;
+    if (N == 0) return GDN_OK;
+    if ((st = check_slots(slots_host, N, pool_rows)) != GDN_OK) return st;
+    if (slots_dev == nullptr || (reinterpret_cast<uintptr_t>(slots_dev) & 3u)) return GDN_ERR_INVALID_ARG;
+    if (state_pool == nullptr || conv_pool == nullptr) return GDN_ERR_INVALID_ARG;
+    if ((st = check_io(total_T, qkv, z, a, b, out, state_pool, conv_pool, state_pool, conv_pool)) != GDN_OK)
+        return st;
     if ((st = check_device()) != GDN_OK) return st;
-    DecodeParams p{};
-    p.Kh = dims->num_k_heads;
-    p.Vh = dims->num_v_heads;
-    p.C = (2 * p.Kh + p.Vh) * 128;
-    p.rows = rows;
-    p.qkv = qkv;
-    p.z = z;
-    p.a = a;
-    p.b = b;
-    p.conv_w = w->conv_w;
-    p.A_log = w->A_log;
-    p.dt_bias = w->dt_bias;
-    p.norm_w = w->norm_w;
-    p.state = state;
-    p.conv = conv;
-    p.out = out;
-    static std::once_flag dec_once;
-    static cudaError_t dec_err = cudaSuccess;
-    std::call_once(dec_once, [] {
-        dec_err = cudaFuncSetAttribute(gdn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)dec::kSmemLimit);
-    });
-    if (dec_err != cudaSuccess) return GDN_ERR_CUDA;
-    const dec::Plan dplan = dec::plan(p.Vh / p.Kh);
-    int dev = 0, nsm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return GDN_ERR_CUDA;
-    // persistent grid: one CTA per SM walking (row, q/k head) items round-robin
-    p.nitems = rows * p.Kh;
-    const int grid = p.nitems < nsm ? p.nitems : nsm;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(dec::kThreads);
-    cfg.dynamicSmemBytes = dplan.smem_bytes;
-    cfg.stream = static_cast<cudaStream_t>(stream);
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
-    return cuda_status(cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p));
+    if (total_T == 0) return GDN_OK;  // the pool rows stay as they are
+    int64_t nch = 0;
+    for (int32_t i = 0; i < N; ++i) nch += (cu_host[i + 1] - cu_host[i] + 63) / 64;
+    return prefill_impl(dims, w, N, cu_dev, 0, total_T, nch, chunk_bound(N, total_T), qkv, z, a, b, state_pool,
+                        conv_pool, out, state_pool, conv_pool, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream), false, slots_dev);
 }
 
 int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, const uint16_t* qkv,

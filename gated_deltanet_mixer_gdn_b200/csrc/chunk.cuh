@@ -46,6 +46,7 @@ struct ChunkParams {
     const float* norm_w;      // f32 [128]
     uint16_t* out;            // bf16 [total][Vh*128]
     int c0, c1;               // chunk window [c0, c1) of every row (c1 < 0: to the end of the row)
+    const int* slots;         // [N] state row of each packed row (validated by the host), or nullptr
 };
 
 namespace chunk {
@@ -128,6 +129,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
     int start, len;
     p.seq.bounds(n, start, len);
+    const int srow = p.slots ? __ldg(p.slots + n) : n;  // state row
     // the chunks [cw, cw + nchunks) of the row; loop indices below count from cw
     const int cw = min(p.c0, (len + C - 1) / C);
     const int nchunks = max(0, (p.c1 < 0 ? (len + C - 1) / C : min(p.c1, (len + C - 1) / C)) - cw);
@@ -293,7 +295,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                 gC = reinterpret_cast<const float*>(buf(0) + BUF_DEC)[128];
             }
             const float* src =
-                p.init_state ? p.init_state + (((size_t)n * p.Vh + h) * 128 + row) * 128 + 64 * hf : nullptr;
+                p.init_state ? p.init_state + (((size_t)srow * p.Vh + h) * 128 + row) * 128 + 64 * hf : nullptr;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];
@@ -380,7 +382,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
         }
 
         if (!broken && p.final_state != nullptr) {
-            float* dst = p.final_state + (((size_t)n * p.Vh + h) * 128 + row) * 128 + 64 * hf;
+            float* dst = p.final_state + (((size_t)srow * p.Vh + h) * 128 + row) * 128 + 64 * hf;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];

@@ -44,10 +44,14 @@ struct DecodeParams {
     const float* A_log;      // [Vh]
     const float* dt_bias;    // [Vh]
     const float* norm_w;     // [128]
-    float* state;            // f32 [rows][Vh][128][128], in place
-    float* conv;             // f32 [rows][3][C], in place
+    float* state;            // f32 [rows or pool][Vh][128][128], in place
+    float* conv;             // f32 [rows or pool][3][C], in place
     uint16_t* out;           // bf16 [rows][Vh*128]
+    const int* slots;        // [rows] state / history row of each batch row (validated by the host), or nullptr
 };
+
+// State and history row of batch row r.
+__device__ __forceinline__ int decode_slot(const DecodeParams& p, int r) { return p.slots ? __ldg(p.slots + r) : r; }
 
 namespace dec {
 constexpr int kMaxStages = GDN_DECODE_STAGES;
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         const int row = it / p.Kh, kap = it % p.Kh;
         const int r = u % units_per_item;
         const int head = kap * G + (r >> 1);
-        return p.state + (((size_t)row * p.Vh + head) * 128 + (r & 1) * 64) * 128;
+        return p.state + (((size_t)decode_slot(p, row) * p.Vh + head) * 128 + (r & 1) * 64) * 128;
     };
 
     if (warp == kComputeThreads / 32) {
@@ -160,8 +164,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 uint64_t* bar = &auxfull[m & 1];
                 mbar_arrive_expect_tx(bar, pl.aux_load_bytes);
                 const int chq = kap * 128, chk = p.Kh * 128 + kap * 128, chv = 2 * p.Kh * 128 + kap * G * 128;
+                const int srow = decode_slot(p, row);
                 for (int r = 0; r < 3; ++r) {
-                    const float* hrow = p.conv + ((size_t)row * 3 + r) * p.C;
+                    const float* hrow = p.conv + ((size_t)srow * 3 + r) * p.C;
                     float* dst = reinterpret_cast<float*>(ax) + r * nch;
                     bulk_load(dst, hrow + chq, 512, bar);
                     bulk_load(dst + 128, hrow + chk, 512, bar);
@@ -214,6 +219,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     for (int m = 0; m < nmine; ++m) {
         const int it = blockIdx.x + m * gridDim.x;
         const int row = it / p.Kh, kap = it % p.Kh;
+        const int srow = decode_slot(p, row);
         const uint8_t* ax = smem + pl.off_aux + (m & 1) * pl.aux_bytes;
         named_barrier_sync(1, kComputeThreads);  // previous item's readers of s_* are done
         bounded_wait(&auxfull[m & 1], (m >> 1) & 1, broken);
@@ -239,7 +245,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 if (grp == 0) s_q[c] = act;
                 else if (grp == 1) s_k[c] = act;
                 else s_v[(grp - 2) * 128 + c] = act;
-                float* hr = p.conv + (size_t)row * 3 * p.C + ch;
+                float* hr = p.conv + (size_t)srow * 3 * p.C + ch;
                 hr[0] = h1;
                 hr[p.C] = h2;
                 hr[2 * p.C] = x;

@@ -60,7 +60,8 @@ struct PrepParams {
     const uint16_t* conv_w;   // bf16 [C][4]
     const float* A_log;
     const float* dt_bias;
-    const float* init_conv;   // f32 [N][3][C] or nullptr
+    const float* init_conv;   // f32 [N or pool][3][C] or nullptr
+    const int* slots;         // [N] history row of each packed row (validated by the host), or nullptr
     __half* Qs;
     __half* Ks;
     __half* Ql;
@@ -137,7 +138,8 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
         if (xi >= 3) {
             unpack4(__ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)tok * p.C + ch0)), x);
         } else if (p.init_conv != nullptr) {
-            const float4 h = __ldg(reinterpret_cast<const float4*>(p.init_conv + ((size_t)nn * 3 + xi) * p.C + ch0));
+            const int sr = p.slots ? __ldg(p.slots + nn) : nn;
+            const float4 h = __ldg(reinterpret_cast<const float4*>(p.init_conv + ((size_t)sr * 3 + xi) * p.C + ch0));
             x[0] = h.x; x[1] = h.y; x[2] = h.z; x[3] = h.w;
         } else {
 #pragma unroll
@@ -218,8 +220,9 @@ struct ConvOutParams {
     int C, N;
     SeqIndex seq;
     const uint16_t* qkv;     // bf16 [total][C]
-    const float* init_conv;  // f32 [N][3][C] or nullptr
-    float* final_conv;       // f32 [N][3][C]; may alias init_conv
+    const float* init_conv;  // f32 [N or pool][3][C] or nullptr
+    float* final_conv;       // f32 [N or pool][3][C]; may alias init_conv
+    const int* slots;        // [N] history row of each packed row, or nullptr
 };
 
 // final_conv[n][r] = row L+r of [history (3 rows); the row's L tokens].
@@ -231,13 +234,14 @@ __global__ void __launch_bounds__(256) gdn_conv_out_kernel(const ConvOutParams p
     if (ch >= p.C) return;
     int start, len;
     p.seq.bounds(n, start, len);
+    const size_t sr = p.slots ? (size_t)__ldg(p.slots + n) : (size_t)n;
 #pragma unroll
     for (int r = 0; r < 3; ++r) {
         const int e = len + r;
         float v;
         if (e >= 3) v = bf16_bits_to_float(p.qkv[(size_t)(start + e - 3) * p.C + ch]);
-        else v = p.init_conv ? p.init_conv[((size_t)n * 3 + e) * p.C + ch] : 0.f;
-        p.final_conv[((size_t)n * 3 + r) * p.C + ch] = v;
+        else v = p.init_conv ? p.init_conv[(sr * 3 + e) * p.C + ch] : 0.f;
+        p.final_conv[(sr * 3 + r) * p.C + ch] = v;
     }
 }
 

@@ -135,6 +135,38 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
                float* state, float* conv, uint16_t* out, void* stream);
 
 /*
+ * Slot-indexed state pool (a server's fixed rows kept in one big buffer).
+ * Model card (Qwen3.8 27B, Nestmodels for Linnet), cache paragraph: rows keep
+ * their conv history and recurrent state between calls; these two entry
+ * points address them through a slot table instead of by batch position.
+ *   state_pool f32 [pool_rows][Vh][D][D], conv_pool f32 [pool_rows][W-1][C]
+ *   slots_host (host memory) and slots_dev (device memory) hold the same int32
+ *   values, one per batch row: batch row r reads and updates pool row
+ *   slots[r].  The host copy is checked during the call: every slot in
+ *   [0, pool_rows) and no slot twice, else GDN_ERR_INVALID_ARG before anything
+ *   is enqueued; the device copy is read by the kernels.  Pool rows that no
+ *   slot names are not touched.
+ */
+
+/* One decode step of `rows` rows (qkv, z, a, b, out as for gdn_decode),
+ * each on pool row slots[r]; the pool rows are updated in place. */
+int gdn_decode_slots(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
+                     const int32_t* slots_host, const int32_t* slots_dev, int32_t pool_rows,
+                     const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                     float* state_pool, float* conv_pool, uint16_t* out, void* stream);
+
+/* Packed prefill of N rows (cu_seqlens, packed tensors, workspace as for
+ * gdn_prefill_varlen with the same workspace size), row n starting from and
+ * leaving its state and history in pool row slots[n] (in place).  total_T = 0
+ * leaves the pool as it is. */
+int gdn_prefill_varlen_slots(const gdn_dims* dims, const gdn_weights* w, int32_t N,
+                             const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int32_t total_T,
+                             const int32_t* slots_host, const int32_t* slots_dev, int32_t pool_rows,
+                             const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                             float* state_pool, float* conv_pool, uint16_t* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * gdn_prefill without a caller-supplied workspace, for callers that cannot
  * call cudaMalloc: for example a plugin inside an inference engine that owns
  * every device allocation, or a latency-critical path that must not take the

@@ -47,7 +47,7 @@ def test_workspace_sizes(lib):
     one = lib.gdn_prefill_workspace_size(ctypes.byref(d), 1, 1)
     big = lib.gdn_prefill_workspace_size(ctypes.byref(d), 2, 1000)
     # per token: q, k and their residual parts (f16), v (f16), gates; per 64-token chunk
-    # and value head a 33,280-byte record of the chunked form
+    # and value head a 33,296-byte record of the chunked form
     assert one > 0 and big >= 2000 * (4 * 16 * 128 * 2 + 48 * 128 * 2 + 2 * 48 * 4) + 2 * 16 * 48 * 33280
     # packed rows are planned for the most chunks N rows of 2000 tokens can have
     assert lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 2, 2000) >= big
@@ -85,6 +85,19 @@ def test_invalid_arguments_rejected(lib):
     # prefill: negative T
     assert lib.gdn_prefill(ctypes.byref(d), ctypes.byref(w), 1, -3, *([16] * 4), None, None, 16, None, None,
                            16, 1 << 30, None) == -1
+
+
+def test_slot_tables_checked_on_host(lib):
+    # a slot twice, a slot past the pool, a negative slot, an empty pool: refused before any launch
+    d = _dims()
+    w = gdn._WeightsC(16, 16, 16, 16)
+    for slots, pool in (([0, 0], 4), ([0, 4], 4), ([-1, 2], 4), ([0, 1], 0)):
+        arr = (ctypes.c_int32 * 2)(*slots)
+        assert lib.gdn_decode_slots(ctypes.byref(d), ctypes.byref(w), 2, arr, 16, pool, *([16] * 4), 16, 16, 16,
+                                    None) == -1
+        cu = (ctypes.c_int32 * 3)(0, 3, 5)
+        assert lib.gdn_prefill_varlen_slots(ctypes.byref(d), ctypes.byref(w), 2, cu, 16, 5, arr, 16, pool,
+                                            *([16] * 4), 16, 16, 16, 16, 1 << 30, None) == -1
 
 
 def test_binding_refuses_cpu_tensors():
