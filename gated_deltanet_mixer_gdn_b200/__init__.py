@@ -26,7 +26,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen_workspace_size",
-           "gdn_prefill_varlen", "gdn_decode", "gdn_decode_slots", "gdn_prefill_varlen_slots",
+           "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
            "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string", "gdn_version")
 
 GDN_OK = 0
@@ -71,6 +71,8 @@ def load_library() -> ctypes.CDLL:
         L.gdn_prefill_varlen.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_decode.argtypes = [dp, wp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.gdn_decode_multi.restype = ctypes.c_int
+        L.gdn_decode_multi.argtypes = [dp, wp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.gdn_decode_slots.restype = ctypes.c_int
         L.gdn_decode_slots.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.gdn_prefill_varlen_slots.restype = ctypes.c_int
@@ -231,6 +233,25 @@ def decode(qkv, z, a, b, weights, state, conv, *, out=None, dims: Dims = MODEL):
     return out
 
 
+def decode_multi(qkv, z, a, b, weights, state, conv, *, out=None, dims: Dims = MODEL):
+    """k successive tokens for each of `rows` rows in one call.  qkv [rows,k,C],
+    z [rows,k,Vh*D], a/b [rows,k,Vh] bf16; state f32 [rows,Vh,D,D] and conv f32
+    [rows,W-1,C] are updated in place.  Returns out [rows,k,Vh*D]."""
+    dev = _device_of(qkv)
+    L = load_library()
+    rows, k = int(qkv.shape[0]), int(qkv.shape[1])
+    for t, dt, nm in ((qkv, torch.bfloat16, "qkv"), (z, torch.bfloat16, "z"), (a, torch.bfloat16, "a"),
+                      (b, torch.bfloat16, "b"), (state, torch.float32, "state"), (conv, torch.float32, "conv")):
+        _need(t, dt, nm, dev)
+    if out is None:
+        out = torch.empty((rows, k, dims.value_width), dtype=torch.bfloat16, device=dev)
+    dc = _dims_c(dims)
+    st = L.gdn_decode_multi(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), rows, k,
+                            _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(state), _ptr(conv), _ptr(out), _stream(dev))
+    _check(st, "gdn_decode_multi")
+    return out
+
+
 def _slot_tables(slots, n, dev):
     if isinstance(slots, torch.Tensor):
         host = slots.detach().to("cpu", torch.int32).contiguous()
@@ -304,5 +325,5 @@ def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tens
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_varlen", "decode", "decode_slots", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
+__all__ = ["prefill", "prefill_varlen", "decode", "decode_multi", "decode_slots", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

@@ -449,7 +449,7 @@ int check_slots(const int32_t* slots_host, int32_t rows, int32_t pool_rows) {
 // The decode launch: rows batch rows, state / history rows through slots (or nullptr).
 int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const uint16_t* qkv, const uint16_t* z,
                 const uint16_t* a, const uint16_t* b, float* state, float* conv, uint16_t* out, const int32_t* slots,
-                void* stream) {
+                int32_t ntok, void* stream) {
     int st = GDN_OK;
     if (!state || !conv || !aligned16(state) || !aligned16(conv)) return GDN_ERR_INVALID_ARG;
     if ((st = check_io(rows, qkv, z, a, b, out, nullptr, nullptr, nullptr, nullptr)) != GDN_OK) return st;
@@ -471,14 +471,19 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
     p.conv = conv;
     p.out = out;
     p.slots = slots;
+    p.ntok = ntok;
     static std::once_flag dec_once;
     static cudaError_t dec_err = cudaSuccess;
     std::call_once(dec_once, [] {
-        dec_err = cudaFuncSetAttribute(gdn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        dec_err = cudaFuncSetAttribute(gdn_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)dec::kSmemLimit);
+        if (dec_err == cudaSuccess)
+            dec_err = cudaFuncSetAttribute(gdn_decode_kernel<dec::kMaxTokens>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dec::kSmemLimit);
     });
     if (dec_err != cudaSuccess) return GDN_ERR_CUDA;
-    const dec::Plan dplan = dec::plan(p.Vh / p.Kh);
+    const dec::Plan dplan = dec::plan(p.Vh / p.Kh, ntok);
+    if (dplan.stages < 2) return GDN_ERR_UNSUPPORTED;  // the group's inputs of ntok tokens leave no room
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -493,7 +498,8 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
     cfg.stream = static_cast<cudaStream_t>(stream);
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;
-    return cuda_status(cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p));
+    return cuda_status(ntok == 1 ? cudaLaunchKernelEx(&cfg, gdn_decode_kernel<1>, p)
+                                 : cudaLaunchKernelEx(&cfg, gdn_decode_kernel<dec::kMaxTokens>, p));
 }
 
 
@@ -562,7 +568,19 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const u
     if ((st = check_weights(w)) != GDN_OK) return st;
     if (rows < 0 || rows > 65535) return GDN_ERR_INVALID_ARG;
     if (rows == 0) return GDN_OK;
-    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, stream);
+    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, 1, stream);
+}
+
+int gdn_decode_multi(const gdn_dims* dims, const gdn_weights* w, int32_t rows, int32_t ntok, const uint16_t* qkv,
+                     const uint16_t* z, const uint16_t* a, const uint16_t* b, float* state, float* conv, uint16_t* out,
+                     void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (rows < 0 || rows > 65535 || ntok < 1) return GDN_ERR_INVALID_ARG;
+    if (ntok > dec::kMaxTokens) return GDN_ERR_UNSUPPORTED;
+    if (rows == 0) return GDN_OK;
+    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, ntok, stream);
 }
 
 
@@ -577,7 +595,7 @@ int gdn_decode_slots(const gdn_dims* dims, const gdn_weights* w, int32_t rows, c
     if (rows == 0) return GDN_OK;
     if ((st = check_slots(slots_host, rows, pool_rows)) != GDN_OK) return st;
     if (slots_dev == nullptr || (reinterpret_cast<uintptr_t>(slots_dev) & 3u)) return GDN_ERR_INVALID_ARG;
-    return decode_impl(dims, w, rows, qkv, z, a, b, state_pool, conv_pool, out, slots_dev, stream);
+    return decode_impl(dims, w, rows, qkv, z, a, b, state_pool, conv_pool, out, slots_dev, 1, stream);
 }
 
 int gdn_prefill_varlen_slots(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_host,

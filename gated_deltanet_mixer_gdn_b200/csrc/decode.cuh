@@ -1,4 +1,5 @@
-// Decode step of the Gated DeltaNet mixer: one token for each of `rows` rows.
+// Decode of the Gated DeltaNet mixer: one token (or k successive tokens) for
+// each of `rows` rows.
 //
 // Qwen3.8 27B model card (Nestmodels for Linnet), "Gated DeltaNet" bullet and
 // cache paragraph: each row keeps its conv history and its per-value-head
@@ -11,7 +12,9 @@
 //     S_new = alpha S + u k^T,  u = beta (v - alpha S k),
 //     o     = S_new q = alpha (S q) + u (k . q),
 // both dot products use the old state row, so each row is read and written
-// once.
+// once.  With k tokens per row (speculative verification, several tokens per
+// call) each state row stays in registers through the k sequential updates:
+// the state is still read and written once per call, k tokens at a time.
 //
 // Work item = (row, q/k head): the conv of the q/k head's 256 channels and of
 // its value heads' 128-channel slices, the L2 norms and gates, then the states
@@ -36,17 +39,18 @@ namespace gdn {
 
 struct DecodeParams {
     int Kh, Vh, C, rows, nitems;
-    const uint16_t* qkv;     // bf16 [rows][C]
-    const uint16_t* z;       // bf16 [rows][Vh*128]
-    const uint16_t* a;       // bf16 [rows][Vh]
-    const uint16_t* b;       // bf16 [rows][Vh]
+    int ntok;                // tokens per row (1 .. the kernel's maximum)
+    const uint16_t* qkv;     // bf16 [rows][ntok][C]
+    const uint16_t* z;       // bf16 [rows][ntok][Vh*128]
+    const uint16_t* a;       // bf16 [rows][ntok][Vh]
+    const uint16_t* b;       // bf16 [rows][ntok][Vh]
     const uint16_t* conv_w;  // bf16 [C][4]
     const float* A_log;      // [Vh]
     const float* dt_bias;    // [Vh]
     const float* norm_w;     // [128]
     float* state;            // f32 [rows or pool][Vh][128][128], in place
     float* conv;             // f32 [rows or pool][3][C], in place
-    uint16_t* out;           // bf16 [rows][Vh*128]
+    uint16_t* out;           // bf16 [rows][ntok][Vh*128]
     const int* slots;        // [rows] state / history row of each batch row (validated by the host), or nullptr
 };
 
@@ -61,31 +65,39 @@ constexpr int kComputeThreads = 256;
 constexpr int kThreads = kComputeThreads + 32;  // + producer warp
 constexpr int kSlots = (2 + kMaxGroup) * 128 / kComputeThreads;  // conv channels per thread (max)
 constexpr uint32_t kSmemLimit = 232448;         // opt-in shared memory per block on sm_100
-// misc: barriers (256 B), q, k (2 x 512 B), v and o (2 x kMaxGroup x 512 B), reductions, gates
-constexpr uint32_t MISC_BYTES = 256 + 2 * 512 + 2 * kMaxGroup * 512 + 512 + 256;
+constexpr int kMaxTokens = 8;                   // tokens per row of the multi-token kernel
 
-// Shared-memory plan for a group size G: a ring of half-tile stages, then two
-// buffers of per-item inputs, bulk-copied one item ahead (history
-// [3][(2+G)*128] f32, new qkv [(2+G)*128] bf16, conv taps [(2+G)*128][4] bf16,
-// z [G*128] bf16), then small scratch.
+// Shared-memory plan for a group size G and n tokens per row: a ring of
+// half-tile stages, then two buffers of per-item inputs, bulk-copied one item
+// ahead (history [3][(2+G)*128] f32, new qkv [n][(2+G)*128] bf16, conv taps
+// [(2+G)*128][4] bf16, z [n][G*128] bf16), then scratch: barriers (256 B),
+// q, k [n][128], v, o [n][G][128], reductions [n][8 + 8G], gates [n][G][2], k.q [n].
 struct Plan {
     int stages;
-    uint32_t aux_x, aux_w, aux_z, aux_bytes, aux_load_bytes, off_aux, off_misc, smem_bytes;
+    uint32_t aux_x, aux_w, aux_z, aux_bytes, aux_load_bytes, off_aux, off_misc, misc_bytes, smem_bytes;
+    uint32_t m_q, m_k, m_v, m_o, m_red, m_gate;  // float offsets of the scratch arrays (from off_misc + 256)
 };
-__host__ __device__ inline Plan plan(int G) {
+__host__ __device__ inline Plan plan(int G, int n) {
     Plan pl{};
     const uint32_t nch = (2 + G) * 128;
     pl.aux_x = 3 * nch * 4;
-    pl.aux_w = pl.aux_x + nch * 2;
+    pl.aux_w = pl.aux_x + n * nch * 2;
     pl.aux_z = pl.aux_w + nch * 8;
-    pl.aux_load_bytes = pl.aux_z + G * 256;
+    pl.aux_load_bytes = pl.aux_z + n * G * 256;
     pl.aux_bytes = (pl.aux_load_bytes + 127) / 128 * 128;
-    const uint32_t rest = 2 * pl.aux_bytes + MISC_BYTES + 1024;
+    pl.m_q = 0;
+    pl.m_k = pl.m_q + n * 128;
+    pl.m_v = pl.m_k + n * 128;
+    pl.m_o = pl.m_v + n * G * 128;
+    pl.m_red = pl.m_o + n * G * 128;
+    pl.m_gate = pl.m_red + n * (8 + 8 * G);
+    pl.misc_bytes = 256 + ((pl.m_gate + n * G * 2 + n) * 4 + 127) / 128 * 128;  // gates, then k.q [n]
+    const uint32_t rest = 2 * pl.aux_bytes + pl.misc_bytes + 1024;
     int st = (int)((kSmemLimit - rest) / kTileBytes);
     pl.stages = st > kMaxStages ? kMaxStages : st;
     pl.off_aux = pl.stages * kTileBytes;
     pl.off_misc = pl.off_aux + 2 * pl.aux_bytes;
-    pl.smem_bytes = pl.off_misc + MISC_BYTES + 1024;
+    pl.smem_bytes = pl.off_misc + pl.misc_bytes + 1024;
     return pl;
 }
 }  // namespace dec
@@ -106,23 +118,28 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, boo
     return true;
 }
 
+template <int KMAX>
 __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const DecodeParams p) {
     using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int G = p.Vh / p.Kh;
-    const Plan pl = plan(G);
+    const int nt = KMAX == 1 ? 1 : p.ntok;  // tokens per row
+    const Plan pl = plan(G, nt);
     const int nst = pl.stages;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.off_misc);
     uint64_t* empty = full + kMaxStages;
     uint64_t* auxfull = empty + kMaxStages;
     uint64_t* auxempty = auxfull + 2;
-    float* s_q = reinterpret_cast<float*>(smem + pl.off_misc + 256);
-    float* s_k = s_q + 128;
-    float* s_v = s_k + 128;                 // [group][128]
-    float* s_o = s_v + kMaxGroup * 128;     // [group][128]
-    float* s_red = s_o + kMaxGroup * 128;   // [128]
-    float* s_gate = s_red + 128;            // [2 * group]
+    float* scratch = reinterpret_cast<float*>(smem + pl.off_misc + 256);
+    float* s_q = scratch + pl.m_q;        // [nt][128]
+    float* s_k = scratch + pl.m_k;        // [nt][128]
+    float* s_v = scratch + pl.m_v;        // [nt][G][128]
+    float* s_o = scratch + pl.m_o;        // [nt][G][128]
+    float* s_red = scratch + pl.m_red;    // [nt][8 + 8G]
+    float* s_gate = scratch + pl.m_gate;  // [nt][G][2], then k.q [nt]
+    float* s_kq = s_gate + nt * G * 2;
+    const int nred = 8 + 8 * G;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -172,16 +189,19 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                     bulk_load(dst + 128, hrow + chk, 512, bar);
                     bulk_load(dst + 256, hrow + chv, G * 512, bar);
                 }
-                const uint16_t* xrow = p.qkv + (size_t)row * p.C;
-                uint16_t* dx = reinterpret_cast<uint16_t*>(ax + pl.aux_x);
-                bulk_load(dx, xrow + chq, 256, bar);
-                bulk_load(dx + 128, xrow + chk, 256, bar);
-                bulk_load(dx + 256, xrow + chv, G * 256, bar);
+                for (int j = 0; j < nt; ++j) {
+                    const uint16_t* xrow = p.qkv + ((size_t)row * nt + j) * p.C;
+                    uint16_t* dx = reinterpret_cast<uint16_t*>(ax + pl.aux_x) + j * nch;
+                    bulk_load(dx, xrow + chq, 256, bar);
+                    bulk_load(dx + 128, xrow + chk, 256, bar);
+                    bulk_load(dx + 256, xrow + chv, G * 256, bar);
+                    bulk_load(ax + pl.aux_z + j * G * 256, p.z + (((size_t)row * nt + j) * p.Vh + kap * G) * 128,
+                              G * 256, bar);
+                }
                 uint16_t* dw = reinterpret_cast<uint16_t*>(ax + pl.aux_w);
                 bulk_load(dw, p.conv_w + (size_t)chq * 4, 1024, bar);
                 bulk_load(dw + 512, p.conv_w + (size_t)chk * 4, 1024, bar);
                 bulk_load(dw + 1024, p.conv_w + (size_t)chv * 4, G * 1024, bar);
-                bulk_load(ax + pl.aux_z, p.z + ((size_t)row * p.Vh + kap * G) * 128, G * 256, bar);
             };
             // the next item's inputs are requested once the ring holds this item's first stages,
             // by which time the item two back has released their buffer
@@ -204,27 +224,27 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
 
     // ---------------- compute warps (tid < 256)
     const float w_n = (tid < 128) ? 1.0f + p.norm_w[tid] : 0.f;
-    // gate inputs of the next item, loaded one item ahead (threads tid < G)
+    // gate inputs of the next item, loaded one item ahead (thread tid < G * nt: token tid / G, head tid % G)
     float ga = 0.f, gb = 0.f, gA = 0.f, gdt = 0.f;
     auto gate_prefetch = [&](int m) {
         const int it = blockIdx.x + m * gridDim.x;
-        const int row = it / p.Kh, head = (it % p.Kh) * G + tid;
-        ga = bf16_bits_to_float(p.a[(size_t)row * p.Vh + head]);
-        gb = bf16_bits_to_float(p.b[(size_t)row * p.Vh + head]);
+        const int row = it / p.Kh, head = (it % p.Kh) * G + tid % G, j = tid / G;
+        ga = bf16_bits_to_float(p.a[((size_t)row * nt + j) * p.Vh + head]);
+        gb = bf16_bits_to_float(p.b[((size_t)row * nt + j) * p.Vh + head]);
         gA = p.A_log[head];
         gdt = p.dt_bias[head];
     };
-    if (tid < G && nmine > 0) gate_prefetch(0);
+    if (tid < G * nt && nmine > 0) gate_prefetch(0);
     int u = 0;
     for (int m = 0; m < nmine; ++m) {
         const int it = blockIdx.x + m * gridDim.x;
         const int row = it / p.Kh, kap = it % p.Kh;
         const int srow = decode_slot(p, row);
         const uint8_t* ax = smem + pl.off_aux + (m & 1) * pl.aux_bytes;
-        named_barrier_sync(1, kComputeThreads);  // previous item's readers of s_* are done
+        named_barrier_sync(1, kComputeThreads);  // previous item's readers of the scratch are done
         bounded_wait(&auxfull[m & 1], (m >> 1) & 1, broken);
 
-        // ---- conv + silu of the item's channels; shift their history in place
+        // ---- conv + silu of the item's channels over the nt tokens; shift their history in place
         const float* ah = reinterpret_cast<const float*>(ax);
         const uint16_t* axx = reinterpret_cast<const uint16_t*>(ax + pl.aux_x);
         const uint2* aw = reinterpret_cast<const uint2*>(ax + pl.aux_w);
@@ -236,48 +256,66 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 const int ch = (grp == 0) ? kap * 128 + c
                              : (grp == 1) ? p.Kh * 128 + kap * 128 + c
                                           : 2 * p.Kh * 128 + (kap * G + grp - 2) * 128 + c;
-                const float h0 = ah[idx], h1 = ah[nch + idx], h2 = ah[2 * nch + idx];
-                const float x = bf16_bits_to_float(axx[idx]);
+                float h0 = ah[idx], h1 = ah[nch + idx], h2 = ah[2 * nch + idx];
                 const uint2 wb = aw[idx];
-                const float cv = __uint_as_float(wb.x << 16) * h0 + __uint_as_float(wb.x & 0xffff0000u) * h1 +
-                                 __uint_as_float(wb.y << 16) * h2 + __uint_as_float(wb.y & 0xffff0000u) * x;
-                const float act = silu_f(cv);
-                if (grp == 0) s_q[c] = act;
-                else if (grp == 1) s_k[c] = act;
-                else s_v[(grp - 2) * 128 + c] = act;
+                const float t0 = __uint_as_float(wb.x << 16), t1 = __uint_as_float(wb.x & 0xffff0000u);
+                const float t2 = __uint_as_float(wb.y << 16), t3 = __uint_as_float(wb.y & 0xffff0000u);
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    if (j < nt) {
+                        const float x = bf16_bits_to_float(axx[j * nch + idx]);
+                        const float act = silu_f(t0 * h0 + t1 * h1 + t2 * h2 + t3 * x);
+                        if (grp == 0) s_q[j * 128 + c] = act;
+                        else if (grp == 1) s_k[j * 128 + c] = act;
+                        else s_v[(j * G + grp - 2) * 128 + c] = act;
+                        h0 = h1;
+                        h1 = h2;
+                        h2 = x;
+                    }
+                }
                 float* hr = p.conv + (size_t)srow * 3 * p.C + ch;
-                hr[0] = h1;
-                hr[p.C] = h2;
-                hr[2 * p.C] = x;
+                hr[0] = h0;
+                hr[p.C] = h1;
+                hr[2 * p.C] = h2;
             }
         }
-        if (tid < G) {
-            s_gate[2 * tid] = expf(-expf(gA) * softplus_f(ga + gdt));  // alpha
+        if (tid < G * nt) {
+            s_gate[2 * tid] = expf(-expf(gA) * softplus_f(ga + gdt));  // alpha of (token tid / G, head tid % G)
             s_gate[2 * tid + 1] = sigmoid_f(gb);                        // beta
             if (m + 1 < nmine) gate_prefetch(m + 1);
         }
         named_barrier_sync(1, kComputeThreads);
-        // ---- L2 norms: q in warps 0-3, k in warps 4-7
-        {
-            const float x = (tid < 128) ? s_q[tid] : s_k[tid - 128];
-            const float ss = warp_sum(x * x);
-            if (lane == 0) s_red[warp] = ss;
+        // ---- L2 norms per token: q in warps 0-3, k in warps 4-7
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < nt) {
+                const float x = (tid < 128) ? s_q[j * 128 + tid] : s_k[j * 128 + tid - 128];
+                const float ss = warp_sum(x * x);
+                if (lane == 0) s_red[j * nred + warp] = ss;
+            }
         }
         named_barrier_sync(1, kComputeThreads);
-        const float qscale = rsqrtf(s_red[0] + s_red[1] + s_red[2] + s_red[3] + kEps) * rsqrtf(128.0f);
-        const float kscale = rsqrtf(s_red[4] + s_red[5] + s_red[6] + s_red[7] + kEps);
-        float4 qf = reinterpret_cast<const float4*>(s_q)[lane];
-        float4 kf = reinterpret_cast<const float4*>(s_k)[lane];
-        qf.x *= qscale; qf.y *= qscale; qf.z *= qscale; qf.w *= qscale;
-        kf.x *= kscale; kf.y *= kscale; kf.z *= kscale; kf.w *= kscale;
-        const float kq = warp_sum(kf.x * qf.x + kf.y * qf.y + kf.z * qf.z + kf.w * qf.w);
+        // q / (|q| sqrt(128)), k / |k| in place; then k.q per token (warp j)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < nt) {
+                const float* r8 = s_red + j * nred;
+                if (tid < 128) s_q[j * 128 + tid] *= rsqrtf(r8[0] + r8[1] + r8[2] + r8[3] + kEps) * rsqrtf(128.0f);
+                else s_k[j * 128 + tid - 128] *= rsqrtf(r8[4] + r8[5] + r8[6] + r8[7] + kEps);
+            }
+        }
+        named_barrier_sync(1, kComputeThreads);
+        if (warp < nt) {
+            const float4 qf = reinterpret_cast<const float4*>(s_q + warp * 128)[lane];
+            const float4 kf = reinterpret_cast<const float4*>(s_k + warp * 128)[lane];
+            const float kq = warp_sum(kf.x * qf.x + kf.y * qf.y + kf.z * qf.z + kf.w * qf.w);
+            if (lane == 0) s_kq[warp] = kq;
+        }
+        named_barrier_sync(1, kComputeThreads);
 
-        // ---- stream the G value heads' states, two half-tiles each
+        // ---- stream the G value heads' states, two half-tiles each; nt updates per row in registers
 #pragma unroll 1
         for (int hh = 0; hh < G; ++hh) {
-            const float alpha = s_gate[2 * hh], beta = s_gate[2 * hh + 1];
-            const float* sv = s_v + hh * 128;
-            float* so = s_o + hh * 128;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half, ++u) {
                 const int st = u % nst;
@@ -288,49 +326,67 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 for (int r = 0; r < 8; ++r) s[r] = reinterpret_cast<const float4*>(tile + (warp * 8 + r) * 128)[lane];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done reading the stage
-                float vals[16];
-#pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    vals[2 * r] = s[r].x * kf.x + s[r].y * kf.y + s[r].z * kf.z + s[r].w * kf.w;
-                    vals[2 * r + 1] = s[r].x * qf.x + s[r].y * qf.y + s[r].z * qf.z + s[r].w * qf.w;
-                }
-                // lane l: row l >> 2 of the warp's 8, S.k if bit 1 of l is clear, else S.q
-                const float tot = warp_transpose_sum16(vals, lane);
                 const int irow = half * 64 + warp * 8 + (lane >> 2);
-                const float u_k = beta * (sv[irow] - alpha * tot);  // meaningful on lanes 4r, 4r+1
-                const float u_r = __shfl_sync(0xffffffffu, u_k, lane & ~3);
-                if ((lane & 3) == 2) so[irow] = alpha * tot + u_r * kq;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    if (j < nt) {
+                        const float alpha = s_gate[2 * (j * G + hh)], beta = s_gate[2 * (j * G + hh) + 1];
+                        const float4 qf = reinterpret_cast<const float4*>(s_q + j * 128)[lane];
+                        const float4 kf = reinterpret_cast<const float4*>(s_k + j * 128)[lane];
+                        float vals[16];
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            vals[2 * r] = s[r].x * kf.x + s[r].y * kf.y + s[r].z * kf.z + s[r].w * kf.w;
+                            vals[2 * r + 1] = s[r].x * qf.x + s[r].y * qf.y + s[r].z * qf.z + s[r].w * qf.w;
+                        }
+                        // lane l: row l >> 2 of the warp's 8, S.k if bit 1 of l is clear, else S.q
+                        const float tot = warp_transpose_sum16(vals, lane);
+                        const float u_k = beta * (s_v[(j * G + hh) * 128 + irow] - alpha * tot);  // lanes 4r, 4r+1
+                        const float u_r = __shfl_sync(0xffffffffu, u_k, lane & ~3);
+                        if ((lane & 3) == 2) s_o[(j * G + hh) * 128 + irow] = alpha * tot + u_r * s_kq[j];
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            const float ur = __shfl_sync(0xffffffffu, u_k, 4 * r);
+                            s[r].x = alpha * s[r].x + ur * kf.x;
+                            s[r].y = alpha * s[r].y + ur * kf.y;
+                            s[r].z = alpha * s[r].z + ur * kf.z;
+                            s[r].w = alpha * s[r].w + ur * kf.w;
+                        }
+                    }
+                }
                 float* gdst = unit_ptr(u) + (warp * 8) * 128;
 #pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    const float ur = __shfl_sync(0xffffffffu, u_k, 4 * r);
-                    float4 n;
-                    n.x = alpha * s[r].x + ur * kf.x;
-                    n.y = alpha * s[r].y + ur * kf.y;
-                    n.z = alpha * s[r].z + ur * kf.z;
-                    n.w = alpha * s[r].w + ur * kf.w;
-                    __stcs(reinterpret_cast<float4*>(gdst + r * 128) + lane, n);
-                }
+                for (int r = 0; r < 8; ++r) __stcs(reinterpret_cast<float4*>(gdst + r * 128) + lane, s[r]);
             }
         }
 
-        // ---- gated RMSNorm of the G heads' 128 outputs each
+        // ---- gated RMSNorm of the G heads' 128 outputs of every token
         named_barrier_sync(1, kComputeThreads);
-        for (int hh = 0; hh < G; ++hh) {
-            const float o = (tid < 128) ? s_o[hh * 128 + tid] : 0.f;
-            const float ss = warp_sum(o * o);
-            if (lane == 0) s_red[8 + hh * 8 + warp] = ss;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < nt) {
+                for (int hh = 0; hh < G; ++hh) {
+                    const float o = (tid < 128) ? s_o[(j * G + hh) * 128 + tid] : 0.f;
+                    const float ss = warp_sum(o * o);
+                    if (lane == 0) s_red[j * nred + 8 + hh * 8 + warp] = ss;
+                }
+            }
         }
         named_barrier_sync(1, kComputeThreads);
         if (tid < 128) {
             const uint16_t* az = reinterpret_cast<const uint16_t*>(ax + pl.aux_z);
-            for (int hh = 0; hh < G; ++hh) {
-                const float* r4 = s_red + 8 + hh * 8;
-                const float ms = (r4[0] + r4[1] + r4[2] + r4[3]) * (1.0f / 128.0f);
-                const int head = kap * G + hh;
-                const float zv = bf16_bits_to_float(az[hh * 128 + tid]);
-                const float y = s_o[hh * 128 + tid] * rsqrtf(ms + kEps) * w_n * silu_f(zv);
-                p.out[(size_t)row * p.Vh * 128 + head * 128 + tid] = float_to_bf16_bits(y);
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < nt) {
+                    for (int hh = 0; hh < G; ++hh) {
+                        const float* r4 = s_red + j * nred + 8 + hh * 8;
+                        const float ms = (r4[0] + r4[1] + r4[2] + r4[3]) * (1.0f / 128.0f);
+                        const int head = kap * G + hh;
+                        const float zv = bf16_bits_to_float(az[(j * G + hh) * 128 + tid]);
+                        const float y = s_o[(j * G + hh) * 128 + tid] * rsqrtf(ms + kEps) * w_n * silu_f(zv);
+                        p.out[(((size_t)row * nt + j) * p.Vh + head) * 128 + tid] = float_to_bf16_bits(y);
+                    }
+                }
             }
         }
         __syncwarp();

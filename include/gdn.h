@@ -135,6 +135,22 @@ int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows,
                float* state, float* conv, uint16_t* out, void* stream);
 
 /*
+ * ntok successive decode tokens for each of `rows` rows in one call
+ * (verification of speculated tokens, or several new tokens per row): each
+ * row's state stays on chip through its ntok sequential updates, so the state
+ * is read and written once per call instead of once per token.  Same
+ * arithmetic per token as gdn_decode (the same results as ntok calls of it).
+ *   qkv bf16 [rows][ntok][C], z bf16 [rows][ntok][Vh*D], a, b bf16 [rows][ntok][Vh]
+ *   state f32 [rows][Vh][D][D] and conv f32 [rows][W-1][C] in/out (after the ntok tokens)
+ *   out   bf16 [rows][ntok][Vh*D]
+ * 1 <= ntok <= 8; GDN_ERR_UNSUPPORTED above 8 or when a q/k head's group of
+ * value heads needs more on-chip room for ntok tokens than a block has.
+ */
+int gdn_decode_multi(const gdn_dims* dims, const gdn_weights* w, int32_t rows, int32_t ntok,
+                     const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                     float* state, float* conv, uint16_t* out, void* stream);
+
+/*
  * Slot-indexed state pool (a server's fixed rows kept in one big buffer).
  * Model card (Qwen3.8 27B, Nestmodels for Linnet), cache paragraph: rows keep
  * their conv history and recurrent state between calls; these two entry
