@@ -6,7 +6,8 @@ steps with the 27B model's GDN shapes, each row with its own f32 state
 whole pass (128 decode launches, 8192 row-tokens).  Metric: row-tokens/s.
 A second measured object, "prefill", times the chunked prefill (one row of
 8192 tokens from zero state, and the 8-row varlen workload) in tokens/s
-against the tensor roofline.
+against the tensor roofline; a third, "decode_multi", the same decode batch
+with 4 tokens per row per call (gdn_decode_multi).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -308,6 +309,55 @@ def run_ours(args, world, rank, local):
     return line, case
 
 
+def bench_decode_multi(args, local, k=4):
+    """The same 64-row, 128-token decode batch with k tokens per row per call
+    (gdn_decode_multi): 128 / k launches per pass, the state read and written once
+    per launch.  CUDA events on the launching stream around a captured pass."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    case = synth.config(1)
+    w = gdn.weights_to(case["weights"], dev)
+    # [steps, rows, ...] -> per launch [rows, k, ...]
+    acts = {n: case[n].to(dev).view(DECODE_STEPS // k, k, ROWS, -1).transpose(1, 2).contiguous()
+            for n in ("qkv", "z", "a", "b")}
+    state = case["init_state"].to(dev)
+    conv = case["init_conv"].to(dev)
+    out = torch.empty((DECODE_STEPS // k, ROWS, k, 6144), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def one_pass():
+        for s in range(DECODE_STEPS // k):
+            gdn.decode_multi(acts["qkv"][s], acts["z"][s], acts["a"][s], acts["b"][s], w, state, conv, out=out[s])
+
+    with torch.cuda.stream(stream):
+        one_pass()
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        one_pass()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t = e0.elapsed_time(e1) / 1000.0
+    launches = args.steps * (DECODE_STEPS // k)
+    achieved = ROWS * STATE_BYTES_PER_ROW_TOKEN / (t / launches) / 1e9  # state bytes per launch / launch time
+    return {"workload": f"decode 64 rows x 128 tokens, {k} tokens per row per call", "tokens_per_call": k,
+            "value": ROWS * DECODE_STEPS * args.steps / t, "unit": "row-tokens/s",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                         "algorithmic_bytes_per_launch": ROWS * STATE_BYTES_PER_ROW_TOKEN},
+            "gpu_launches": launches}
+
+
 def _time_prefill(call, dev, stream, warmup, reps):
     """Median seconds of `call` (CUDA events on `stream`), L2 flushed before each timed call."""
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > L2, written between iterations
@@ -397,8 +447,10 @@ def main():
             return 0
         line, case = run_ours(args, world, rank, local)
         pre = bench_prefill(args, world, rank, local, args.prefill_T)
+        multi = bench_decode_multi(args, local)
         if rank == 0:
             line["prefill"] = pre
+            line["decode_multi"] = multi
             if world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline_line(case)
             print(json.dumps(line))

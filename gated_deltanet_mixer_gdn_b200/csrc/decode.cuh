@@ -260,9 +260,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 const uint2 wb = aw[idx];
                 const float t0 = __uint_as_float(wb.x << 16), t1 = __uint_as_float(wb.x & 0xffff0000u);
                 const float t2 = __uint_as_float(wb.y << 16), t3 = __uint_as_float(wb.y & 0xffff0000u);
-#pragma unroll
-                for (int j = 0; j < KMAX; ++j) {
-                    if (j < nt) {
+#pragma unroll 1
+                for (int j = 0; j < nt; ++j) {
+                    {
                         const float x = bf16_bits_to_float(axx[j * nch + idx]);
                         const float act = silu_f(t0 * h0 + t1 * h1 + t2 * h2 + t3 * x);
                         if (grp == 0) s_q[j * 128 + c] = act;
@@ -286,9 +286,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         }
         named_barrier_sync(1, kComputeThreads);
         // ---- L2 norms per token: q in warps 0-3, k in warps 4-7
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (j < nt) {
+#pragma unroll 1
+        for (int j = 0; j < nt; ++j) {
+            {
                 const float x = (tid < 128) ? s_q[j * 128 + tid] : s_k[j * 128 + tid - 128];
                 const float ss = warp_sum(x * x);
                 if (lane == 0) s_red[j * nred + warp] = ss;
@@ -296,9 +296,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         }
         named_barrier_sync(1, kComputeThreads);
         // q / (|q| sqrt(128)), k / |k| in place; then k.q per token (warp j)
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (j < nt) {
+#pragma unroll 1
+        for (int j = 0; j < nt; ++j) {
+            {
                 const float* r8 = s_red + j * nred;
                 if (tid < 128) s_q[j * 128 + tid] *= rsqrtf(r8[0] + r8[1] + r8[2] + r8[3] + kEps) * rsqrtf(128.0f);
                 else s_k[j * 128 + tid - 128] *= rsqrtf(r8[4] + r8[5] + r8[6] + r8[7] + kEps);
@@ -327,9 +327,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done reading the stage
                 const int irow = half * 64 + warp * 8 + (lane >> 2);
-#pragma unroll
-                for (int j = 0; j < KMAX; ++j) {
-                    if (j < nt) {
+#pragma unroll 1
+                for (int j = 0; j < nt; ++j) {
+                    {
                         const float alpha = s_gate[2 * (j * G + hh)], beta = s_gate[2 * (j * G + hh) + 1];
                         const float4 qf = reinterpret_cast<const float4*>(s_q + j * 128)[lane];
                         const float4 kf = reinterpret_cast<const float4*>(s_k + j * 128)[lane];
@@ -362,9 +362,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
 
         // ---- gated RMSNorm of the G heads' 128 outputs of every token
         named_barrier_sync(1, kComputeThreads);
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (j < nt) {
+#pragma unroll 1
+        for (int j = 0; j < nt; ++j) {
+            {
                 for (int hh = 0; hh < G; ++hh) {
                     const float o = (tid < 128) ? s_o[(j * G + hh) * 128 + tid] : 0.f;
                     const float ss = warp_sum(o * o);
@@ -375,9 +375,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         named_barrier_sync(1, kComputeThreads);
         if (tid < 128) {
             const uint16_t* az = reinterpret_cast<const uint16_t*>(ax + pl.aux_z);
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                if (j < nt) {
+#pragma unroll 1
+            for (int j = 0; j < nt; ++j) {
+                {
                     for (int hh = 0; hh < G; ++hh) {
                         const float* r4 = s_red + j * nred + 8 + hh * 8;
                         const float ms = (r4[0] + r4[1] + r4[2] + r4[3]) * (1.0f / 128.0f);
