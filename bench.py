@@ -420,7 +420,50 @@ def bench_prefill(args, world, rank, local, T):
                                dev, stream, max(3, args.warmup), max(5, args.steps))
         out["varlen8"] = line(total, t2, f"varlen prefill 8 rows ({total} tokens, lengths U[512,16384]), "
                                          "random initial state and history", 5 * n2)
+        out["long2"] = bench_long_context(args, local, line)
     return out
+
+
+def bench_long_context(args, local, line):
+    """Long-context prefill: 2 rows x 65536 tokens from zero state, returning the final
+    states (overlapped schedule); then 256 decode steps per row from those states."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    case = synth.config(4)
+    w = gdn.weights_to(case["weights"], dev)
+    acts = {k: case[k].to(dev) for k in ("qkv", "z", "a", "b")}
+    B, T = acts["qkv"].shape[0], acts["qkv"].shape[1]
+    out = torch.empty((B, T, 6144), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((B, 48, 128, 128), dtype=torch.float32, device=dev)
+    fc = torch.empty((B, 3, 10240), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    reps = max(3, min(args.steps, 5))
+    t, n = _time_prefill(lambda: gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w, out=out, final_state=fs,
+                                             final_conv=fc), dev, stream, 3, reps)
+    res = line(B * T, t, f"long-context prefill B={B} T={T}, zero initial state, final states returned", 4 * n)
+    # 256 decode steps per row from the prefill's states (2 rows: launch-latency bound, reported)
+    steps = case["decode"]["qkv"].shape[0]
+    dq = {k: case["decode"][k].to(dev) for k in ("qkv", "z", "a", "b")}
+    dout = torch.empty((steps, B, 6144), dtype=torch.bfloat16, device=dev)
+    st, cv = fs.clone(), fc.clone()
+    with torch.cuda.stream(stream):
+        for s in range(steps):
+            gdn.decode(dq["qkv"][s], dq["z"][s], dq["a"][s], dq["b"][s], w, st, cv, out=dout[s])
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        st.copy_(fs)
+        cv.copy_(fc)
+        e0.record(stream)
+        for s in range(steps):
+            gdn.decode(dq["qkv"][s], dq["z"][s], dq["a"][s], dq["b"][s], w, st, cv, out=dout[s])
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    td = e0.elapsed_time(e1) / 1000.0
+    res["decode_after"] = {"workload": f"{steps} decode steps x {B} rows from the prefill's states",
+                           "value": B * steps / td, "unit": "row-tokens/s", "us_per_step": td / steps * 1e6,
+                           "gpu_launches": steps}
+    return res
 
 
 def main():
