@@ -27,7 +27,8 @@ LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen_workspace_size",
            "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
-           "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string", "gdn_version")
+           "gdn_in_proj", "gdn_out_proj", "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string",
+           "gdn_version")
 
 GDN_OK = 0
 
@@ -71,6 +72,10 @@ def load_library() -> ctypes.CDLL:
         L.gdn_prefill_varlen.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_decode.argtypes = [dp, wp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.gdn_in_proj.restype = ctypes.c_int
+        L.gdn_in_proj.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.gdn_out_proj.restype = ctypes.c_int
+        L.gdn_out_proj.argtypes = [dp, i32, i32, vp, vp, vp, vp]
         L.gdn_decode_multi.restype = ctypes.c_int
         L.gdn_decode_multi.argtypes = [dp, wp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.gdn_decode_slots.restype = ctypes.c_int
@@ -252,6 +257,42 @@ def decode_multi(qkv, z, a, b, weights, state, conv, *, out=None, dims: Dims = M
     return out
 
 
+def in_proj(x, w_in, *, dims: Dims = MODEL, out=None):
+    """x bf16 [T, hidden] times the stacked in_proj weights w_in bf16 [C + Vh*D + 2*Vh, hidden]
+    (qkv, z, b, a rows).  Returns (qkv [T,C], z [T,Vh*D], a [T,Vh], b [T,Vh])."""
+    dev = _device_of(x)
+    L = load_library()
+    _need(x, torch.bfloat16, "x", dev)
+    _need(w_in, torch.bfloat16, "w_in", dev)
+    T, hidden = int(x.shape[0]), int(x.shape[1])
+    C, VD, Vh = dims.conv_channels, dims.value_width, dims.num_v_heads
+    if tuple(w_in.shape) != (C + VD + 2 * Vh, hidden):
+        raise ValueError("in_proj: w_in shape")
+    qkv, z, a, b = out if out is not None else (
+        torch.empty((T, C), dtype=torch.bfloat16, device=dev), torch.empty((T, VD), dtype=torch.bfloat16, device=dev),
+        torch.empty((T, Vh), dtype=torch.bfloat16, device=dev), torch.empty((T, Vh), dtype=torch.bfloat16, device=dev))
+    dc = _dims_c(dims)
+    st = L.gdn_in_proj(ctypes.byref(dc), T, hidden, _ptr(x), _ptr(w_in), _ptr(qkv), _ptr(z), _ptr(b), _ptr(a),
+                       _stream(dev))
+    _check(st, "gdn_in_proj")
+    return qkv, z, a, b
+
+
+def out_proj(y, w_out, *, dims: Dims = MODEL, out=None):
+    """y bf16 [T, Vh*D] times w_out bf16 [hidden, Vh*D]^T.  Returns out [T, hidden]."""
+    dev = _device_of(y)
+    L = load_library()
+    _need(y, torch.bfloat16, "y", dev)
+    _need(w_out, torch.bfloat16, "w_out", dev)
+    T, hidden = int(y.shape[0]), int(w_out.shape[0])
+    if out is None:
+        out = torch.empty((T, hidden), dtype=torch.bfloat16, device=dev)
+    dc = _dims_c(dims)
+    st = L.gdn_out_proj(ctypes.byref(dc), T, hidden, _ptr(y), _ptr(w_out), _ptr(out), _stream(dev))
+    _check(st, "gdn_out_proj")
+    return out
+
+
 def _slot_tables(slots, n, dev):
     if isinstance(slots, torch.Tensor):
         host = slots.detach().to("cpu", torch.int32).contiguous()
@@ -325,5 +366,5 @@ def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tens
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_varlen", "decode", "decode_multi", "decode_slots", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
+__all__ = ["prefill", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

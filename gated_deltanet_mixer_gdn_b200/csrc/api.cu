@@ -15,6 +15,7 @@
 #include "chunk.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "gemm.cuh"
 #include "prep.cuh"
 
 namespace {
@@ -503,9 +504,76 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
 }
 
 
+// C = A W^T over bf16 A [M][K] and W [N][K], columns routed to the segments of gp.
+int gemm_launch(const uint16_t* A, const uint16_t* W, GemmParams gp, cudaStream_t stream) {
+    if (gp.M == 0 || gp.N == 0) return GDN_OK;
+    if (gp.K <= 0 || gp.K % gemm::BK != 0) return GDN_ERR_UNSUPPORTED;
+    if (!A || !W || !aligned16(A) || !aligned16(W)) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < gp.nseg; ++i)
+        if (gp.seg[i].dst == nullptr || (reinterpret_cast<uintptr_t>(gp.seg[i].dst) & 1u)) return GDN_ERR_INVALID_ARG;
+    int st = check_device();
+    if (st != GDN_OK) return st;
+    CUtensorMap mA, mW;
+    if (!make_map(&mA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)gp.K, (uint64_t)gp.M, gemm::BK, gemm::BM,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)gp.K, (uint64_t)gp.N, gemm::BK, gemm::BN,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return GDN_ERR_CUDA;
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        err = cudaFuncSetAttribute(gdn_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::SMEM_BYTES);
+    });
+    if (err != cudaSuccess) return GDN_ERR_CUDA;
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int64_t ntiles = (int64_t)((gp.M + gemm::BM - 1) / gemm::BM) * ((gp.N + gemm::BN - 1) / gemm::BN);
+    const int grid = (int)(ntiles < nsm ? ntiles : nsm);
+    gdn_gemm_kernel<<<grid, gemm::kThreads, gemm::SMEM_BYTES, stream>>>(mA, mW, gp);
+    return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
+
+int gdn_in_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t* x, const uint16_t* w_in,
+                uint16_t* qkv, uint16_t* z, uint16_t* b, uint16_t* a, void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if (T < 0 || hidden <= 0) return GDN_ERR_INVALID_ARG;
+    if (T == 0) return GDN_OK;
+    const int Vh = dims->num_v_heads, D = dims->head_dim;
+    const int C = (2 * dims->num_k_heads + Vh) * D;
+    GemmParams gp{};
+    gp.M = T;
+    gp.N = C + Vh * D + 2 * Vh;
+    gp.K = hidden;
+    gp.nseg = 4;
+    gp.seg[0] = GemmSegment{0, C, qkv};
+    gp.seg[1] = GemmSegment{C, Vh * D, z};
+    gp.seg[2] = GemmSegment{C + Vh * D, Vh, b};
+    gp.seg[3] = GemmSegment{C + Vh * D + Vh, Vh, a};
+    return gemm_launch(x, w_in, gp, static_cast<cudaStream_t>(stream));
+}
+
+int gdn_out_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t* y, const uint16_t* w_out,
+                 uint16_t* out, void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if (T < 0 || hidden <= 0) return GDN_ERR_INVALID_ARG;
+    if (T == 0) return GDN_OK;
+    GemmParams gp{};
+    gp.M = T;
+    gp.N = hidden;
+    gp.K = dims->num_v_heads * dims->head_dim;
+    gp.nseg = 1;
+    gp.seg[0] = GemmSegment{0, hidden, out};
+    return gemm_launch(y, w_out, gp, static_cast<cudaStream_t>(stream));
+}
+
 
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
     if (check_dims(dims) != GDN_OK || B < 0 || T < 0) return 0;

@@ -183,6 +183,27 @@ int gdn_prefill_varlen_slots(const gdn_dims* dims, const gdn_weights* w, int32_t
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The projections around the mixer as bf16 tensor-core GEMMs with f32
+ * accumulation and one rounding to bf16 (Qwen/Qwen3.8-27B architecture page,
+ * module tree of `linear_attn`: in_proj_qkv 10240x5120, in_proj_z 6144x5120,
+ * in_proj_b and in_proj_a 48x5120, out_proj 5120x6144; row-major weights
+ * [out_features][in_features]).
+ *   gdn_in_proj:  x bf16 [T][hidden]; w_in bf16 [C + Vh*D + 2*Vh][hidden], the
+ *                 rows of in_proj_qkv, in_proj_z, in_proj_b and in_proj_a
+ *                 stacked in that order; writes qkv [T][C], z [T][Vh*D],
+ *                 b [T][Vh] and a [T][Vh] (the mixer's inputs).
+ *   gdn_out_proj: y bf16 [T][Vh*D] (the mixer's output), w_out bf16
+ *                 [hidden][Vh*D]; writes out bf16 [T][hidden].
+ * The contraction width (hidden, or Vh*D) must be a multiple of 64
+ * (GDN_ERR_UNSUPPORTED otherwise); x, y and the weights 16-byte aligned.
+ * T = 0 is a legal no-op.  No workspace; asynchronous on `stream`.
+ */
+int gdn_in_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t* x, const uint16_t* w_in,
+                uint16_t* qkv, uint16_t* z, uint16_t* b, uint16_t* a, void* stream);
+int gdn_out_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t* y, const uint16_t* w_out,
+                 uint16_t* out, void* stream);
+
+/*
  * gdn_prefill without a caller-supplied workspace, for callers that cannot
  * call cudaMalloc: for example a plugin inside an inference engine that owns
  * every device allocation, or a latency-critical path that must not take the

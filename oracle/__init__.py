@@ -172,5 +172,14 @@ def mixer(dims, cu_seqlens, qkv, z, a, b, conv_w, A_log, dt_bias, norm_w,
     return {"out": out, "state": st, "conv": cv}
 
 
+# ---- the projections around the mixer ------------------------------------------
+
+def projection(x, w):
+    """x [T, K] times w [N, K] transposed, in float64: the plain definition of a
+    linear layer y = x W^T (the module tree's in_proj / out_proj, row-major
+    weights [out_features][in_features]); numpy's matmul is the step."""
+    return np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
+
+
 def max_threads() -> int:
     return lib().oracle_max_threads()

@@ -338,3 +338,23 @@ def test_group_case_reproduces_full_mixer_heads():
     assert np.array_equal(part["out"], full["out"][:, hs[0] * D:(hs[-1] + 1) * D])
     assert np.array_equal(part["state"], full["state"][:, hs])
     assert np.array_equal(part["conv"], full["conv"][:, :, sub["channels"].numpy()])
+
+
+def test_projection_is_the_linear_layer_definition():
+    """y[t][n] = sum_k x[t][k] w[n][k]: against an explicit triple loop on a tiny
+    case, the identity weight, and a one-hot row of the weight."""
+    import oracle
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3, 4))
+    w = rng.standard_normal((5, 4))
+    y = oracle.projection(x, w)
+    ref = np.zeros((3, 5))
+    for t in range(3):
+        for n in range(5):
+            for k in range(4):
+                ref[t, n] += x[t, k] * w[n, k]
+    assert y.shape == (3, 5) and np.allclose(y, ref, rtol=0, atol=1e-12)
+    assert np.array_equal(oracle.projection(x, np.eye(4)), x)
+    w1 = np.zeros((2, 4))
+    w1[1, 2] = 1.0
+    assert np.array_equal(oracle.projection(x, w1)[:, 1], x[:, 2]) and not oracle.projection(x, w1)[:, 0].any()
