@@ -7,7 +7,8 @@ whole pass (128 decode launches, 8192 row-tokens).  Metric: row-tokens/s.
 A second measured object, "prefill", times the chunked prefill (one row of
 8192 tokens from zero state, and the 8-row varlen workload) in tokens/s
 against the tensor roofline; a third, "decode_multi", the same decode batch
-with 4 tokens per row per call (gdn_decode_multi).
+with 4 tokens per row per call (gdn_decode_multi); a fourth, "projections",
+the in_proj / out_proj GEMMs around the mixer at the layer's shapes.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -358,6 +359,39 @@ def bench_decode_multi(args, local, k=4):
             "gpu_launches": launches}
 
 
+def bench_projections(args, local, T=8192):
+    """The projections around the mixer at the 27B layer's shapes: in_proj
+    [T,5120] x [16480,5120]^T and out_proj [T,6144] x [5120,6144]^T (bf16, f32
+    accumulation), random inputs; CUDA events on the launching stream, L2 flushed
+    between calls."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    d = synth.MODEL
+    H = 5120
+    N = d.conv_channels + d.value_width + 2 * d.num_v_heads
+    g = torch.Generator(device=dev).manual_seed(7)
+    x = torch.randn((T, H), generator=g, device=dev).to(torch.bfloat16)
+    w_in = (torch.randn((N, H), generator=g, device=dev) * H ** -0.5).to(torch.bfloat16)
+    y = torch.randn((T, d.value_width), generator=g, device=dev).to(torch.bfloat16)
+    w_out = (torch.randn((H, d.value_width), generator=g, device=dev) * d.value_width ** -0.5).to(torch.bfloat16)
+    outs = gdn.in_proj(x, w_in)
+    o = gdn.out_proj(y, w_out)
+    stream = torch.cuda.Stream(dev)
+    res = {}
+    for name, call, flop, shape in (
+            ("in_proj", lambda: gdn.in_proj(x, w_in, out=outs), 2 * T * N * H, f"[{T},{H}] x [{N},{H}]^T"),
+            ("out_proj", lambda: gdn.out_proj(y, w_out, out=o), 2 * T * H * d.value_width,
+             f"[{T},{d.value_width}] x [{H},{d.value_width}]^T")):
+        t, n = _time_prefill(call, dev, stream, max(3, args.warmup), max(5, args.steps))
+        tf = flop / t / 1e12
+        res[name] = {"workload": shape + " bf16, f32 accumulation", "ms": t * 1000.0, "tflops": tf,
+                     "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                  "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"]},
+                     "gpu_launches": n}
+    return res
+
+
 def _time_prefill(call, dev, stream, warmup, reps):
     """Median seconds of `call` (CUDA events on `stream`), L2 flushed before each timed call."""
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > L2, written between iterations
@@ -491,9 +525,11 @@ def main():
         line, case = run_ours(args, world, rank, local)
         pre = bench_prefill(args, world, rank, local, args.prefill_T)
         multi = bench_decode_multi(args, local)
+        proj = bench_projections(args, local)
         if rank == 0:
             line["prefill"] = pre
             line["decode_multi"] = multi
+            line["projections"] = proj
             if world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline_line(case)
             print(json.dumps(line))
