@@ -8,7 +8,9 @@ A second measured object, "prefill", times the chunked prefill (one row of
 8192 tokens from zero state, and the 8-row varlen workload) in tokens/s
 against the tensor roofline; a third, "decode_multi", the same decode batch
 with 4 tokens per row per call (gdn_decode_multi); a fourth, "projections",
-the in_proj / out_proj GEMMs around the mixer at the layer's shapes.
+the in_proj / out_proj GEMMs around the mixer at the layer's shapes; a fifth,
+"prefill_from_hidden", one row of 8192 tokens from the hidden states with the
+load stage inside the in_proj GEMM, beside in_proj followed by the prefill.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -392,6 +394,53 @@ def bench_projections(args, local, T=8192):
     return res
 
 
+def prefill_launches(B, T, nsm=148, Vh=48):
+    """Kernels one dense prefill call launches (the library's schedule): load stage,
+    history out, then WY records + recurrence per segment; rows of >= 16 chunks whose
+    recurrence leaves 32 SMs free run in 2 segments (4 from 32 chunks up)."""
+    per = (T + 63) // 64
+    S = 1
+    if B * Vh + 32 <= nsm and per >= 16:
+        S = 4 if per >= 32 else 2
+    return 2 + 2 * S
+
+
+def bench_hidden(args, local, T=8192):
+    """Prefill of one row of T tokens from the layer's hidden states [T,5120]: the load
+    stage inside the in_proj GEMM (gdn_prefill_hidden) against in_proj followed by the
+    prefill (both on the same inputs, bit-identical results)."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    d = synth.MODEL
+    H = 5120
+    N = d.conv_channels + d.value_width + 2 * d.num_v_heads
+    g = torch.Generator(device=dev).manual_seed(11)
+    w = gdn.weights_to(synth.draw_weights(torch.Generator().manual_seed(11), d), dev)
+    x = torch.randn((1, T, H), generator=g, device=dev).to(torch.bfloat16)
+    w_in = (torch.randn((N, H), generator=g, device=dev) * H ** -0.5).to(torch.bfloat16)
+    out = torch.empty((1, T, d.value_width), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, d.num_v_heads, 128, 128), dtype=torch.float32, device=dev)
+    fc = torch.empty((1, 3, d.conv_channels), dtype=torch.float32, device=dev)
+    proj = gdn.in_proj(x[0], w_in)
+    stream = torch.cuda.Stream(dev)
+
+    def unfused():
+        gdn.in_proj(x[0], w_in, out=proj)
+        q, z, a, b = (t.unsqueeze(0) for t in proj)
+        gdn.prefill(q, z, a, b, w, out=out, final_state=fs, final_conv=fc)
+
+    reps = max(5, args.steps)
+    tf, nf = _time_prefill(lambda: gdn.prefill_hidden(x, w_in, w, out=out, final_state=fs, final_conv=fc),
+                           dev, stream, max(3, args.warmup), reps)
+    tu, nu = _time_prefill(unfused, dev, stream, max(3, args.warmup), reps)
+    k = prefill_launches(1, T)
+    return {"workload": f"prefill B=1 T={T} from hidden states [{T},{H}] (in_proj 5120->{N} + mixer), "
+                        "zero initial state",
+            "fused": {"value": T / tf, "unit": "tokens/s", "ms": tf * 1000.0, "gpu_launches": (k - 1) * nf},
+            "unfused": {"value": T / tu, "unit": "tokens/s", "ms": tu * 1000.0, "gpu_launches": (k + 1) * nu},
+            "l2": "flushed (256 MiB write) before each timed call"}
+
+
 def _time_prefill(call, dev, stream, warmup, reps):
     """Median seconds of `call` (CUDA events on `stream`), L2 flushed before each timed call."""
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > L2, written between iterations
@@ -436,8 +485,8 @@ def bench_prefill(args, world, rank, local, T):
                              "algorithmic_flop_per_token": PREFILL_FLOP_PER_TOKEN},
                 "l2": "flushed (256 MiB write) before each timed call", "gpu_launches": launches}
 
-    # launches per call: load stage, history out, WY records, recurrence (+ chunk offsets for packed rows)
-    out = {"b1": line(T, t1, f"prefill B=1 T={T}, zero initial state", 4 * n1)}
+    # launches per call: see prefill_launches (packed rows: load stage, history out, chunk offsets, WY, recurrence)
+    out = {"b1": line(T, t1, f"prefill B=1 T={T}, zero initial state", prefill_launches(1, T) * n1)}
     if T == 8192:
         vcase = synth.config(3)
         vw = gdn.weights_to(vcase["weights"], dev)
@@ -474,7 +523,8 @@ def bench_long_context(args, local, line):
     reps = max(3, min(args.steps, 5))
     t, n = _time_prefill(lambda: gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w, out=out, final_state=fs,
                                              final_conv=fc), dev, stream, 3, reps)
-    res = line(B * T, t, f"long-context prefill B={B} T={T}, zero initial state, final states returned", 4 * n)
+    res = line(B * T, t, f"long-context prefill B={B} T={T}, zero initial state, final states returned",
+               prefill_launches(B, T) * n)
     # 256 decode steps per row from the prefill's states (2 rows: launch-latency bound, reported)
     steps = case["decode"]["qkv"].shape[0]
     dq = {k: case["decode"][k].to(dev) for k in ("qkv", "z", "a", "b")}
@@ -526,10 +576,12 @@ def main():
         pre = bench_prefill(args, world, rank, local, args.prefill_T)
         multi = bench_decode_multi(args, local)
         proj = bench_projections(args, local)
+        hid = bench_hidden(args, local)
         if rank == 0:
             line["prefill"] = pre
             line["decode_multi"] = multi
             line["projections"] = proj
+            line["prefill_from_hidden"] = hid
             if world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline_line(case)
             print(json.dumps(line))

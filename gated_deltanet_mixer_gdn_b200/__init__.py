@@ -27,7 +27,8 @@ LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen_workspace_size",
            "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
-           "gdn_in_proj", "gdn_out_proj", "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string",
+           "gdn_in_proj", "gdn_out_proj", "gdn_prefill_hidden_workspace_size", "gdn_prefill_hidden",
+           "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string",
            "gdn_version")
 
 GDN_OK = 0
@@ -74,6 +75,10 @@ def load_library() -> ctypes.CDLL:
         L.gdn_decode.argtypes = [dp, wp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.gdn_in_proj.restype = ctypes.c_int
         L.gdn_in_proj.argtypes = [dp, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.gdn_prefill_hidden_workspace_size.restype = sz
+        L.gdn_prefill_hidden_workspace_size.argtypes = [dp, i32, i32]
+        L.gdn_prefill_hidden.restype = ctypes.c_int
+        L.gdn_prefill_hidden.argtypes = [dp, wp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_out_proj.restype = ctypes.c_int
         L.gdn_out_proj.argtypes = [dp, i32, i32, vp, vp, vp, vp]
         L.gdn_decode_multi.restype = ctypes.c_int
@@ -278,6 +283,42 @@ def in_proj(x, w_in, *, dims: Dims = MODEL, out=None):
     return qkv, z, a, b
 
 
+def prefill_hidden(x, w_in, weights, init_state=None, init_conv=None, *, out=None, final_state=None,
+                   final_conv=None, dims: Dims = MODEL, in_place: bool = False):
+    """Dense prefill from the layer's hidden states: x bf16 [B,T,hidden] through the stacked in_proj
+    weights w_in (rows of qkv, z, b, a) into the mixer, the load stage running inside the in_proj GEMM.
+    Returns (out bf16 [B,T,Vh*D] before out_proj, final_state f32 [B,Vh,D,D], final_conv f32 [B,W-1,C]);
+    the same results, bit for bit, as in_proj followed by prefill."""
+    dev = _device_of(x)
+    L = load_library()
+    _need(x, torch.bfloat16, "x", dev)
+    _need(w_in, torch.bfloat16, "w_in", dev)
+    B, T, hidden = int(x.shape[0]), int(x.shape[1]), int(x.shape[2])
+    C, VD, Vh, D, Wm = dims.conv_channels, dims.value_width, dims.num_v_heads, dims.head_dim, dims.conv_width - 1
+    if tuple(w_in.shape) != (C + VD + 2 * Vh, hidden):
+        raise ValueError("prefill_hidden: w_in shape")
+    if init_state is not None:
+        _need(init_state, torch.float32, "init_state", dev)
+    if init_conv is not None:
+        _need(init_conv, torch.float32, "init_conv", dev)
+    if out is None:
+        out = torch.empty((B, T, VD), dtype=torch.bfloat16, device=dev)
+    if final_state is None:
+        final_state = init_state if (in_place and init_state is not None) else \
+            torch.empty((B, Vh, D, D), dtype=torch.float32, device=dev)
+    if final_conv is None:
+        final_conv = init_conv if (in_place and init_conv is not None) else \
+            torch.empty((B, Wm, C), dtype=torch.float32, device=dev)
+    dc = _dims_c(dims)
+    ws_bytes = L.gdn_prefill_hidden_workspace_size(ctypes.byref(dc), B, T)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    st = L.gdn_prefill_hidden(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), B, T, hidden,
+                              _ptr(x), _ptr(w_in), _ptr(init_state), _ptr(init_conv), _ptr(out),
+                              _ptr(final_state), _ptr(final_conv), _ptr(ws), ws_bytes, _stream(dev))
+    _check(st, "gdn_prefill_hidden")
+    return out, final_state, final_conv
+
+
 def out_proj(y, w_out, *, dims: Dims = MODEL, out=None):
     """y bf16 [T, Vh*D] times w_out bf16 [hidden, Vh*D]^T.  Returns out [T, hidden]."""
     dev = _device_of(y)
@@ -366,5 +407,5 @@ def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tens
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
+__all__ = ["prefill", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "gemm.cuh"
+#include "inproj.cuh"
 #include "prep.cuh"
 
 namespace {
@@ -146,6 +147,19 @@ int side_streams(int dev, SideStreams** out) {
     return GDN_OK;
 }
 
+int gemm_setup(const void* kernel_fn);  // defined with the GEMM launches below
+
+// The load stage fused into the in_proj GEMM: the hidden states and the
+// stacked in_proj weights go in; the staged operands, z and the rows' last
+// pre-conv tokens come out (z and the latter into workspace buffers).
+struct FusedLoad {
+    const uint16_t* x;     // bf16 [total][hidden]
+    const uint16_t* w_in;  // bf16 [C + Vh*128 + 2*Vh][hidden]
+    int hidden;
+    uint16_t* z;           // bf16 [total][Vh*128]
+    float* conv_last;      // f32 [N][3][C]
+};
+
 // Everything one prefill call launches, with the workspace carved and the
 // tensor maps built once.
 struct PrefillPlan {
@@ -158,6 +172,7 @@ struct PrefillPlan {
     uint16_t* out;
     const float* norm_w;
     const int* slots;  // state / history row of each packed row, or nullptr
+    const FusedLoad* fused;  // load stage inside the in_proj GEMM (dense rows), or nullptr
     __half *Qs, *Ks, *Ql, *Kl, *Vs;
     float *Gs, *Bs;
     int* chunk_base;
@@ -166,6 +181,7 @@ struct PrefillPlan {
 
     int prep(int tok_begin, int tok_end, cudaStream_t st) const {
         if (tok_end <= tok_begin) return GDN_OK;
+        if (fused != nullptr) return fused_prep(st);  // always the whole range
         PrepParams pp{};
         pp.Kh = Kh;
         pp.Vh = Vh;
@@ -193,8 +209,47 @@ struct PrefillPlan {
         gdn_prep_kernel<<<grid, 256, 0, st>>>(pp);
         return cuda_status(cudaGetLastError());
     }
+    // in_proj + load stage over all tokens: 128-row tiles advancing by 125 tokens
+    int fused_prep(cudaStream_t st) const {
+        GemmParams gp{};
+        gp.M = total;
+        gp.N = C + Vh * 128 + 2 * Vh;
+        gp.K = fused->hidden;
+        FusedPrep f{};
+        f.Kh = Kh;
+        f.Vh = Vh;
+        f.T = uniform_T;
+        f.conv_w = w->conv_w;
+        f.A_log = w->A_log;
+        f.dt_bias = w->dt_bias;
+        f.init_conv = init_conv;
+        f.Qs = Qs;
+        f.Ks = Ks;
+        f.Ql = Ql;
+        f.Kl = Kl;
+        f.Vs = Vs;
+        f.Gs = Gs;
+        f.Bs = Bs;
+        f.z = fused->z;
+        f.conv_last = fused->conv_last;
+        CUtensorMap mA, mW;
+        if (!make_map(&mA, fused->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)gp.K, (uint64_t)gp.M, gemm::BK,
+                      gemm::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mW, fused->w_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)gp.K, (uint64_t)gp.N, gemm::BK,
+                      gemm::BN, CU_TENSOR_MAP_SWIZZLE_128B))
+            return GDN_ERR_CUDA;
+        int rc = gemm_setup(reinterpret_cast<const void*>(gdn_gemm_kernel<1>));
+        if (rc != GDN_OK) return rc;
+        const int64_t ntiles = (int64_t)((gp.M + gemm::BM - 4) / (gemm::BM - 3)) * ((gp.N + gemm::BN - 1) / gemm::BN);
+        const int grid = (int)(ntiles < nsm ? ntiles : nsm);
+        gdn_gemm_kernel<1><<<grid, gemm::kThreads, gemm::SMEM_BYTES, st>>>(mA, mW, gp, f);
+        return cuda_status(cudaGetLastError());
+    }
     int conv_out(cudaStream_t st) const {
         if (final_conv == nullptr) return GDN_OK;
+        if (fused != nullptr)  // the rows' last three tokens, staged by the fused load stage
+            return cuda_status(cudaMemcpyAsync(final_conv, fused->conv_last, (size_t)N * 3 * C * 4,
+                                               cudaMemcpyDeviceToDevice, st));
         ConvOutParams cp{};
         cp.C = C;
         cp.N = N;
@@ -267,7 +322,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                  int32_t total, int64_t nchunks, int64_t nchunks_planned, const uint16_t* qkv, const uint16_t* z,
                  const uint16_t* a, const uint16_t* b, const float* init_state, const float* init_conv, uint16_t* out,
                  float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-                 bool may_overlap, const int32_t* slots_dev = nullptr) {
+                 bool may_overlap, const int32_t* slots_dev = nullptr, const FusedLoad* fused = nullptr) {
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
     const int C = (2 * Kh + Vh) * 128;
     const size_t state_bytes = (size_t)N * Vh * 128 * 128 * 4;
@@ -318,6 +373,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     P.out = out;
     P.norm_w = w->norm_w;
     P.slots = slots_dev;
+    P.fused = fused;
     P.Qs = reinterpret_cast<__half*>(wsb + ws.off_q);
     P.Ks = reinterpret_cast<__half*>(wsb + ws.off_k);
     P.Ql = reinterpret_cast<__half*>(wsb + ws.off_ql);
@@ -504,6 +560,22 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
 }
 
 
+// Dynamic shared memory opt-in of a GEMM kernel instance, once per instance and device.
+int gemm_setup(const void* kernel_fn) {
+    static std::mutex mu;
+    static std::vector<std::pair<const void*, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto& d : done)
+        if (d.first == kernel_fn && d.second == dev) return GDN_OK;
+    if (cudaFuncSetAttribute(kernel_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::SMEM_BYTES) !=
+        cudaSuccess)
+        return GDN_ERR_CUDA;
+    done.emplace_back(kernel_fn, dev);
+    return GDN_OK;
+}
+
 // C = A W^T over bf16 A [M][K] and W [N][K], columns routed to the segments of gp.
 int gemm_launch(const uint16_t* A, const uint16_t* W, GemmParams gp, cudaStream_t stream) {
     if (gp.M == 0 || gp.N == 0) return GDN_OK;
@@ -519,20 +591,53 @@ int gemm_launch(const uint16_t* A, const uint16_t* W, GemmParams gp, cudaStream_
         !make_map(&mW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)gp.K, (uint64_t)gp.N, gemm::BK, gemm::BN,
                   CU_TENSOR_MAP_SWIZZLE_128B))
         return GDN_ERR_CUDA;
-    static std::once_flag once;
-    static cudaError_t err = cudaSuccess;
-    std::call_once(once, [] {
-        err = cudaFuncSetAttribute(gdn_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::SMEM_BYTES);
-    });
-    if (err != cudaSuccess) return GDN_ERR_CUDA;
+    st = gemm_setup(reinterpret_cast<const void*>(gdn_gemm_kernel<0>));
+    if (st != GDN_OK) return st;
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
     const int64_t ntiles = (int64_t)((gp.M + gemm::BM - 1) / gemm::BM) * ((gp.N + gemm::BN - 1) / gemm::BN);
     const int grid = (int)(ntiles < nsm ? ntiles : nsm);
-    gdn_gemm_kernel<<<grid, gemm::kThreads, gemm::SMEM_BYTES, stream>>>(mA, mW, gp);
+    gdn_gemm_kernel<0><<<grid, gemm::kThreads, gemm::SMEM_BYTES, stream>>>(mA, mW, gp, FusedPrep{});
     return cuda_status(cudaGetLastError());
+}
+
+// Workspace of gdn_prefill_hidden: the prefill workspace, then z, then either the
+// rows' staged histories (fused load stage) or the unfused in_proj outputs.
+struct HiddenLayout {
+    bool fused;
+    size_t off_z, off_conv, off_qkv, off_b, off_a, bytes;
+};
+
+// The fused load stage needs whole 256-column tiles of qkv and z, b and a in one
+// tile, and rows of at least 3 tokens (the history after a row is then its own tokens).
+bool fused_load_ok(const gdn_dims* d, int32_t T) {
+    const int Kh = d->num_k_heads, Vh = d->num_v_heads;
+    return T >= 3 && (2 * Kh + Vh) % 2 == 0 && Vh % 2 == 0 && 2 * Vh <= gemm::BN;
+}
+
+HiddenLayout hidden_layout(const gdn_dims* d, int32_t B, int32_t T) {
+    HiddenLayout L{};
+    const int64_t total = (int64_t)B * T;
+    const int Kh = d->num_k_heads, Vh = d->num_v_heads;
+    const size_t C = (size_t)(2 * Kh + Vh) * 128;
+    L.fused = fused_load_ok(d, T);
+    L.off_z = plan_workspace(d, total, B, (int64_t)B * ((T + 63) / 64)).bytes;
+    size_t o = L.off_z + align_up((size_t)total * Vh * 128 * 2);
+    if (L.fused) {
+        L.off_conv = o;
+        o += align_up((size_t)B * 3 * C * 4);
+    } else {
+        L.off_qkv = o;
+        o += align_up((size_t)total * C * 2);
+        L.off_b = o;
+        o += align_up((size_t)total * Vh * 2);
+        L.off_a = o;
+        o += align_up((size_t)total * Vh * 2);
+    }
+    L.bytes = o;
+    return L;
 }
 
 }  // namespace
@@ -574,6 +679,53 @@ int gdn_out_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t
     return gemm_launch(y, w_out, gp, static_cast<cudaStream_t>(stream));
 }
 
+
+size_t gdn_prefill_hidden_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
+    if (check_dims(dims) != GDN_OK || B < 0 || T < 0) return 0;
+    if ((int64_t)B * T > INT32_MAX) return 0;
+    return hidden_layout(dims, B, T).bytes;
+}
+
+int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, int32_t hidden,
+                       const uint16_t* x, const uint16_t* w_in, const float* init_state, const float* init_conv,
+                       uint16_t* out, float* final_state, float* final_conv, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (B < 0 || T < 0 || B > 65535 || hidden <= 0) return GDN_ERR_INVALID_ARG;
+    if (hidden % gemm::BK != 0) return GDN_ERR_UNSUPPORTED;
+    const int64_t total = (int64_t)B * T;
+    if (total > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (total > 0 && (!x || !w_in || !out || !aligned16(x) || !aligned16(w_in) || !aligned16(out)))
+        return GDN_ERR_INVALID_ARG;
+    const void* fs[4] = {init_state, init_conv, final_state, final_conv};
+    for (const void* p : fs)
+        if (p != nullptr && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    if ((st = check_device()) != GDN_OK) return st;
+    const HiddenLayout L = hidden_layout(dims, B, T);
+    if (total > 0 && (workspace == nullptr || workspace_bytes < L.bytes)) return GDN_ERR_WORKSPACE;
+    if (workspace != nullptr && !aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    const int64_t nch = (int64_t)B * ((T + 63) / 64);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint16_t* z = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_z) : nullptr;
+    if (total > 0 && L.fused) {
+        FusedLoad fl{x, w_in, hidden, z, reinterpret_cast<float*>(wsb + L.off_conv)};
+        return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, nullptr, z, nullptr, nullptr,
+                            init_state, init_conv, out, final_state, final_conv, workspace, L.off_z, s, true, nullptr,
+                            &fl);
+    }
+    // rows shorter than the conv window (or head counts the fused tiles do not cover):
+    // in_proj into the workspace, then the prefill over it
+    uint16_t* qkv = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_qkv) : nullptr;
+    uint16_t* bb = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_b) : nullptr;
+    uint16_t* aa = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_a) : nullptr;
+    if (total > 0 && (st = gdn_in_proj(dims, (int32_t)total, hidden, x, w_in, qkv, z, bb, aa, stream)) != GDN_OK)
+        return st;
+    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, aa, bb, init_state, init_conv, out,
+                        final_state, final_conv, workspace, total > 0 ? L.off_z : 0, s, true);
+}
 
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
     if (check_dims(dims) != GDN_OK || B < 0 || T < 0) return 0;

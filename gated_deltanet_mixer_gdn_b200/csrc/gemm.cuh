@@ -11,7 +11,9 @@
 // W K-slices (64 wide, 128B swizzle) into a 4-stage ring, one warp issues
 // tcgen05.mma (M = 128, N = 256, bf16) into one of two TMEM accumulators, and
 // four warps drain the other accumulator (tcgen05.ld, round to bf16, store)
-// while the next tile is multiplied.
+// while the next tile is multiplied.  The fused instance (FUSED = 1, see
+// inproj.cuh) runs the mixer's load stage in that epilogue instead of storing
+// the projection.
 #pragma once
 
 #include "common.cuh"
@@ -30,13 +32,29 @@ struct GemmParams {
     GemmSegment seg[4];
 };
 
+// The load stage fused into the in_proj epilogue (see inproj.cuh).
+struct FusedPrep {
+    int Kh, Vh, T;                 // dense rows of T tokens
+    const uint16_t* conv_w;        // bf16 [C][4]
+    const float* A_log;            // [Vh]
+    const float* dt_bias;          // [Vh]
+    const float* init_conv;        // f32 [rows][3][C] or nullptr
+    __half *Qs, *Ks, *Ql, *Kl, *Vs;
+    float *Gs, *Bs;                // [Vh][M]
+    uint16_t* z;                   // bf16 [M][Vh*128]
+    float* conv_last;              // f32 [rows][3][C]: pre-conv values of each row's last three tokens
+};
+
 namespace gemm {
 constexpr int BM = 128, BN = 256, BK = 64, kStages = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t OFF_MISC = kStages * STAGE_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 256 + 1024;
+constexpr int kXStride = 36;  // floats per row of the epilogue's exchange buffer (32 + 4: no bank conflicts)
+constexpr uint32_t XBUF_BYTES = BM * kXStride * 4;       // 32 columns of every tile row
+constexpr uint32_t SCRATCH_BYTES = XBUF_BYTES + 256 * 16;  // + the tile's conv taps as f32
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 256 + SCRATCH_BYTES + 1024;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators
 // bf16 A and B (format 1), f32 accumulator, both K-major, M = 128, N = 256
@@ -46,17 +64,27 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uin
 constexpr int B_FULL = 0, B_EMPTY = kStages, B_ACCF = 2 * kStages, B_ACCE = 2 * kStages + 2;
 }  // namespace gemm
 
+template <int FUSED>
+__device__ void fused_prep_epilogue(const FusedPrep& f, const GemmParams& p, uint32_t tacc, int r0, int n0,
+                                    uint8_t* scratch, int q4, int lane);
+
+// FUSED = 0: plain C = A W^T.  FUSED = 1: in_proj with the load stage in the
+// epilogue; M tiles then start 3 rows early (each 128-row tile yields 125
+// tokens whose conv window lies inside the tile).
+template <int FUSED>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gdn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-                    const GemmParams p) {
+                    const GemmParams p, const FusedPrep f) {
     using namespace gemm;
+    constexpr int kStepM = FUSED ? BM - 3 : BM;  // tokens per M tile
+    constexpr int kLead = FUSED ? 3 : 0;        // rows of the tile before its first output token
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_MISC);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 128);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tiles_m = (p.M + BM - 1) / BM, tiles_n = (p.N + BN - 1) / BN;
+    const int tiles_m = (p.M + kStepM - 1) / kStepM, tiles_n = (p.N + BN - 1) / BN;
     const int ntiles = tiles_m * tiles_n;
     const int ksteps = p.K / BK;
 
@@ -94,7 +122,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         if (lane == 0) {
             uint32_t q = 0;  // ring position over all tiles
             for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-                const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+                const int m0 = (t % tiles_m) * kStepM - kLead, n0 = (t / tiles_m) * BN;  // m0 < 0: zero rows
                 for (int ks = 0; ks < ksteps; ++ks, ++q) {
                     const int s = q % kStages;
                     if (q >= kStages) wait1(B_EMPTY + s, ((q / kStages) - 1) & 1);
@@ -137,10 +165,17 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
             const int ab = it & 1;
-            const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+            const int m0 = (t % tiles_m) * kStepM - kLead, n0 = (t / tiles_m) * BN;
             wait1(B_ACCF + ab, (it >> 1) & 1);
             __syncwarp();
             tc_fence_after();
+            if constexpr (FUSED != 0) {
+                fused_prep_epilogue<FUSED>(f, p, tbase + tl + ab * BN, m0, n0, smem + OFF_MISC + 256, q4, lane);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_ACCE + ab]);
+                continue;
+            }
             const int row = m0 + 32 * q4 + lane;
 #pragma unroll 1
             for (int j = 0; j < BN / 32; ++j) {

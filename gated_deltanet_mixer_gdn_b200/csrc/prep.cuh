@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
         }
         float xs[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) xs[e] = act[e] * scale;
+        for (int e = 0; e < 4; ++e) xs[e] = __fmul_rn(act[e], scale);  // rounded product (no contraction into the lo split)
         uint2 pk;
         pk.x = pack_half2(xs[0], xs[1]);
         pk.y = pack_half2(xs[2], xs[3]);

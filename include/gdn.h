@@ -204,6 +204,29 @@ int gdn_out_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t
                  uint16_t* out, void* stream);
 
 /*
+ * Dense prefill from the layer's hidden states: gdn_in_proj and gdn_prefill
+ * in one call, with the load stage (conv + silu, q/k L2 norms, gates; model
+ * card, "Gated DeltaNet" bullet) computed inside the in_proj GEMM's epilogue,
+ * so that qkv, a and b never reach HBM.  Same arithmetic, in the same order,
+ * as gdn_in_proj followed by gdn_prefill: the results are bit-identical.
+ *   x      bf16 [B*T][hidden] (B rows of T tokens), hidden a multiple of 64
+ *   w_in   bf16 [C + Vh*D + 2*Vh][hidden] (as for gdn_in_proj)
+ *   init_state, init_conv, out, final_state, final_conv: as for gdn_prefill
+ *          (out is the mixer's output, before out_proj; NULL and in-place
+ *          rules as there).
+ * workspace: gdn_prefill_hidden_workspace_size(dims, B, T) bytes, 16-byte
+ * aligned (it also holds z).  Rows shorter than 3 tokens, or head counts
+ * whose q/k/v or z widths are not whole 256-column tiles, take the unfused
+ * pair of launches inside the same call (the workspace size accounts for it).
+ * Returns GDN_ERR_UNSUPPORTED for hidden % 64 != 0; otherwise as gdn_prefill.
+ */
+size_t gdn_prefill_hidden_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
+int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, int32_t hidden,
+                       const uint16_t* x, const uint16_t* w_in, const float* init_state, const float* init_conv,
+                       uint16_t* out, float* final_state, float* final_conv, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
  * gdn_prefill without a caller-supplied workspace, for callers that cannot
  * call cudaMalloc: for example a plugin inside an inference engine that owns
  * every device allocation, or a latency-critical path that must not take the
