@@ -557,8 +557,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
-                    help="decode: the 64-row decode batch (default line); prefill: only the chunked prefill")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "hidden"],
+                    help="decode: the 64-row decode batch (default line); prefill: only the chunked prefill; "
+                         "hidden: only the prefill from hidden states (fused in_proj + load stage)")
     ap.add_argument("--prefill-T", type=int, default=PREFILL_T, help="tokens of the prefill measurement")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -567,6 +568,11 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.workload == "hidden":
+            hid = bench_hidden(args, local)
+            if rank == 0:
+                print(json.dumps({"metric": "GDN prefill from hidden states tokens/s", **hid}))
+            return 0
         if args.workload == "prefill":
             pre = bench_prefill(args, world, rank, local, args.prefill_T)
             if rank == 0:

@@ -6,8 +6,8 @@
 // with the columns of C routed to up to four output tensors (in_proj writes
 // qkv, z, b and a from one product over the stacked weights).
 //
-// Persistent CTAs walk 128 x 256 output tiles (M-fastest, so consecutive
-// tiles share the weight tile in L2).  One warp issues the TMA loads of A and
+// Persistent CTAs walk 128 x 256 output tiles (grouped: 16 M tiles swept across
+// all N tiles, so a round's operands stay in L2).  One warp issues the TMA loads of A and
 // W K-slices (64 wide, 128B swizzle) into a 4-stage ring, one warp issues
 // tcgen05.mma (M = 128, N = 256, bf16) into one of two TMEM accumulators, and
 // four warps drain the other accumulator (tcgen05.ld, round to bf16, store)
@@ -63,6 +63,20 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uin
 // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[2]
 constexpr int B_FULL = 0, B_EMPTY = kStages, B_ACCF = 2 * kStages, B_ACCE = 2 * kStages + 2;
 }  // namespace gemm
+
+// Tile t of the walk -> (M tile, N tile).  Groups of kGroupM M tiles are swept across all
+// N tiles, M-fastest inside the group: a round of the persistent grid then touches about
+// kGroupM row blocks of A and ~148 / kGroupM weight tiles, a working set that stays in L2,
+// instead of streaming all of A for every weight tile.
+constexpr int kGroupM = 32;
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+    const int per_group = kGroupM * tiles_n;
+    const int g = t / per_group;
+    const int r = t - g * per_group;
+    const int gm = min(kGroupM, tiles_m - g * kGroupM);
+    tn = r / gm;
+    tm = g * kGroupM + (r - tn * gm);
+}
 
 template <int FUSED>
 __device__ void fused_prep_epilogue(const FusedPrep& f, const GemmParams& p, uint32_t tacc, int r0, int n0,
@@ -122,7 +136,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         if (lane == 0) {
             uint32_t q = 0;  // ring position over all tiles
             for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-                const int m0 = (t % tiles_m) * kStepM - kLead, n0 = (t / tiles_m) * BN;  // m0 < 0: zero rows
+                int tm, tn;
+                tile_coords(t, tiles_m, tiles_n, tm, tn);
+                const int m0 = tm * kStepM - kLead, n0 = tn * BN;  // m0 < 0: zero rows
                 for (int ks = 0; ks < ksteps; ++ks, ++q) {
                     const int s = q % kStages;
                     if (q >= kStages) wait1(B_EMPTY + s, ((q / kStages) - 1) & 1);
@@ -165,7 +181,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
             const int ab = it & 1;
-            const int m0 = (t % tiles_m) * kStepM - kLead, n0 = (t / tiles_m) * BN;
+            int tm, tn;
+            tile_coords(t, tiles_m, tiles_n, tm, tn);
+            const int m0 = tm * kStepM - kLead, n0 = tn * BN;
             wait1(B_ACCF + ab, (it >> 1) & 1);
             __syncwarp();
             tc_fence_after();
