@@ -71,8 +71,13 @@ struct PrepParams {
     float* Bs;
 };
 
+template <bool B>
+struct Flag {
+    static constexpr bool value = B;
+};
+
 constexpr int kPrepTokens = 16;  // consecutive tokens per thread
-constexpr int kPrepAhead = 8;    // rows loaded ahead of the token being computed
+constexpr int kPrepAhead = 4;    // rows loaded ahead of the token being computed
 constexpr int kPrepSlots = 8;    // head slots (warps) per CTA
 
 __device__ __forceinline__ void unpack4(const uint2 v, float (&x)[4]) {
@@ -153,68 +158,84 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
         fetch_xbar(n, s + 2, t0 - 1, w2);
     }
 
+    // The token loop, instantiated for v / q-k slots and for blocks that lie inside one row
+    // (FAST: no row start to watch for, no ragged end, so the 16 tokens are straight-line
+    // code the compiler can interleave) or not.
+    auto run = [&](auto v_flag, auto fast_flag) {
+        constexpr bool IS_V = decltype(v_flag)::value;
+        constexpr bool FAST = decltype(fast_flag)::value;
 #pragma unroll
-    for (int tt = 0; tt < kPrepTokens; ++tt) {
-        if (tt >= nt) break;
-        const int t = t0 + tt;
-        float xn[4];
-        unpack4(ahead[tt % kPrepAhead], xn);
-        if (tt + kPrepAhead < nt)
-            ahead[tt % kPrepAhead] =
-                __ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)(t + kPrepAhead) * p.C + ch0));
-        if (t == start + len) {  // a new row starts here (skip empty rows): restart from its history
-            if (p.seq.cu == nullptr) {
-                ++n;
-                start += len;
-            } else {
-                do {
+        for (int tt = 0; tt < kPrepTokens; ++tt) {
+            if (!FAST && tt >= nt) break;
+            const int t = t0 + tt;
+            float xn[4];
+            unpack4(ahead[tt % kPrepAhead], xn);
+            if (FAST ? (tt + kPrepAhead < kPrepTokens) : (tt + kPrepAhead < nt))
+                ahead[tt % kPrepAhead] =
+                    __ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)(t + kPrepAhead) * p.C + ch0));
+            if (!FAST && t == start + len) {  // a new row starts here (skip empty rows): restart from its history
+                if (p.seq.cu == nullptr) {
                     ++n;
-                    start = __ldg(p.seq.cu + n);
-                    len = __ldg(p.seq.cu + n + 1) - start;
-                } while (len == 0);
+                    start += len;
+                } else {
+                    do {
+                        ++n;
+                        start = __ldg(p.seq.cu + n);
+                        len = __ldg(p.seq.cu + n + 1) - start;
+                    } while (len == 0);
+                }
+                fetch_xbar(n, 0, 0, w0);
+                fetch_xbar(n, 1, 0, w1);
+                fetch_xbar(n, 2, 0, w2);
             }
-            fetch_xbar(n, 0, 0, w0);
-            fetch_xbar(n, 1, 0, w1);
-            fetch_xbar(n, 2, 0, w2);
-        }
-        float act[4];
-        float ss = 0.f;
+            float act[4];
+            float ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float cv = fmaf(w[0][e], w0[e], fmaf(w[1][e], w1[e], fmaf(w[2][e], w2[e], w[3][e] * xn[e])));
-            act[e] = silu_f(cv);
-            ss = fmaf(act[e], act[e], ss);
-            w0[e] = w1[e];
-            w1[e] = w2[e];
-            w2[e] = xn[e];
-        }
-        float scale = 1.0f;
-        if (!is_v) {  // warp-uniform
+            for (int e = 0; e < 4; ++e) {
+                const float cv = fmaf(w[0][e], w0[e], fmaf(w[1][e], w1[e], fmaf(w[2][e], w2[e], w[3][e] * xn[e])));
+                act[e] = silu_f(cv);
+                ss = fmaf(act[e], act[e], ss);
+                w0[e] = w1[e];
+                w1[e] = w2[e];
+                w2[e] = xn[e];
+            }
+            float scale = 1.0f;
+            if constexpr (!IS_V) {
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            scale = rsqrtf(ss + kEps);
-            if (is_q) scale *= rsqrtf((float)kD);
-        }
-        float xs[4];
+                for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                scale = rsqrtf(ss + kEps);
+                if (is_q) scale *= rsqrtf((float)kD);
+            }
+            float xs[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) xs[e] = __fmul_rn(act[e], scale);  // rounded product (no contraction into the lo split)
-        uint2 pk;
-        pk.x = pack_half2(xs[0], xs[1]);
-        pk.y = pack_half2(xs[2], xs[3]);
-        if (is_v) {
-            *reinterpret_cast<uint2*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + lane * 4) = pk;
-        } else {
-            const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + lane * 4;
-            const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&pk.x));
-            const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&pk.y));
-            uint2 lo;
-            lo.x = pack_half2(xs[0] - h0.x, xs[1] - h0.y);
-            lo.y = pack_half2(xs[2] - h1.x, xs[3] - h1.y);
-            *reinterpret_cast<uint2*>((is_q ? p.Qs : p.Ks) + off) = pk;
-            *reinterpret_cast<uint2*>((is_q ? p.Ql : p.Kl) + off) = lo;
+            for (int e = 0; e < 4; ++e) xs[e] = __fmul_rn(act[e], scale);  // rounded product (no contraction into the lo split)
+            uint2 pk;
+            pk.x = pack_half2(xs[0], xs[1]);
+            pk.y = pack_half2(xs[2], xs[3]);
+            if constexpr (IS_V) {
+                *reinterpret_cast<uint2*>(p.Vs + (size_t)t * p.Vh * kD + vh * kD + lane * 4) = pk;
+            } else {
+                const size_t off = (size_t)t * p.Kh * kD + (is_q ? slot : slot - p.Kh) * kD + lane * 4;
+                const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&pk.x));
+                const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&pk.y));
+                uint2 lo;
+                lo.x = pack_half2(xs[0] - h0.x, xs[1] - h0.y);
+                lo.y = pack_half2(xs[2] - h1.x, xs[3] - h1.y);
+                *reinterpret_cast<uint2*>((is_q ? p.Qs : p.Ks) + off) = pk;
+                *reinterpret_cast<uint2*>((is_q ? p.Ql : p.Kl) + off) = lo;
+            }
         }
+    };
+    const bool fast = nt == kPrepTokens && t0 + kPrepTokens <= start + len;  // CTA-uniform
+    if (is_v) {
+        if (fast) run(Flag<true>{}, Flag<true>{});
+        else run(Flag<true>{}, Flag<false>{});
+    } else {
+        if (fast) run(Flag<false>{}, Flag<true>{});
+        else run(Flag<false>{}, Flag<false>{});
     }
 }
+
 
 struct ConvOutParams {
     int C, N;
