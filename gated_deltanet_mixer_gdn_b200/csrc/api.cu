@@ -160,6 +160,77 @@ struct FusedLoad {
     float* conv_last;      // f32 [N][3][C]
 };
 
+// Segment plan of the overlapped dense prefill.  Segment 0's WY records run on
+// every SM; after that, the recurrence of segment k (one CTA per row and value
+// head) runs beside the WY records of segment k+1 on the remaining SMs.  The plan
+// is picked on the host by simulating candidate plans with a cost model of this
+// library's kernels measured on B200: a WY launch takes about 11.2 us per wave of
+// tasks (a task: one chunk, one q/k head, up to 3 of its value heads) plus 4 us; a
+// recurrence launch about 9.5 us plus 2.3 us per chunk (the WY figure as measured beside a
+// running recurrence; erring slow keeps the recurrence from waiting).  Candidates: segment sizes
+// growing or shrinking geometrically (s_k = s_0 rho^k: rho > 1 lets the recurrence
+// start early when it bounds the call, rho < 1 runs most WY records on every SM
+// first when they bound it), 2..kMaxSegments segments of at least one chunk.
+// Returns the segment count (1: no overlap pays) and fills cs[0..S].
+namespace seg_model {
+constexpr double kWaveUs = 11.2, kWyFixedUs = 4.0, kChainFixedUs = 9.5, kChainChunkUs = 2.3;
+}
+
+double simulate_segments(const int* cs, int S, int tasks_per_chunk, int nsm, int chain_ctas) {
+    using namespace seg_model;
+    auto wy_us = [&](int chunks, int P) {
+        const int64_t tasks = (int64_t)chunks * tasks_per_chunk;
+        return kWaveUs * (double)((tasks + P - 1) / P) + kWyFixedUs;
+    };
+    double wy_end = wy_us(cs[1] - cs[0], nsm), chain_end = 0.0;
+    for (int k = 0; k < S; ++k) {
+        const double start = chain_end > wy_end ? chain_end : wy_end;
+        chain_end = start + kChainFixedUs + kChainChunkUs * (cs[k + 1] - cs[k]);
+        if (k + 1 < S) wy_end += wy_us(cs[k + 2] - cs[k + 1], nsm - chain_ctas);
+    }
+    return chain_end;
+}
+
+int plan_segments(int per, int N, int Kh, int Vh, int nsm, int* cs) {
+    const int tasks_per_chunk = N * Kh * ((Vh / Kh + wy::kHeads - 1) / wy::kHeads);
+    const int chain_ctas = N * Vh;
+    // no overlap: every WY record on every SM, then one recurrence launch
+    int best_S = 1;
+    double best = 0.0;
+    {
+        const int one[2] = {0, per};
+        best = simulate_segments(one, 1, tasks_per_chunk, nsm, nsm);
+    }
+    int best_cs[kMaxSegments + 1] = {0, per};
+    static const double kRho[] = {0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8, 0.9, 1.0, 1.1, 1.2, 1.35, 1.5, 1.75, 2.0};
+    const int max_S = per < kMaxSegments ? per : kMaxSegments;
+    for (int S = 2; S <= max_S; ++S) {
+        for (double rho : kRho) {
+            int c[kMaxSegments + 1];
+            double total = 0.0, f = 1.0;
+            for (int k = 0; k < S; ++k, f *= rho) total += f;
+            double acc = 0.0;
+            f = 1.0;
+            c[0] = 0;
+            for (int k = 1; k <= S; ++k, f *= rho) {
+                acc += f / total * per;
+                const int v = (int)(acc + 0.5);
+                const int lo = c[k - 1] + 1, hi = per - (S - k);  // every segment keeps at least one chunk
+                c[k] = v < lo ? lo : (v > hi ? hi : v);
+            }
+            c[S] = per;
+            const double t = simulate_segments(c, S, tasks_per_chunk, nsm, chain_ctas);
+            if (t < best) {
+                best = t;
+                best_S = S;
+                for (int k = 0; k <= S; ++k) best_cs[k] = c[k];
+            }
+        }
+    }
+    for (int k = 0; k <= best_S; ++k) cs[k] = best_cs[k];
+    return best_S;
+}
+
 // Everything one prefill call launches, with the workspace carved and the
 // tensor maps built once.
 struct PrefillPlan {
@@ -408,8 +479,9 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     const int per = cu_dev ? 0 : (uniform_T + 63) / 64;
     const int chain_ctas = N * Vh;
     int S = 1;
+    int cs[kMaxSegments + 1];
     if (may_overlap && cu_dev == nullptr && final_state != nullptr && chain_ctas + 32 <= nsm && per >= 16)
-        S = per >= 4 * kMaxSegments ? 4 : 2;
+        S = plan_segments(per, N, Kh, Vh, nsm, cs);
     if (S > 1) {
         std::lock_guard<std::mutex> lock(g_side_mu);
         SideStreams* ss = nullptr;
@@ -418,8 +490,6 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         if (cudaEventRecord(ss->fork, stream) != cudaSuccess || cudaStreamWaitEvent(ss->prod, ss->fork, 0) != cudaSuccess ||
             cudaStreamWaitEvent(ss->chain, ss->fork, 0) != cudaSuccess)
             return GDN_ERR_CUDA;
-        int cs[kMaxSegments + 1];
-        for (int k = 0; k <= S; ++k) cs[k] = (int)((int64_t)k * per / S);
         if ((st = P.prep(0, total, ss->prod)) != GDN_OK) return st;
         if ((st = P.conv_out(ss->prod)) != GDN_OK) return st;  // after the load stage read the history
         for (int k = 0; k < S; ++k) {
