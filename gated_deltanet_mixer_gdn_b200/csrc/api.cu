@@ -108,7 +108,7 @@ Workspace plan_workspace(const gdn_dims* d, int64_t total, int64_t N, int64_t nc
     w.off_g = w.off_v + align_up(vv);
     w.off_b = w.off_g + align_up(gb);
     w.off_cb = w.off_b + align_up(gb);
-    w.off_rec = w.off_cb + align_up((size_t)(N + 1) * 4);
+    w.off_rec = w.off_cb + align_up((size_t)(2 * N + 1) * 4);  // chunk bases [N+1], then the row order [N]
     w.bytes = w.off_rec + align_up((size_t)nchunks * d->num_v_heads * wy::REC_BYTES);
     return w;
 }
@@ -247,6 +247,7 @@ struct PrefillPlan {
     __half *Qs, *Ks, *Ql, *Kl, *Vs;
     float *Gs, *Bs;
     int* chunk_base;
+    int* order;  // recurrence row order (packed rows), or nullptr
     uint8_t* rec;
     CUtensorMap mK, mQ, mKl, mQl, mV, mZ, mO;
 
@@ -368,6 +369,7 @@ struct PrefillPlan {
         cp.total = total;
         cp.seq = seq;
         cp.chunk_base = chunk_base;
+        cp.order = order;
         cp.rec = rec;
         cp.init_state = init_state;
         cp.final_state = final_state;
@@ -453,6 +455,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     P.Gs = reinterpret_cast<float*>(wsb + ws.off_g);
     P.Bs = reinterpret_cast<float*>(wsb + ws.off_b);
     P.chunk_base = cu_dev ? reinterpret_cast<int*>(wsb + ws.off_cb) : nullptr;
+    P.order = cu_dev ? P.chunk_base + N + 1 : nullptr;
     P.rec = wsb + ws.off_rec;
     if (!make_map(&P.mK, P.Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -516,7 +519,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     if (st != GDN_OK) return st;
     if ((st = P.conv_out(stream)) != GDN_OK) return st;  // 2. final history (after the load stage read it)
     if (P.chunk_base != nullptr) {                        // 3. first chunk of every packed row
-        gdn_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu_dev, N, P.chunk_base);
+        gdn_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu_dev, N, P.chunk_base, P.order);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     if ((st = P.wy_records(nchunks, 0, 0, nsm, stream)) != GDN_OK) return st;  // 4. WY records, all chunks

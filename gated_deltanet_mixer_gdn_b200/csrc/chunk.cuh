@@ -47,6 +47,7 @@ struct ChunkParams {
     uint16_t* out;            // bf16 [total][Vh*128]
     int c0, c1;               // chunk window [c0, c1) of every row (c1 < 0: to the end of the row)
     const int* slots;         // [N] state row of each packed row (validated by the host), or nullptr
+    const int* order;         // [N] packed row of each grid row (longest first), or nullptr: grid row = row
 };
 
 namespace chunk {
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int h = blockIdx.x;
-    const int n = blockIdx.y;
+    const int n = p.order ? __ldg(p.order + blockIdx.y) : (int)blockIdx.y;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int kap = h / (p.Vh / p.Kh);

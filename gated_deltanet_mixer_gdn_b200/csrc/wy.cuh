@@ -221,7 +221,11 @@ __device__ __forceinline__ float chunk_cumsum(float g, float* sG, int p, int lan
 
 // cb[n] = number of 64-token chunks in rows 0..n-1 (cb[0] = 0, cb[N] = all),
 // from cu_seqlens; one block of 1024 threads walks the rows in tiles.
-__global__ void __launch_bounds__(1024) gdn_chunk_base_kernel(const int* cu, int N, int* cb) {
+// ord[0..N): the rows by length, longest first (ties: lower index first), by a bitonic
+// sort in shared memory when N <= kOrderMax; otherwise the identity.  The recurrence
+// launches its rows in this order, so the longest rows are not left for the last wave.
+constexpr int kOrderMax = 2048;
+__global__ void __launch_bounds__(1024) gdn_chunk_base_kernel(const int* cu, int N, int* cb, int* ord) {
     __shared__ int s_warp[32];
     __shared__ int s_carry;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -258,6 +262,35 @@ __global__ void __launch_bounds__(1024) gdn_chunk_base_kernel(const int* cu, int
         if (tid == 1023) s_carry = incl;
         __syncthreads();
     }
+    if (ord == nullptr) return;
+    if (N > kOrderMax) {
+        for (int i = tid; i < N; i += 1024) ord[i] = i;
+        return;
+    }
+    __shared__ unsigned long long s_key[kOrderMax];
+    int P = 2;
+    while (P < N) P <<= 1;
+    for (int i = tid; i < P; i += 1024) {  // key: (INT_MAX - length, index); padding sorts last
+        const int len = i < N ? __ldg(cu + i + 1) - __ldg(cu + i) : 0;
+        s_key[i] = i < N ? ((unsigned long long)(0x7fffffff - len) << 32) | (unsigned)i : ~0ull;
+    }
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += 1024) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const unsigned long long x = s_key[i], y = s_key[ixj];
+                    if ((x > y) == ((i & k) == 0)) {
+                        s_key[i] = y;
+                        s_key[ixj] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = tid; i < N; i += 1024) ord[i] = (int)(s_key[i] & 0xffffffffu);
 }
 
 // Row n and chunk index c of global chunk g.
