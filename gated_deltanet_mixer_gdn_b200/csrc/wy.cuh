@@ -54,20 +54,24 @@ constexpr uint32_t REC_DEC = 32768;       // f32 e^{G_C - G_t} [64], e^{G_t} [64
 constexpr uint32_t REC_DEC_BYTES = 528;
 constexpr uint32_t REC_BYTES = REC_DEC + REC_DEC_BYTES;
 // shared memory (bytes from a 1024-aligned base)
+// two input buffers (b = 0, 1 at b * IN_STRIDE), filled two tasks ahead
+constexpr uint32_t IN_STRIDE = 65536;
 constexpr uint32_t OFF_KQ = 0;            // [K t0-63 | Q t0-63] x k 0-63, then x k 64-127: f16 hi parts
-constexpr uint32_t OFF_LO = 32768;        // same layout, lo parts; then T diag(beta e^G) f16 per warpgroup
-constexpr uint32_t OFF_WG = 65536;        // per warpgroup: A / T f32 [64][LDA] and the solve scratch
+constexpr uint32_t OFF_LO = 32768;        // same layout, lo parts
+constexpr uint32_t OFF_T2 = 2 * IN_STRIDE;  // T diag(beta e^G) f16 [64][64], 8 KB per warpgroup
+constexpr uint32_t OFF_WG = OFF_T2 + kHeads * 8192;  // per warpgroup: A / T f32 [64][LDA] and the solve scratch
 constexpr uint32_t WG_BYTES = 64 * LDA * 4 + 32 * 36 * 4;
 constexpr uint32_t OFF_MISC = OFF_WG + kHeads * WG_BYTES;
 constexpr uint32_t MISC_BYTES = 4096;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
 // misc: 0 barriers, 128 TMEM slot, 256 + 1024 * wg: G[64], e^G[64], beta[64], column decays[64]
-constexpr uint32_t T_KQ = 0;              // [K;Q] K^T, 64 columns; then W^T of warpgroup w at 64 (w + 1)
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t T_KQ = 0;              // [K;Q] K^T, 64 columns, of even tasks; W^T of warpgroup w at 64 (w + 1)
+constexpr uint32_t T_KQ1 = 256;           // [K;Q] K^T of odd tasks (issued during the task before)
+constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IN_BYTES = 8 * 8192;
 constexpr uint32_t ID_KK = idesc_f16_f32(128, 64, false, false, false);
 constexpr uint32_t ID_AMN = idesc_f16_f32(128, 64, true, false, false);
-constexpr int B_IN = 0, B_MMA1 = 1, B_FREE = 2, B_W = 3;  // B_W + warpgroup
+constexpr int B_IN = 0, B_MMA1 = 2, B_FREE = 4, B_W = 6;  // B_IN, B_MMA1, B_FREE + buffer; B_W + warpgroup
 constexpr int kBars = B_W + kHeads;
 }  // namespace wy
 
@@ -335,16 +339,19 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
     float* scol = sG + 192;  // e^{G_r - G_j}, r the last token of j's 16-token block
     float* sA = reinterpret_cast<float*>(smem + OFF_WG + wg * WG_BYTES);
     float* sP = sA + 64 * LDA;
-    uint8_t* sT2 = smem + OFF_LO + 8192 * wg;
+    uint8_t* sT2 = smem + OFF_T2 + 8192 * wg;
 
     const int ratio = p.Vh / p.Kh;
     const int nsub = (ratio + kHeads - 1) / kHeads;
     const int ntasks = p.nchunks * p.Kh * nsub;
 
     if (tid == 0) {
-        mbar_init(&bars[B_IN], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars[B_IN + b], 1);
+            mbar_init(&bars[B_FREE + b], kHeads);
+        }
         mbar_init(&bars[B_MMA1], 1);
-        mbar_init(&bars[B_FREE], kHeads);
+        mbar_init(&bars[B_MMA1 + 1], 1);
         for (int w = 0; w < kHeads; ++w) mbar_init(&bars[B_W + w], 1);
         fence_barrier_init();
         prefetch_tensormap(&tmK);
@@ -373,24 +380,29 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             g = (g / p.win) * per + p.c0 + g % p.win;
         }
     };
-    auto issue_loads = [&](int task) {
+    auto issue_loads = [&](int task, int b) {
         int g, kap, sub, n, c;
         task_coords(task, g, kap, sub);
         chunk_row(p, g, n, c);
         int start, len;
         p.seq.bounds(n, start, len);
         const int y = start + c * C;
-        mbar_arrive_expect_tx(&bars[B_IN], IN_BYTES);
-        tma_load_2d(smem + OFF_KQ, &tmK, kap * 128, y, &bars[B_IN]);
-        tma_load_2d(smem + OFF_KQ + 16384, &tmK, kap * 128 + 64, y, &bars[B_IN]);
-        tma_load_2d(smem + OFF_KQ + 8192, &tmQ, kap * 128, y, &bars[B_IN]);
-        tma_load_2d(smem + OFF_KQ + 24576, &tmQ, kap * 128 + 64, y, &bars[B_IN]);
-        tma_load_2d(smem + OFF_LO, &tmKl, kap * 128, y, &bars[B_IN]);
-        tma_load_2d(smem + OFF_LO + 16384, &tmKl, kap * 128 + 64, y, &bars[B_IN]);
-        tma_load_2d(smem + OFF_LO + 8192, &tmQl, kap * 128, y, &bars[B_IN]);
-        tma_load_2d(smem + OFF_LO + 24576, &tmQl, kap * 128 + 64, y, &bars[B_IN]);
+        uint8_t* in = smem + b * IN_STRIDE;
+        uint64_t* full = &bars[B_IN + b];
+        mbar_arrive_expect_tx(full, IN_BYTES);
+        tma_load_2d(in + OFF_KQ, &tmK, kap * 128, y, full);
+        tma_load_2d(in + OFF_KQ + 16384, &tmK, kap * 128 + 64, y, full);
+        tma_load_2d(in + OFF_KQ + 8192, &tmQ, kap * 128, y, full);
+        tma_load_2d(in + OFF_KQ + 24576, &tmQ, kap * 128 + 64, y, full);
+        tma_load_2d(in + OFF_LO, &tmKl, kap * 128, y, full);
+        tma_load_2d(in + OFF_LO + 16384, &tmKl, kap * 128 + 64, y, full);
+        tma_load_2d(in + OFF_LO + 8192, &tmQl, kap * 128, y, full);
+        tma_load_2d(in + OFF_LO + 24576, &tmQl, kap * 128 + 64, y, full);
     };
-    if (tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
+    if (tid == 0) {  // the first two tasks of this CTA
+        if ((int)blockIdx.x < ntasks) issue_loads(blockIdx.x, 0);
+        if ((int)(blockIdx.x + gridDim.x) < ntasks) issue_loads(blockIdx.x + gridDim.x, 1);
+    }
 
     bool broken = false;
     auto wait = [&](int slot, uint32_t parity) {
@@ -429,9 +441,40 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
     float gv_next, bv_next;
     load_gates(blockIdx.x, gv_next, bv_next);
 
+    // MMA1 of the task in input buffer b: [K;Q] K^T from hi/lo f16 parts into accumulator b
+    // (one thread).  The task's own MMA1 was issued during the task before it, so the
+    // tensor core runs it while that task solves its triangular system.
+    auto issue_mma1 = [&](int b, uint32_t parity) {
+        wait1(B_IN + b, parity);
+        tc_fence_after();
+        const uint32_t aKQ = sbase + b * IN_STRIDE + OFF_KQ, aLO = sbase + b * IN_STRIDE + OFF_LO;
+        const uint32_t d = tbase + (b ? T_KQ1 : T_KQ);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+            mma_f16(d, sw128_desc(aKQ + off, 16, 1024), sw128_desc(aKQ + off, 16, 1024), ID_KK, s > 0);
+        }
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+            mma_f16(d, sw128_desc(aKQ + off, 16, 1024), sw128_desc(aLO + off, 16, 1024), ID_KK, 1);
+        }
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+            mma_f16(d, sw128_desc(aLO + off, 16, 1024), sw128_desc(aKQ + off, 16, 1024), ID_KK, 1);
+        }
+        mma_commit(&bars[B_MMA1 + b]);
+    };
+    if (tid == 0 && (int)blockIdx.x < ntasks) issue_mma1(0, 0);
+    __syncwarp();
+
     uint32_t it = 0;
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x, ++it) {
-        const uint32_t ph = it & 1;
+        const uint32_t ph = it & 1;          // barriers used once per task
+        const int buf = it & 1;              // input buffer of this task
+        const uint32_t pb = (it >> 1) & 1;   // barriers of that buffer: used every other task
+        const uint32_t in_base = sbase + buf * IN_STRIDE;
         int g, kap, sub, n, c;
         task_coords(task, g, kap, sub);
         chunk_row(p, g, n, c);
@@ -449,30 +492,6 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         (void)tok0;
         (void)nv;
 
-        // ---- MMA1: [K;Q] K^T from hi/lo f16 parts (runs while the gates are formed)
-        if (tid == 0) {
-            wait1(B_IN, ph);
-            tc_fence_after();
-            const uint32_t aKQ = sbase + OFF_KQ, aLO = sbase + OFF_LO;
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                mma_f16(tbase + T_KQ, sw128_desc(aKQ + off, 16, 1024), sw128_desc(aKQ + off, 16, 1024), ID_KK, s > 0);
-            }
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                mma_f16(tbase + T_KQ, sw128_desc(aKQ + off, 16, 1024), sw128_desc(aLO + off, 16, 1024), ID_KK, 1);
-            }
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                mma_f16(tbase + T_KQ, sw128_desc(aLO + off, 16, 1024), sw128_desc(aKQ + off, 16, 1024), ID_KK, 1);
-            }
-            mma_commit(&bars[B_MMA1]);
-        }
-        __syncwarp();
-
         // ---- gates: G, e^G, beta, the column decays; the decay part of the record
         if (active) {
             const float Gi = chunk_cumsum(gv, sG, wt, lane, wbar, 128);
@@ -488,12 +507,12 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             }
             named_barrier_sync(wbar, 128);
         }
-        wait(B_MMA1, ph);
+        wait(B_MMA1 + buf, pb);
         tc_fence_after();
 
         if (!active) {
             // nothing to do for this slot; the input buffer is not read by it
-            if (wt == 0) mbar_arrive(&bars[B_FREE]);
+            if (wt == 0) mbar_arrive(&bars[B_FREE + buf]);
             __syncwarp();
         } else {
             // ---- A (rows of K K^T) and M (rows of Q K^T), masked before the exp
@@ -516,7 +535,7 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
-                    tmem_ld32(tlane + T_KQ + 32 * hh, v);
+                    tmem_ld32(tlane + (buf ? T_KQ1 : T_KQ) + 32 * hh, v);
                     tmem_ld_wait();
                     float e[32];
 #pragma unroll
@@ -537,6 +556,11 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
                 }
             }
             named_barrier_sync(wbar, 128);
+            tc_fence_before();
+            // the next task's MMA1 (its accumulator was last read two tasks ago, and every
+            // warpgroup has passed that task's MMA3)
+            if (tid == 0 && task + (int)gridDim.x < ntasks) issue_mma1(buf ^ 1, ((it + 1) >> 1) & 1);
+            __syncwarp();
 
             // ---- T = (I + A)^-1; T diag(beta) to the record, T diag(beta e^G) to shared memory
             // (over the lo tiles, which only MMA1 reads)
@@ -564,18 +588,18 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
                 const uint32_t tW = tbase + 64 * (wg + 1);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_f16(tW, sw128_desc(sbase + OFF_KQ + s * 2048, 16384, 1024),
+                    mma_f16(tW, sw128_desc(in_base + OFF_KQ + s * 2048, 16384, 1024),
                             sw128_desc(smem_u32(sT2) + s * 32, 16, 1024), ID_AMN, s > 0);
                 mma_commit(&bars[B_W + wg]);
-                mma_commit(&bars[B_FREE]);
+                mma_commit(&bars[B_FREE + buf]);
             }
             __syncwarp();
         }
 
-        // ---- once every slot is done with the input tiles, fetch the next task's
+        // ---- once every slot is done with this buffer, fill it with the task after next
         if (tid == 0) {
-            wait1(B_FREE, ph);
-            if (task + (int)gridDim.x < ntasks) issue_loads(task + gridDim.x);
+            wait1(B_FREE + buf, pb);
+            if (task + 2 * (int)gridDim.x < ntasks) issue_loads(task + 2 * gridDim.x, buf);
         }
         __syncwarp();
 
