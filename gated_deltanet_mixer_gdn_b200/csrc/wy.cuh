@@ -524,6 +524,10 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
                 const float Gr = sG[i], scale = is_a ? sbeta[i] : 1.f;
                 // e^{G_i - G_j} = e^{G_i - G_r} e^{G_r - G_j} for j in an earlier block (r its last
                 // token, both factors <= 1); direct exponentials inside the row's own block
+                // the first half of the row is read from TMEM while the exponentials are formed
+                const uint32_t tkq = tlane + (buf ? T_KQ1 : T_KQ);
+                float v[32];
+                tmem_ld32(tkq, v);
                 float rowf[3], diag[16];
 #pragma unroll
                 for (int J = 0; J < 3; ++J) rowf[J] = (J < I) ? scale * __expf(Gr - sG[16 * J + 15]) : 0.f;
@@ -534,8 +538,7 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
                 }
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    float v[32];
-                    tmem_ld32(tlane + (buf ? T_KQ1 : T_KQ) + 32 * hh, v);
+                    if (hh == 1) tmem_ld32(tkq + 32, v);
                     tmem_ld_wait();
                     float e[32];
 #pragma unroll
@@ -607,7 +610,10 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         if (active) {
             wait(B_W + wg, ph);
             tc_fence_after();
-            uint8_t* dst = rec + REC_MW + (row >> 6) * 8192 + (row & 7) * 2;
+            // Lanes k (even) and k + 1 swap halves of their packed token pairs, so that the even
+            // lane stores columns k, k + 1 of token t and the odd lane those of token t + 1.
+            const uint32_t odd = row & 1;
+            uint8_t* dst = rec + REC_MW + (row >> 6) * 8192 + (row & 6) * 2;
             const uint32_t kc = (row & 63) >> 3;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -615,10 +621,11 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
                 tmem_ld32(tlane + 64 * (wg + 1) + 32 * hh, v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {  // one paired conversion for tokens j, j + 1
+                for (int j = 0; j < 32; j += 2) {  // tokens 32 hh + j, + 1 of column k = row
                     const uint32_t pr = pack_half2(-v[j], -v[j + 1]);
-                    *reinterpret_cast<uint16_t*>(dst + sw128_chunk(32 * hh + j, kc)) = static_cast<uint16_t>(pr);
-                    *reinterpret_cast<uint16_t*>(dst + sw128_chunk(32 * hh + j + 1, kc)) = static_cast<uint16_t>(pr >> 16);
+                    const uint32_t q = __shfl_xor_sync(0xffffffffu, pr, 1);
+                    const uint32_t word = odd ? ((q >> 16) | (pr & 0xffff0000u)) : ((pr & 0xffffu) | (q << 16));
+                    *reinterpret_cast<uint32_t*>(dst + sw128_chunk(32 * hh + j + odd, kc)) = word;
                 }
             }
             tc_fence_before();
