@@ -394,15 +394,11 @@ def bench_projections(args, local, T=8192):
     return res
 
 
-def prefill_launches(B, T, nsm=148, Vh=48):
-    """Kernels one dense prefill call launches (the library's schedule): load stage,
-    history out, then WY records + recurrence per segment; rows of >= 16 chunks whose
-    recurrence leaves 32 SMs free run in 2 segments (4 from 32 chunks up)."""
-    per = (T + 63) // 64
-    S = 1
-    if B * Vh + 32 <= nsm and per >= 16:
-        S = 4 if per >= 32 else 2
-    return 2 + 2 * S
+def prefill_launches(B, T):
+    """Kernels one dense prefill call (final state returned) launches, from the library's own
+    schedule: load stage, history writer, then WY records + recurrence per segment."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    return 2 + 2 * gdn.prefill_segments(B, T)
 
 
 def bench_hidden(args, local, T=8192):

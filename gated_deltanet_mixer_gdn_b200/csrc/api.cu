@@ -231,6 +231,15 @@ int plan_segments(int per, int N, int Kh, int Vh, int nsm, int* cs) {
     return best_S;
 }
 
+// Segments of an overlapped dense prefill of N rows of T tokens (1: the plain schedule):
+// the overlap needs a recurrence that leaves at least 32 SMs to the WY records and rows
+// of at least 16 chunks.
+int dense_segments(int Kh, int Vh, int N, int T, int nsm, int* cs) {
+    const int per = (T + 63) / 64;
+    if (N * Vh + 32 > nsm || per < 16) return 1;
+    return plan_segments(per, N, Kh, Vh, nsm, cs);
+}
+
 // Everything one prefill call launches, with the workspace carved and the
 // tensor maps built once.
 struct PrefillPlan {
@@ -479,12 +488,10 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     // persistent grid that leaves the recurrence its SMs) while the recurrence of
     // segment s runs on the high-priority one, each segment's recurrence starting from
     // the state the previous one left in final_state.
-    const int per = cu_dev ? 0 : (uniform_T + 63) / 64;
     const int chain_ctas = N * Vh;
     int S = 1;
     int cs[kMaxSegments + 1];
-    if (may_overlap && cu_dev == nullptr && final_state != nullptr && chain_ctas + 32 <= nsm && per >= 16)
-        S = plan_segments(per, N, Kh, Vh, nsm, cs);
+    if (may_overlap && cu_dev == nullptr && final_state != nullptr) S = dense_segments(Kh, Vh, N, uniform_T, nsm, cs);
     if (S > 1) {
         std::lock_guard<std::mutex> lock(g_side_mu);
         SideStreams* ss = nullptr;
@@ -798,6 +805,20 @@ int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, in
         return st;
     return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, aa, bb, init_state, init_conv, out,
                         final_state, final_conv, workspace, total > 0 ? L.off_z : 0, s, true);
+}
+
+int gdn_prefill_segments(const gdn_dims* dims, int32_t B, int32_t T) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if (B < 0 || T < 0 || B > 65535 || (int64_t)B * T > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return 0;
+    if ((st = check_device()) != GDN_OK) return st;
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    int cs[kMaxSegments + 1];
+    return dense_segments(dims->num_k_heads, dims->num_v_heads, B, T, nsm, cs);
 }
 
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {

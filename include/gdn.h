@@ -96,6 +96,19 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
                 uint16_t* out, float* final_state, float* final_conv,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Schedule of a dense gdn_prefill (B rows x T tokens) that returns its final
+ * state, on the current device: the number S of recurrence segments.  S = 1
+ * is the plain schedule on the caller's stream; S > 1 overlaps the WY records
+ * of segment s+1 with the recurrence of segment s on internal streams (the
+ * segment sizes come from a cost model of the kernels; see gdn_prefill).
+ * Such a call launches 2 + 2*S kernels (load stage, history writer, S WY
+ * launches, S recurrence launches); gdn_prefill_hidden launches 1 + 2*S.
+ * Returns 0 for an empty call, a negative status for invalid arguments or an
+ * unsupported device.  Host-only: enqueues nothing.
+ */
+int gdn_prefill_segments(const gdn_dims* dims, int32_t B, int32_t T);
+
 /* Bytes of device workspace gdn_prefill_varlen needs for N rows with
  * total_T tokens in all.  Returns 0 for invalid dims. */
 size_t gdn_prefill_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T);
