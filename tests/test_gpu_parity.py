@@ -158,6 +158,26 @@ def test_varlen_ragged_rows():
     _check_prefill(case, res, oracle_prefill(case))
 
 
+@pytest.mark.parametrize("n", [1500, 2100])
+def test_varlen_many_short_rows(n):
+    """Thousands of packed rows of 0-5 tokens and one of 200: the recurrence launches rows
+    longest first (a device-side sort up to 2048 rows, the identity above), which must not
+    change any row's result.  Oracle on value head 0 (zero initial state and history)."""
+    rng = np.random.default_rng(n)
+    lengths = [int(x) for x in rng.integers(0, 6, n)]
+    lengths[n // 3] = 200
+    case = synth.prefill_case(900 + n, lengths, init=False)
+    w, acts, _, _ = to_dev(case)
+    out, fs, fc = gdn.prefill_varlen(case["cu_seqlens"], acts["qkv"], acts["z"], acts["a"], acts["b"], w)
+    torch.cuda.synchronize()
+    ref = oracle_prefill(case, heads=(0, 1))
+    assert out_err(out[:, :128], ref["out"]) <= OUT_TOL
+    assert out_rms_err(out[:, :128], ref["out"]) <= OUT_RMS_TOL
+    assert state_err(fs[:, 0:1], ref["state"]) <= STATE_TOL
+    assert conv_exact(fc, ref["conv"])
+    assert gdn.last_device_error() == 0
+
+
 def test_varlen_zero_initial_state():
     case = synth.prefill_case(82, [5, 90, 33], init=False)
     w, acts, _, _ = to_dev(case)
