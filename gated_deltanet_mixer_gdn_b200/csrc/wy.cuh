@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             __syncwarp();
 
             // ---- T = (I + A)^-1; T diag(beta) to the record, T diag(beta e^G) to shared memory
-            // (over the lo tiles, which only MMA1 reads)
+            // (the warpgroup's own 8 KB, read by its MMA3)
             wy_tsolve(sA, sP, wt, wbar);
             {
                 const int t = wt >> 1, hh = wt & 1;
