@@ -394,11 +394,11 @@ def bench_projections(args, local, T=8192):
     return res
 
 
-def prefill_launches(B, T):
+def prefill_launches(B, T, from_hidden=False):
     """Kernels one dense prefill call (final state returned) launches, from the library's own
-    schedule: load stage, history writer, then WY records + recurrence per segment."""
+    schedule (load stage, history writer, WY records and recurrence per segment)."""
     import gated_deltanet_mixer_gdn_b200 as gdn
-    return 2 + 2 * gdn.prefill_segments(B, T)
+    return gdn.prefill_schedule(B, T, from_hidden)[1]
 
 
 def bench_hidden(args, local, T=8192):
@@ -429,11 +429,12 @@ def bench_hidden(args, local, T=8192):
     tf, nf = _time_prefill(lambda: gdn.prefill_hidden(x, w_in, w, out=out, final_state=fs, final_conv=fc),
                            dev, stream, max(3, args.warmup), reps)
     tu, nu = _time_prefill(unfused, dev, stream, max(3, args.warmup), reps)
-    k = prefill_launches(1, T)
     return {"workload": f"prefill B=1 T={T} from hidden states [{T},{H}] (in_proj 5120->{N} + mixer), "
                         "zero initial state",
-            "fused": {"value": T / tf, "unit": "tokens/s", "ms": tf * 1000.0, "gpu_launches": (k - 1) * nf},
-            "unfused": {"value": T / tu, "unit": "tokens/s", "ms": tu * 1000.0, "gpu_launches": (k + 1) * nu},
+            "fused": {"value": T / tf, "unit": "tokens/s", "ms": tf * 1000.0,
+                      "gpu_launches": prefill_launches(1, T, True) * nf},
+            "unfused": {"value": T / tu, "unit": "tokens/s", "ms": tu * 1000.0,
+                        "gpu_launches": (1 + prefill_launches(1, T)) * nu},
             "l2": "flushed (256 MiB write) before each timed call"}
 
 

@@ -25,7 +25,7 @@ from .synth import Dims, MODEL
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
-EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_segments", "gdn_prefill_varlen_workspace_size",
+EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_schedule", "gdn_prefill_varlen_workspace_size",
            "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
            "gdn_in_proj", "gdn_out_proj", "gdn_prefill_hidden_workspace_size", "gdn_prefill_hidden",
            "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string",
@@ -68,8 +68,8 @@ def load_library() -> ctypes.CDLL:
         L.gdn_prefill_varlen_workspace_size.restype = sz
         L.gdn_prefill_varlen_workspace_size.argtypes = [dp, i32, i32]
         L.gdn_prefill.restype = ctypes.c_int
-        L.gdn_prefill_segments.restype = ctypes.c_int
-        L.gdn_prefill_segments.argtypes = [dp, i32, i32]
+        L.gdn_prefill_schedule.restype = ctypes.c_int
+        L.gdn_prefill_schedule.argtypes = [dp, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
         L.gdn_prefill.argtypes = [dp, wp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_prefill_varlen.restype = ctypes.c_int
         L.gdn_prefill_varlen.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -184,15 +184,16 @@ def prefill(qkv, z, a, b, weights, init_state=None, init_conv=None, *, out=None,
     return out, final_state, final_conv
 
 
-def prefill_segments(B: int, T: int, dims: Dims = MODEL) -> int:
-    """Recurrence segments of a dense prefill of B x T tokens that returns its final state on
-    the current device (1: plain schedule); such a call launches 2 + 2 * segments kernels."""
+def prefill_schedule(B: int, T: int, from_hidden: bool = False, dims: Dims = MODEL):
+    """(segments, launches) of a dense prefill of B x T tokens that returns its final state, on
+    the current device: recurrence segments of the overlapped schedule (1: plain) and the number
+    of kernels the call launches (prefill, or prefill_hidden with from_hidden)."""
     L = load_library()
     dc = _dims_c(dims)
-    st = L.gdn_prefill_segments(ctypes.byref(dc), int(B), int(T))
-    if st < 0:
-        _check(st, "gdn_prefill_segments")
-    return st
+    seg, lau = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(L.gdn_prefill_schedule(ctypes.byref(dc), int(B), int(T), int(bool(from_hidden)), ctypes.byref(seg),
+                                  ctypes.byref(lau)), "gdn_prefill_schedule")
+    return seg.value, lau.value
 
 
 def prefill_varlen(cu_seqlens, qkv, z, a, b, weights, init_state=None, init_conv=None, *, out=None,
@@ -420,5 +421,5 @@ def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tens
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_segments", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
+__all__ = ["prefill", "prefill_schedule", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

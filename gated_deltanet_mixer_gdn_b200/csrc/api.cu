@@ -160,85 +160,86 @@ struct FusedLoad {
     float* conv_last;      // f32 [N][3][C]
 };
 
-// Segment plan of the overlapped dense prefill.  Segment 0's WY records run on
-// every SM; after that, the recurrence of segment k (one CTA per row and value
-// head) runs beside the WY records of segment k+1 on the remaining SMs.  The plan
-// is picked on the host by simulating candidate plans with a cost model of this
-// library's kernels measured on B200: a WY launch takes about 11.2 us per wave of
-// tasks (a task: one chunk, one q/k head, up to 3 of its value heads) plus 4 us; a
-// recurrence launch about 9.5 us plus 2.3 us per chunk (the WY figure as measured beside a
-// running recurrence; erring slow keeps the recurrence from waiting).  Candidates: segment sizes
-// growing or shrinking geometrically (s_k = s_0 rho^k: rho > 1 lets the recurrence
-// start early when it bounds the call, rho < 1 runs most WY records on every SM
-// first when they bound it), 2..kMaxSegments segments of at least one chunk.
-// Returns the segment count (1: no overlap pays) and fills cs[0..S].
+// Segment plan of the overlapped dense prefill.  The load stage runs over all
+// tokens first; segment 0's WY records run on every SM; after that, the recurrence
+// of segment k (one CTA per row and value head) runs beside the WY records of
+// segment k+1 on the remaining SMs.  The plan is picked on the host by simulating
+// candidate plans with a cost model of this library's kernels measured on B200: a
+// WY launch takes about 11.2 us per wave of tasks (a task: one chunk, one q/k head,
+// up to 3 of its value heads) plus 4 us; a recurrence launch about 9.5 us plus 2.3 us
+// per chunk (the WY figure as measured beside a running recurrence; erring slow keeps
+// the recurrence from waiting).  Candidates: segment sizes growing or shrinking
+// geometrically (s_k = s_0 rho^k: rho > 1 lets the recurrence start early when it
+// bounds the call, rho < 1 runs most WY records on every SM first when they bound
+// it), 2..kMaxSegments segments of at least one chunk, and the plain schedule.
+// (Running the load stage per segment on the WY stream as well was measured no
+// faster at one row and slower at two.)
 namespace seg_model {
 constexpr double kWaveUs = 11.2, kWyFixedUs = 4.0, kChainFixedUs = 9.5, kChainChunkUs = 2.3;
 }
 
-double simulate_segments(const int* cs, int S, int tasks_per_chunk, int nsm, int chain_ctas) {
+struct SegPlan {
+    int S = 1;  // segments (1: the plain schedule on the caller's stream)
+    int cs[kMaxSegments + 1] = {};
+};
+
+// Time from the end of the load stage to the end of the last recurrence launch.
+double simulate_plan(const SegPlan& pl, int tasks_per_chunk, int nsm, int chain_ctas) {
     using namespace seg_model;
-    auto wy_us = [&](int chunks, int P) {
+    const int P = pl.S > 1 ? nsm - chain_ctas : nsm;  // SMs of the WY stream beside a running recurrence
+    auto wy_us = [&](int chunks, int sms) {
         const int64_t tasks = (int64_t)chunks * tasks_per_chunk;
-        return kWaveUs * (double)((tasks + P - 1) / P) + kWyFixedUs;
+        return kWaveUs * (double)((tasks + sms - 1) / sms) + kWyFixedUs;
     };
-    double wy_end = wy_us(cs[1] - cs[0], nsm), chain_end = 0.0;
-    for (int k = 0; k < S; ++k) {
+    double wy_end = wy_us(pl.cs[1], nsm), chain_end = 0.0;
+    for (int k = 0; k < pl.S; ++k) {
         const double start = chain_end > wy_end ? chain_end : wy_end;
-        chain_end = start + kChainFixedUs + kChainChunkUs * (cs[k + 1] - cs[k]);
-        if (k + 1 < S) wy_end += wy_us(cs[k + 2] - cs[k + 1], nsm - chain_ctas);
+        chain_end = start + kChainFixedUs + kChainChunkUs * (pl.cs[k + 1] - pl.cs[k]);
+        if (k + 1 < pl.S) wy_end += wy_us(pl.cs[k + 2] - pl.cs[k + 1], P);
     }
     return chain_end;
 }
 
-int plan_segments(int per, int N, int Kh, int Vh, int nsm, int* cs) {
+// The plan for N dense rows of T tokens: overlap needs a recurrence that leaves at least
+// 32 SMs to the WY records and rows of at least 16 chunks.
+SegPlan dense_plan(int Kh, int Vh, int N, int T, int nsm) {
+    const int per = (T + 63) / 64;
+    SegPlan best;
+    best.cs[1] = per;
+    if (N * Vh + 32 > nsm || per < 16) return best;
     const int tasks_per_chunk = N * Kh * ((Vh / Kh + wy::kHeads - 1) / wy::kHeads);
     const int chain_ctas = N * Vh;
-    // no overlap: every WY record on every SM, then one recurrence launch
-    int best_S = 1;
-    double best = 0.0;
-    {
-        const int one[2] = {0, per};
-        best = simulate_segments(one, 1, tasks_per_chunk, nsm, nsm);
-    }
-    int best_cs[kMaxSegments + 1] = {0, per};
+    double best_t = simulate_plan(best, tasks_per_chunk, nsm, chain_ctas);
     static const double kRho[] = {0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8, 0.9, 1.0, 1.1, 1.2, 1.35, 1.5, 1.75, 2.0};
     const int max_S = per < kMaxSegments ? per : kMaxSegments;
     for (int S = 2; S <= max_S; ++S) {
         for (double rho : kRho) {
-            int c[kMaxSegments + 1];
+            SegPlan c;
+            c.S = S;
             double total = 0.0, f = 1.0;
             for (int k = 0; k < S; ++k, f *= rho) total += f;
             double acc = 0.0;
             f = 1.0;
-            c[0] = 0;
             for (int k = 1; k <= S; ++k, f *= rho) {
                 acc += f / total * per;
                 const int v = (int)(acc + 0.5);
-                const int lo = c[k - 1] + 1, hi = per - (S - k);  // every segment keeps at least one chunk
-                c[k] = v < lo ? lo : (v > hi ? hi : v);
+                const int lo = c.cs[k - 1] + 1, hi = per - (S - k);  // every segment keeps at least one chunk
+                c.cs[k] = v < lo ? lo : (v > hi ? hi : v);
             }
-            c[S] = per;
-            const double t = simulate_segments(c, S, tasks_per_chunk, nsm, chain_ctas);
-            if (t < best) {
-                best = t;
-                best_S = S;
-                for (int k = 0; k <= S; ++k) best_cs[k] = c[k];
+            c.cs[S] = per;
+            const double t = simulate_plan(c, tasks_per_chunk, nsm, chain_ctas);
+            if (t < best_t) {
+                best_t = t;
+                best = c;
             }
         }
     }
-    for (int k = 0; k <= best_S; ++k) cs[k] = best_cs[k];
-    return best_S;
+    return best;
 }
 
-// Segments of an overlapped dense prefill of N rows of T tokens (1: the plain schedule):
-// the overlap needs a recurrence that leaves at least 32 SMs to the WY records and rows
-// of at least 16 chunks.
-int dense_segments(int Kh, int Vh, int N, int T, int nsm, int* cs) {
-    const int per = (T + 63) / 64;
-    if (N * Vh + 32 > nsm || per < 16) return 1;
-    return plan_segments(per, N, Kh, Vh, nsm, cs);
-}
+// Kernels one dense call launches under a plan (history writer included; a fused load
+// stage is one GEMM and its history copy is not a kernel).
+int plan_launches(const SegPlan& pl, bool fused) { return (fused ? 1 : 2) + 2 * pl.S; }
 
 // Everything one prefill call launches, with the workspace carved and the
 // tensor maps built once.
@@ -489,9 +490,11 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     // segment s runs on the high-priority one, each segment's recurrence starting from
     // the state the previous one left in final_state.
     const int chain_ctas = N * Vh;
-    int S = 1;
-    int cs[kMaxSegments + 1];
-    if (may_overlap && cu_dev == nullptr && final_state != nullptr) S = dense_segments(Kh, Vh, N, uniform_T, nsm, cs);
+    SegPlan plan;
+    if (may_overlap && cu_dev == nullptr && final_state != nullptr)
+        plan = dense_plan(Kh, Vh, N, uniform_T, nsm);
+    const int S = plan.S;
+    const int* cs = plan.cs;
     if (S > 1) {
         std::lock_guard<std::mutex> lock(g_side_mu);
         SideStreams* ss = nullptr;
@@ -807,18 +810,25 @@ int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, in
                         final_state, final_conv, workspace, total > 0 ? L.off_z : 0, s, true);
 }
 
-int gdn_prefill_segments(const gdn_dims* dims, int32_t B, int32_t T) {
+int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t* segments,
+                         int32_t* launches) {
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
-    if (B < 0 || T < 0 || B > 65535 || (int64_t)B * T > INT32_MAX) return GDN_ERR_INVALID_ARG;
-    if (B == 0 || T == 0) return 0;
+    if (B < 0 || T < 0 || B > 65535 || (int64_t)B * T > INT32_MAX || !segments || !launches)
+        return GDN_ERR_INVALID_ARG;
+    *segments = 0;
+    *launches = 0;
+    if (B == 0 || T == 0) return GDN_OK;
     if ((st = check_device()) != GDN_OK) return st;
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
-    int cs[kMaxSegments + 1];
-    return dense_segments(dims->num_k_heads, dims->num_v_heads, B, T, nsm, cs);
+    const bool fused = from_hidden != 0 && fused_load_ok(dims, T);
+    const SegPlan pl = dense_plan(dims->num_k_heads, dims->num_v_heads, B, T, nsm);
+    *segments = pl.S;
+    *launches = plan_launches(pl, fused) + (from_hidden != 0 && !fused ? 1 : 0);  // + the unfused in_proj
+    return GDN_OK;
 }
 
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {

@@ -97,17 +97,20 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Schedule of a dense gdn_prefill (B rows x T tokens) that returns its final
- * state, on the current device: the number S of recurrence segments.  S = 1
- * is the plain schedule on the caller's stream; S > 1 overlaps the WY records
- * of segment s+1 with the recurrence of segment s on internal streams (the
- * segment sizes come from a cost model of the kernels; see gdn_prefill).
- * Such a call launches 2 + 2*S kernels (load stage, history writer, S WY
- * launches, S recurrence launches); gdn_prefill_hidden launches 1 + 2*S.
- * Returns 0 for an empty call, a negative status for invalid arguments or an
- * unsupported device.  Host-only: enqueues nothing.
+ * Schedule of a dense prefill of B rows x T tokens that returns its final
+ * state, on the current device: gdn_prefill (from_hidden = 0) or
+ * gdn_prefill_hidden (from_hidden = 1).  *segments = S, the number of
+ * recurrence segments: S = 1 is the plain schedule on the caller's stream;
+ * S > 1 overlaps the WY records of segment s+1 with the recurrence of segment
+ * s on internal streams, with segment sizes chosen by a cost model of the
+ * kernels.  *launches = the number of kernels one such call launches (2 + 2*S
+ * for gdn_prefill, 1 + 2*S for the fused gdn_prefill_hidden, one more when
+ * that call takes the unfused in_proj).  Both 0 for an empty call.  Returns a
+ * status (negative for invalid arguments or an unsupported device).
+ * Host-only: enqueues nothing.
  */
-int gdn_prefill_segments(const gdn_dims* dims, int32_t B, int32_t T);
+int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t* segments,
+                         int32_t* launches);
 
 /* Bytes of device workspace gdn_prefill_varlen needs for N rows with
  * total_T tokens in all.  Returns 0 for invalid dims. */

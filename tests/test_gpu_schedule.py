@@ -1,6 +1,6 @@
-"""The dense prefill's schedule as the library reports it (gdn_prefill_segments):
+"""The dense prefill's schedule as the library reports it (gdn_prefill_schedule):
 overlap only where the recurrence leaves SMs free and the rows are long enough,
-and segment counts within the library's bound."""
+segment counts within the library's bound, launch counts consistent with them."""
 import pytest
 import torch
 
@@ -16,16 +16,20 @@ def _gpu():
     gdn.load_library()
 
 
-def test_segments():
+def test_schedule():
     nsm = torch.cuda.get_device_properties(0).multi_processor_count
-    assert gdn.prefill_segments(0, 100) == 0
-    assert gdn.prefill_segments(1, 0) == 0
-    assert gdn.prefill_segments(1, 15 * 64) == 1          # under 16 chunks: plain schedule
-    s1 = gdn.prefill_segments(1, 8192)
-    assert 2 <= s1 <= 8                                  # one row: the recurrence leaves SMs free
-    s2 = gdn.prefill_segments(2, 65536)
-    assert 2 <= s2 <= 8
-    rows = (nsm - 32) // 48 + 1                          # the recurrence would take too many SMs
-    assert gdn.prefill_segments(rows, 8192) == 1
+    assert gdn.prefill_schedule(0, 100) == (0, 0)
+    assert gdn.prefill_schedule(1, 0) == (0, 0)
+    assert gdn.prefill_schedule(1, 15 * 64) == (1, 4)          # under 16 chunks: plain schedule
+    assert gdn.prefill_schedule(1, 15 * 64, True) == (1, 3)    # fused load stage, history copied
+    assert gdn.prefill_schedule(1, 2, True) == (1, 5)          # too short to fuse: in_proj + 4
+    s1, l1 = gdn.prefill_schedule(1, 8192)
+    assert 2 <= s1 <= 8 and l1 == 2 + 2 * s1
+    s2, l2 = gdn.prefill_schedule(1, 8192, True)
+    assert 2 <= s2 <= 8 and l2 == 1 + 2 * s2
+    s3, l3 = gdn.prefill_schedule(2, 65536)
+    assert 2 <= s3 <= 8 and l3 == 2 + 2 * s3
+    rows = (nsm - 32) // 48 + 1                                # the recurrence would take too many SMs
+    assert gdn.prefill_schedule(rows, 8192) == (1, 4)
     with pytest.raises(gdn.GdnError):
-        gdn.prefill_segments(-1, 8)
+        gdn.prefill_schedule(-1, 8)
