@@ -87,6 +87,38 @@ def test_invalid_arguments_rejected(lib):
                            16, 1 << 30, None) == -1
 
 
+def test_projection_and_hidden_arguments_checked_on_host(lib):
+    d = _dims()
+    w = gdn._WeightsC(16, 16, 16, 16)
+    # contraction width not a multiple of 64: unsupported, before any CUDA call
+    assert lib.gdn_in_proj(ctypes.byref(d), 8, 100, 16, 16, 16, 16, 16, 16, None) == -2
+    assert lib.gdn_out_proj(ctypes.byref(d), -8, 128, 16, 16, 16, None) == -1
+    assert lib.gdn_prefill_hidden(ctypes.byref(d), ctypes.byref(w), 1, 8, 100, 16, 16, None, None, 16, None,
+                                  None, 16, 1 << 30, None) == -2
+    # negative sizes, null hidden states, null weights
+    assert lib.gdn_prefill_hidden(ctypes.byref(d), ctypes.byref(w), -1, 8, 128, 16, 16, None, None, 16, None,
+                                  None, 16, 1 << 30, None) == -1
+    assert lib.gdn_prefill_hidden(ctypes.byref(d), ctypes.byref(w), 1, 8, 128, None, 16, None, None, 16, None,
+                                  None, 16, 1 << 30, None) == -1
+    assert lib.gdn_prefill_hidden(ctypes.byref(d), None, 1, 8, 128, 16, 16, None, None, 16, None,
+                                  None, 16, 1 << 30, None) == -1
+    # misaligned hidden states
+    assert lib.gdn_prefill_hidden(ctypes.byref(d), ctypes.byref(w), 1, 8, 128, 8, 16, None, None, 16, None,
+                                  None, 16, 1 << 30, None) == -1
+    # the hidden-state prefill's workspace holds the prefill's, z and the staged histories
+    ws = lib.gdn_prefill_hidden_workspace_size(ctypes.byref(d), 2, 1000)
+    assert ws >= lib.gdn_prefill_workspace_size(ctypes.byref(d), 2, 1000) + 2000 * 6144 * 2 + 2 * 3 * 10240 * 4
+    # rows shorter than the conv window take the unfused launches: room for qkv, z, a, b as well
+    assert lib.gdn_prefill_hidden_workspace_size(ctypes.byref(d), 4, 2) >= \
+        lib.gdn_prefill_workspace_size(ctypes.byref(d), 4, 2) + 8 * (10240 + 6144 + 96) * 2
+    # the schedule query: null outputs, negative sizes
+    seg, lau = ctypes.c_int32(-7), ctypes.c_int32(-7)
+    assert lib.gdn_prefill_schedule(ctypes.byref(d), 1, 8192, 0, None, None) == -1
+    assert lib.gdn_prefill_schedule(ctypes.byref(d), -1, 8192, 0, ctypes.byref(seg), ctypes.byref(lau)) == -1
+    assert lib.gdn_prefill_schedule(ctypes.byref(d), 0, 8192, 0, ctypes.byref(seg), ctypes.byref(lau)) == 0
+    assert (seg.value, lau.value) == (0, 0)
+
+
 def test_slot_tables_checked_on_host(lib):
     # a slot twice, a slot past the pool, a negative slot, an empty pool: refused before any launch
     d = _dims()
