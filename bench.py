@@ -384,6 +384,7 @@ def bench_decode_multi(args, local, k=4):
     achieved = ROWS * STATE_BYTES_PER_ROW_TOKEN / (t / launches) / 1e9  # state bytes per launch / launch time
     return {"workload": f"decode 64 rows x 128 tokens, {k} tokens per row per call", "tokens_per_call": k,
             "value": ROWS * DECODE_STEPS * args.steps / t, "unit": "row-tokens/s",
+            "us_per_launch": t / launches * 1e6,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
                          "algorithmic_bytes_per_launch": ROWS * STATE_BYTES_PER_ROW_TOKEN},
