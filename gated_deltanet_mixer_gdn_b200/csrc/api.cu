@@ -147,7 +147,21 @@ int side_streams(int dev, SideStreams** out) {
     return GDN_OK;
 }
 
-int gemm_setup(const void* kernel_fn);  // defined with the GEMM launches below
+// Dynamic shared memory opt-in of a kernel (the attribute belongs to the device's context):
+// once per kernel and device, under a lock.
+int smem_optin(const void* kernel_fn, uint32_t bytes) {
+    static std::mutex mu;
+    static std::vector<std::pair<const void*, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto& d : done)
+        if (d.first == kernel_fn && d.second == dev) return GDN_OK;
+    if (cudaFuncSetAttribute(kernel_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    done.emplace_back(kernel_fn, dev);
+    return GDN_OK;
+}
 
 // The load stage fused into the in_proj GEMM: the hidden states and the
 // stacked in_proj weights go in; the staged operands, z and the rows' last
@@ -320,7 +334,7 @@ struct PrefillPlan {
             !make_map(&mW, fused->w_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)gp.K, (uint64_t)gp.N, gemm::BK,
                       gemm::BN, CU_TENSOR_MAP_SWIZZLE_128B))
             return GDN_ERR_CUDA;
-        int rc = gemm_setup(reinterpret_cast<const void*>(gdn_gemm_kernel<1>));
+        int rc = smem_optin(reinterpret_cast<const void*>(gdn_gemm_kernel<1>), gemm::SMEM_BYTES);
         if (rc != GDN_OK) return rc;
         const int64_t ntiles = (int64_t)((gp.M + gemm::BM - 4) / (gemm::BM - 3)) * ((gp.N + gemm::BN - 1) / gemm::BN);
         const int grid = (int)(ntiles < nsm ? ntiles : nsm);
@@ -359,12 +373,8 @@ struct PrefillPlan {
         wp.Gs = Gs;
         wp.Bs = Bs;
         wp.rec = rec;
-        static std::once_flag once;
-        static cudaError_t err = cudaSuccess;
-        std::call_once(once, [] {
-            err = cudaFuncSetAttribute(gdn_wy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wy::SMEM_BYTES);
-        });
-        if (err != cudaSuccess) return GDN_ERR_CUDA;
+        int rc = smem_optin(reinterpret_cast<const void*>(gdn_wy_kernel), wy::SMEM_BYTES);
+        if (rc != GDN_OK) return rc;
         const int ratio = Vh / Kh;
         const int64_t ntasks = nch * Kh * ((ratio + wy::kHeads - 1) / wy::kHeads);
         const int grid = (int)(ntasks < grid_cap ? ntasks : grid_cap);
@@ -388,13 +398,8 @@ struct PrefillPlan {
         cp.c0 = c0;
         cp.c1 = c1;
         cp.slots = slots;
-        static std::once_flag once;
-        static cudaError_t err = cudaSuccess;
-        std::call_once(once, [] {
-            err = cudaFuncSetAttribute(gdn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)chunk::SMEM_BYTES);
-        });
-        if (err != cudaSuccess) return GDN_ERR_CUDA;
+        int rc = smem_optin(reinterpret_cast<const void*>(gdn_chunk_kernel), chunk::SMEM_BYTES);
+        if (rc != GDN_OK) return rc;
         dim3 grid(Vh, N);
         gdn_chunk_kernel<<<grid, chunk::kThreads, chunk::SMEM_BYTES, st>>>(mV, mQ, mK, mZ, mO, cp);
         return cuda_status(cudaGetLastError());
@@ -612,16 +617,10 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
     p.out = out;
     p.slots = slots;
     p.ntok = ntok;
-    static std::once_flag dec_once;
-    static cudaError_t dec_err = cudaSuccess;
-    std::call_once(dec_once, [] {
-        dec_err = cudaFuncSetAttribute(gdn_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)dec::kSmemLimit);
-        if (dec_err == cudaSuccess)
-            dec_err = cudaFuncSetAttribute(gdn_decode_kernel<dec::kMaxTokens>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dec::kSmemLimit);
-    });
-    if (dec_err != cudaSuccess) return GDN_ERR_CUDA;
+    if ((st = smem_optin(reinterpret_cast<const void*>(gdn_decode_kernel<1>), dec::kSmemLimit)) != GDN_OK ||
+        (st = smem_optin(reinterpret_cast<const void*>(gdn_decode_kernel<dec::kMaxTokens>), dec::kSmemLimit)) !=
+            GDN_OK)
+        return st;
     const dec::Plan dplan = dec::plan(p.Vh / p.Kh, ntok);
     if (dplan.stages < 2) return GDN_ERR_UNSUPPORTED;  // the group's inputs of ntok tokens leave no room
     int dev = 0, nsm = 0;
@@ -643,22 +642,6 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
 }
 
 
-// Dynamic shared memory opt-in of a GEMM kernel instance, once per instance and device.
-int gemm_setup(const void* kernel_fn) {
-    static std::mutex mu;
-    static std::vector<std::pair<const void*, int>> done;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(mu);
-    for (auto& d : done)
-        if (d.first == kernel_fn && d.second == dev) return GDN_OK;
-    if (cudaFuncSetAttribute(kernel_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::SMEM_BYTES) !=
-        cudaSuccess)
-        return GDN_ERR_CUDA;
-    done.emplace_back(kernel_fn, dev);
-    return GDN_OK;
-}
-
 // C = A W^T over bf16 A [M][K] and W [N][K], columns routed to the segments of gp.
 int gemm_launch(const uint16_t* A, const uint16_t* W, GemmParams gp, cudaStream_t stream) {
     if (gp.M == 0 || gp.N == 0) return GDN_OK;
@@ -674,7 +657,7 @@ int gemm_launch(const uint16_t* A, const uint16_t* W, GemmParams gp, cudaStream_
         !make_map(&mW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)gp.K, (uint64_t)gp.N, gemm::BK, gemm::BN,
                   CU_TENSOR_MAP_SWIZZLE_128B))
         return GDN_ERR_CUDA;
-    st = gemm_setup(reinterpret_cast<const void*>(gdn_gemm_kernel<0>));
+    st = smem_optin(reinterpret_cast<const void*>(gdn_gemm_kernel<0>), gemm::SMEM_BYTES);
     if (st != GDN_OK) return st;
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
