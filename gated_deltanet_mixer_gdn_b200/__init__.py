@@ -28,6 +28,7 @@ LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_schedule", "gdn_prefill_varlen_workspace_size",
            "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
            "gdn_in_proj", "gdn_out_proj", "gdn_prefill_hidden_workspace_size", "gdn_prefill_hidden",
+           "gdn_prefill_hidden_varlen_workspace_size", "gdn_prefill_hidden_varlen",
            "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string",
            "gdn_version")
 
@@ -81,6 +82,11 @@ def load_library() -> ctypes.CDLL:
         L.gdn_prefill_hidden_workspace_size.argtypes = [dp, i32, i32]
         L.gdn_prefill_hidden.restype = ctypes.c_int
         L.gdn_prefill_hidden.argtypes = [dp, wp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.gdn_prefill_hidden_varlen_workspace_size.restype = sz
+        L.gdn_prefill_hidden_varlen_workspace_size.argtypes = [dp, i32, i32]
+        L.gdn_prefill_hidden_varlen.restype = ctypes.c_int
+        L.gdn_prefill_hidden_varlen.argtypes = [dp, wp, i32, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                sz, vp]
         L.gdn_out_proj.restype = ctypes.c_int
         L.gdn_out_proj.argtypes = [dp, i32, i32, vp, vp, vp, vp]
         L.gdn_decode_multi.restype = ctypes.c_int
@@ -333,6 +339,49 @@ def prefill_hidden(x, w_in, weights, init_state=None, init_conv=None, *, out=Non
     return out, final_state, final_conv
 
 
+def prefill_hidden_varlen(cu_seqlens, x, w_in, weights, init_state=None, init_conv=None, *, out=None,
+                          final_state=None, final_conv=None, dims: Dims = MODEL, cu_seqlens_dev=None,
+                          in_place: bool = False):
+    """Packed prefill from hidden states: x bf16 [total, hidden] holds the rows given by cu_seqlens
+    (int32 [N+1]); the load stage runs inside the in_proj GEMM.  Returns (out bf16 [total, Vh*D],
+    final_state f32 [N,Vh,D,D], final_conv f32 [N,W-1,C]); the same bits as in_proj followed by
+    prefill_varlen."""
+    dev = _device_of(x)
+    L = load_library()
+    _need(x, torch.bfloat16, "x", dev)
+    _need(w_in, torch.bfloat16, "w_in", dev)
+    cu_host = torch.as_tensor(cu_seqlens, dtype=torch.int32).cpu().contiguous()
+    N = int(cu_host.numel()) - 1
+    total, hidden = int(x.shape[0]), int(x.shape[1])
+    if N < 0 or int(cu_host[-1]) != total:
+        raise ValueError("prefill_hidden_varlen: cu_seqlens must end at the token count")
+    C, VD, Vh, D, Wm = dims.conv_channels, dims.value_width, dims.num_v_heads, dims.head_dim, dims.conv_width - 1
+    if tuple(w_in.shape) != (C + VD + 2 * Vh, hidden):
+        raise ValueError("prefill_hidden_varlen: w_in shape")
+    cu_dev = cu_seqlens_dev if cu_seqlens_dev is not None else cu_host.to(dev)
+    if init_state is not None:
+        _need(init_state, torch.float32, "init_state", dev)
+    if init_conv is not None:
+        _need(init_conv, torch.float32, "init_conv", dev)
+    if out is None:
+        out = torch.empty((total, VD), dtype=torch.bfloat16, device=dev)
+    if final_state is None:
+        final_state = init_state if (in_place and init_state is not None) else \
+            torch.empty((N, Vh, D, D), dtype=torch.float32, device=dev)
+    if final_conv is None:
+        final_conv = init_conv if (in_place and init_conv is not None) else \
+            torch.empty((N, Wm, C), dtype=torch.float32, device=dev)
+    dc = _dims_c(dims)
+    ws_bytes = L.gdn_prefill_hidden_varlen_workspace_size(ctypes.byref(dc), N, total)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    st = L.gdn_prefill_hidden_varlen(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), N,
+                                     ctypes.c_void_p(cu_host.data_ptr()), _ptr(cu_dev), total, hidden, _ptr(x),
+                                     _ptr(w_in), _ptr(init_state), _ptr(init_conv), _ptr(out), _ptr(final_state),
+                                     _ptr(final_conv), _ptr(ws), ws_bytes, _stream(dev))
+    _check(st, "gdn_prefill_hidden_varlen")
+    return out, final_state, final_conv
+
+
 def out_proj(y, w_out, *, dims: Dims = MODEL, out=None):
     """y bf16 [T, Vh*D] times w_out bf16 [hidden, Vh*D]^T.  Returns out [T, hidden]."""
     dev = _device_of(y)
@@ -421,5 +470,5 @@ def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tens
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_schedule", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
+__all__ = ["prefill", "prefill_schedule", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_hidden_varlen", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

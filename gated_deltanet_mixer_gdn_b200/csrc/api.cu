@@ -251,9 +251,9 @@ SegPlan dense_plan(int Kh, int Vh, int N, int T, int nsm) {
     return best;
 }
 
-// Kernels one dense call launches under a plan (history writer included; a fused load
-// stage is one GEMM and its history copy is not a kernel).
-int plan_launches(const SegPlan& pl, bool fused) { return (fused ? 1 : 2) + 2 * pl.S; }
+// Kernels one dense call launches under a plan: the load stage (or the fused in_proj GEMM),
+// the history writer, then WY records and recurrence per segment.
+int plan_launches(const SegPlan& pl) { return 2 + 2 * pl.S; }
 
 // Everything one prefill call launches, with the workspace carved and the
 // tensor maps built once.
@@ -315,6 +315,8 @@ struct PrefillPlan {
         f.Kh = Kh;
         f.Vh = Vh;
         f.T = uniform_T;
+        f.cu = seq.cu;
+        f.N = N;
         f.conv_w = w->conv_w;
         f.A_log = w->A_log;
         f.dt_bias = w->dt_bias;
@@ -343,9 +345,11 @@ struct PrefillPlan {
     }
     int conv_out(cudaStream_t st) const {
         if (final_conv == nullptr) return GDN_OK;
-        if (fused != nullptr)  // the rows' last three tokens, staged by the fused load stage
-            return cuda_status(cudaMemcpyAsync(final_conv, fused->conv_last, (size_t)N * 3 * C * 4,
-                                               cudaMemcpyDeviceToDevice, st));
+        if (fused != nullptr) {  // the rows' last tokens, staged by the fused load stage, and the history
+            dim3 grid((C + 255) / 256, N);
+            gdn_conv_merge_kernel<<<grid, 256, 0, st>>>(seq, C, fused->conv_last, init_conv, final_conv);
+            return cuda_status(cudaGetLastError());
+        }
         ConvOutParams cp{};
         cp.C = C;
         cp.N = N;
@@ -676,24 +680,23 @@ struct HiddenLayout {
     size_t off_z, off_conv, off_qkv, off_b, off_a, bytes;
 };
 
-// The fused load stage needs whole 256-column tiles of qkv and z, b and a in one
-// tile, and rows of at least 3 tokens (the history after a row is then its own tokens).
-bool fused_load_ok(const gdn_dims* d, int32_t T) {
+// The fused load stage needs whole 256-column tiles of qkv and of z, and b and a in one tile.
+bool fused_load_ok(const gdn_dims* d) {
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
-    return T >= 3 && (2 * Kh + Vh) % 2 == 0 && Vh % 2 == 0 && 2 * Vh <= gemm::BN;
+    return (2 * Kh + Vh) % 2 == 0 && Vh % 2 == 0 && 2 * Vh <= gemm::BN;
 }
 
-HiddenLayout hidden_layout(const gdn_dims* d, int32_t B, int32_t T) {
+// rows: N packed rows (or B dense rows) of `total` tokens in all; nchunks: the prefill's chunk plan
+HiddenLayout hidden_layout(const gdn_dims* d, int32_t rows, int64_t total, int64_t nchunks) {
     HiddenLayout L{};
-    const int64_t total = (int64_t)B * T;
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
     const size_t C = (size_t)(2 * Kh + Vh) * 128;
-    L.fused = fused_load_ok(d, T);
-    L.off_z = plan_workspace(d, total, B, (int64_t)B * ((T + 63) / 64)).bytes;
+    L.fused = fused_load_ok(d);
+    L.off_z = plan_workspace(d, total, rows, nchunks).bytes;
     size_t o = L.off_z + align_up((size_t)total * Vh * 128 * 2);
     if (L.fused) {
         L.off_conv = o;
-        o += align_up((size_t)B * 3 * C * 4);
+        o += align_up((size_t)rows * 3 * C * 4);
     } else {
         L.off_qkv = o;
         o += align_up((size_t)total * C * 2);
@@ -704,6 +707,43 @@ HiddenLayout hidden_layout(const gdn_dims* d, int32_t B, int32_t T) {
     }
     L.bytes = o;
     return L;
+}
+
+// The prefill from hidden states over dense rows (cu_dev == nullptr, uniform_T) or packed rows:
+// the fused in_proj + load stage where the head counts allow, else in_proj then the prefill.
+int prefill_hidden_impl(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_dev,
+                        int32_t uniform_T, int32_t total, int64_t nch, int64_t nch_planned, int32_t hidden,
+                        const uint16_t* x, const uint16_t* w_in, const float* init_state, const float* init_conv,
+                        uint16_t* out, float* final_state, float* final_conv, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    int st = GDN_OK;
+    if (hidden % gemm::BK != 0) return GDN_ERR_UNSUPPORTED;
+    if (total > 0 && (!x || !w_in || !out || !aligned16(x) || !aligned16(w_in) || !aligned16(out)))
+        return GDN_ERR_INVALID_ARG;
+    const void* fs[4] = {init_state, init_conv, final_state, final_conv};
+    for (const void* p : fs)
+        if (p != nullptr && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    if ((st = check_device()) != GDN_OK) return st;
+    const HiddenLayout L = hidden_layout(dims, N, total, nch_planned);
+    if (total > 0 && (workspace == nullptr || workspace_bytes < L.bytes)) return GDN_ERR_WORKSPACE;
+    if (workspace != nullptr && !aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool dense = cu_dev == nullptr;
+    uint16_t* z = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_z) : nullptr;
+    if (total > 0 && L.fused) {
+        FusedLoad fl{x, w_in, hidden, z, reinterpret_cast<float*>(wsb + L.off_conv)};
+        return prefill_impl(dims, w, N, cu_dev, uniform_T, total, nch, nch_planned, nullptr, z, nullptr, nullptr,
+                            init_state, init_conv, out, final_state, final_conv, workspace, L.off_z, s, dense,
+                            nullptr, &fl);
+    }
+    // head counts the fused tiles do not cover: in_proj into the workspace, then the prefill over it
+    uint16_t* qkv = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_qkv) : nullptr;
+    uint16_t* bb = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_b) : nullptr;
+    uint16_t* aa = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_a) : nullptr;
+    if (total > 0 && (st = gdn_in_proj(dims, total, hidden, x, w_in, qkv, z, bb, aa, stream)) != GDN_OK) return st;
+    return prefill_impl(dims, w, N, cu_dev, uniform_T, total, nch, nch_planned, qkv, z, aa, bb, init_state,
+                        init_conv, out, final_state, final_conv, workspace, total > 0 ? L.off_z : 0, s, dense);
 }
 
 }  // namespace
@@ -748,8 +788,9 @@ int gdn_out_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t
 
 size_t gdn_prefill_hidden_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
     if (check_dims(dims) != GDN_OK || B < 0 || T < 0) return 0;
-    if ((int64_t)B * T > INT32_MAX) return 0;
-    return hidden_layout(dims, B, T).bytes;
+    const int64_t total = (int64_t)B * T;
+    if (total > INT32_MAX) return 0;
+    return hidden_layout(dims, B, total, (int64_t)B * ((T + 63) / 64)).bytes;
 }
 
 int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, int32_t hidden,
@@ -760,37 +801,37 @@ int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, in
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
     if (B < 0 || T < 0 || B > 65535 || hidden <= 0) return GDN_ERR_INVALID_ARG;
-    if (hidden % gemm::BK != 0) return GDN_ERR_UNSUPPORTED;
     const int64_t total = (int64_t)B * T;
     if (total > INT32_MAX) return GDN_ERR_INVALID_ARG;
-    if (total > 0 && (!x || !w_in || !out || !aligned16(x) || !aligned16(w_in) || !aligned16(out)))
-        return GDN_ERR_INVALID_ARG;
-    const void* fs[4] = {init_state, init_conv, final_state, final_conv};
-    for (const void* p : fs)
-        if (p != nullptr && !aligned16(p)) return GDN_ERR_INVALID_ARG;
-    if ((st = check_device()) != GDN_OK) return st;
-    const HiddenLayout L = hidden_layout(dims, B, T);
-    if (total > 0 && (workspace == nullptr || workspace_bytes < L.bytes)) return GDN_ERR_WORKSPACE;
-    if (workspace != nullptr && !aligned16(workspace)) return GDN_ERR_INVALID_ARG;
-    uint8_t* wsb = static_cast<uint8_t*>(workspace);
     const int64_t nch = (int64_t)B * ((T + 63) / 64);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint16_t* z = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_z) : nullptr;
-    if (total > 0 && L.fused) {
-        FusedLoad fl{x, w_in, hidden, z, reinterpret_cast<float*>(wsb + L.off_conv)};
-        return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, nullptr, z, nullptr, nullptr,
-                            init_state, init_conv, out, final_state, final_conv, workspace, L.off_z, s, true, nullptr,
-                            &fl);
-    }
-    // rows shorter than the conv window (or head counts the fused tiles do not cover):
-    // in_proj into the workspace, then the prefill over it
-    uint16_t* qkv = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_qkv) : nullptr;
-    uint16_t* bb = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_b) : nullptr;
-    uint16_t* aa = total > 0 ? reinterpret_cast<uint16_t*>(wsb + L.off_a) : nullptr;
-    if (total > 0 && (st = gdn_in_proj(dims, (int32_t)total, hidden, x, w_in, qkv, z, bb, aa, stream)) != GDN_OK)
-        return st;
-    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, aa, bb, init_state, init_conv, out,
-                        final_state, final_conv, workspace, total > 0 ? L.off_z : 0, s, true);
+    return prefill_hidden_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, hidden, x, w_in, init_state,
+                               init_conv, out, final_state, final_conv, workspace, workspace_bytes, stream);
+}
+
+size_t gdn_prefill_hidden_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T) {
+    if (check_dims(dims) != GDN_OK || N < 0 || total_T < 0) return 0;
+    return hidden_layout(dims, N, total_T, chunk_bound(N, total_T)).bytes;
+}
+
+int gdn_prefill_hidden_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_host,
+                              const int32_t* cu_dev, int32_t total_T, int32_t hidden, const uint16_t* x,
+                              const uint16_t* w_in, const float* init_state, const float* init_conv, uint16_t* out,
+                              float* final_state, float* final_conv, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (N < 0 || N > 65535 || total_T < 0 || hidden <= 0) return GDN_ERR_INVALID_ARG;
+    if (cu_host == nullptr || (N > 0 && cu_dev == nullptr)) return GDN_ERR_INVALID_ARG;
+    if (cu_host[0] != 0 || cu_host[N] != total_T) return GDN_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < N; ++i)
+        if (cu_host[i + 1] < cu_host[i]) return GDN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_dev) & 3u) != 0) return GDN_ERR_INVALID_ARG;
+    int64_t nch = 0;
+    for (int32_t i = 0; i < N; ++i) nch += (cu_host[i + 1] - cu_host[i] + 63) / 64;
+    return prefill_hidden_impl(dims, w, N, cu_dev, 0, total_T, nch, chunk_bound(N, total_T), hidden, x, w_in,
+                               init_state, init_conv, out, final_state, final_conv, workspace, workspace_bytes,
+                               stream);
 }
 
 int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t* segments,
@@ -807,10 +848,10 @@ int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t fro
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
-    const bool fused = from_hidden != 0 && fused_load_ok(dims, T);
+    const bool fused = from_hidden != 0 && fused_load_ok(dims);
     const SegPlan pl = dense_plan(dims->num_k_heads, dims->num_v_heads, B, T, nsm);
     *segments = pl.S;
-    *launches = plan_launches(pl, fused) + (from_hidden != 0 && !fused ? 1 : 0);  // + the unfused in_proj
+    *launches = plan_launches(pl) + (from_hidden != 0 && !fused ? 1 : 0);  // + the unfused in_proj
     return GDN_OK;
 }
 

@@ -34,7 +34,9 @@ struct GemmParams {
 
 // The load stage fused into the in_proj epilogue (see inproj.cuh).
 struct FusedPrep {
-    int Kh, Vh, T;                 // dense rows of T tokens
+    int Kh, Vh, T;                 // dense rows of T tokens (cu == nullptr)
+    const int* cu;                 // packed rows: cu_seqlens [N+1] (device), or nullptr
+    int N;                         // packed rows
     const uint16_t* conv_w;        // bf16 [C][4]
     const float* A_log;            // [Vh]
     const float* dt_bias;          // [Vh]
@@ -43,6 +45,7 @@ struct FusedPrep {
     float *Gs, *Bs;                // [Vh][M]
     uint16_t* z;                   // bf16 [M][Vh*128]
     float* conv_last;              // f32 [rows][3][C]: pre-conv values of each row's last three tokens
+                                   // (token pos of a row of len tokens in slot pos + 3 - len)
 };
 
 namespace gemm {

@@ -33,8 +33,24 @@ __device__ void fused_prep_epilogue(const FusedPrep& f, const GemmParams& p, uin
     const int lrow = 32 * q4 + lane;  // row of the tile
     const int r = r0 + lrow;          // token (rows before 0 or past M are padding)
     const bool out_row = lrow >= 3 && r < p.M;
-    const int n = out_row ? r / f.T : 0;    // packed row of the token
-    const int pos = out_row ? r - n * f.T : 0;  // position inside it
+    int n = 0, pos = 0, len = f.T;           // packed row of the token, position in it, its length
+    if (out_row) {
+        if (f.cu == nullptr) {
+            n = r / f.T;
+            pos = r - n * f.T;
+        } else {  // the last row starting at or before r (empty rows share their start with the next)
+            int lo = 0, hi = f.N;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (__ldg(f.cu + mid) <= r) lo = mid;
+                else hi = mid;
+            }
+            n = lo;
+            const int start = __ldg(f.cu + n);
+            pos = r - start;
+            len = __ldg(f.cu + n + 1) - start;
+        }
+    }
     float* xbuf = reinterpret_cast<float*>(scratch);                          // [128][kXStride]
     float4* taps = reinterpret_cast<float4*>(scratch + gemm::XBUF_BYTES);       // [256] {w0, w1, w2, w3}
 
@@ -51,7 +67,7 @@ __device__ void fused_prep_epilogue(const FusedPrep& f, const GemmParams& p, uin
         const int slot = n0 / kD;  // head slot of the tile's first head: q 0..Kh-1, k Kh..2Kh-1, v after
         const bool is_v = slot >= 2 * f.Kh;
         const bool is_q = slot < f.Kh;
-        const bool at_end = out_row && pos >= f.T - 3;  // one of the row's last three tokens
+        const bool at_end = out_row && pos >= len - 3;  // one of the row's last three tokens
         const int rm[3] = {max(lrow - 1, 0), max(lrow - 2, 0), max(lrow - 3, 0)};  // rows 0-2 only pad
         // conv + silu of channels [32 j, 32 j + 32) of head hh of the tile
         auto conv_chunk = [&](int hh, int j, float* act) {
@@ -70,7 +86,7 @@ __device__ void fused_prep_epilogue(const FusedPrep& f, const GemmParams& p, uin
 #pragma unroll
             for (int q = 0; q < 8; ++q) xr[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             if (at_end) {
-                float4* dst = reinterpret_cast<float4*>(f.conv_last + ((size_t)n * 3 + pos - (f.T - 3)) * C + n0 + cb);
+                float4* dst = reinterpret_cast<float4*>(f.conv_last + ((size_t)n * 3 + pos + 3 - len) * C + n0 + cb);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) dst[q] = xr[q];
             }
@@ -201,6 +217,27 @@ __device__ void fused_prep_epilogue(const FusedPrep& f, const GemmParams& p, uin
                 }
             }
         }
+    }
+}
+
+// Final histories after the fused load stage: row n's history after its len tokens is rows
+// len .. len + 2 of [initial history (3 rows); the row's tokens].  The epilogue staged the
+// row's last min(len, 3) pre-conv tokens (token pos in slot pos + 3 - len); the other rows
+// come from the initial history (zeros without one).  final_conv may alias init_conv: for each
+// channel the thread reads initial row j + len before writing row j, in increasing j.
+__global__ void __launch_bounds__(256) gdn_conv_merge_kernel(SeqIndex seq, int C, const float* staged,
+                                                             const float* init_conv, float* final_conv) {
+    const int n = blockIdx.y;
+    const int ch = blockIdx.x * blockDim.x + threadIdx.x;
+    if (ch >= C) return;
+    int start, len;
+    seq.bounds(n, start, len);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        float v;
+        if (j >= 3 - len) v = staged[((size_t)n * 3 + j) * C + ch];
+        else v = init_conv ? init_conv[((size_t)n * 3 + j + len) * C + ch] : 0.f;
+        final_conv[((size_t)n * 3 + j) * C + ch] = v;
     }
 }
 

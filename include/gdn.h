@@ -103,9 +103,10 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
  * recurrence segments: S = 1 is the plain schedule on the caller's stream;
  * S > 1 overlaps the WY records of segment s+1 with the recurrence of segment
  * s on internal streams, with segment sizes chosen by a cost model of the
- * kernels.  *launches = the number of kernels one such call launches (2 + 2*S
- * for gdn_prefill, 1 + 2*S for the fused gdn_prefill_hidden, one more when
- * that call takes the unfused in_proj).  Both 0 for an empty call.  Returns a
+ * kernels.  *launches = the number of kernels one such call launches (2 + 2*S:
+ * the load stage or the fused in_proj GEMM, the history writer, S WY and S
+ * recurrence launches; one more when gdn_prefill_hidden takes the unfused
+ * in_proj).  Both 0 for an empty call.  Returns a
  * status (negative for invalid arguments or an unsupported device).
  * Host-only: enqueues nothing.
  */
@@ -231,9 +232,9 @@ int gdn_out_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t
  *          (out is the mixer's output, before out_proj; NULL and in-place
  *          rules as there).
  * workspace: gdn_prefill_hidden_workspace_size(dims, B, T) bytes, 16-byte
- * aligned (it also holds z).  Rows shorter than 3 tokens, or head counts
- * whose q/k/v or z widths are not whole 256-column tiles, take the unfused
- * pair of launches inside the same call (the workspace size accounts for it).
+ * aligned (it also holds z and the rows' staged last tokens).  Head counts
+ * whose q/k/v or z widths are not whole 256-column tiles take the unfused pair
+ * of launches inside the same call (the workspace size accounts for it).
  * Returns GDN_ERR_UNSUPPORTED for hidden % 64 != 0; otherwise as gdn_prefill.
  */
 size_t gdn_prefill_hidden_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
@@ -241,6 +242,22 @@ int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, in
                        const uint16_t* x, const uint16_t* w_in, const float* init_state, const float* init_conv,
                        uint16_t* out, float* final_state, float* final_conv, void* workspace,
                        size_t workspace_bytes, void* stream);
+
+/*
+ * gdn_prefill_hidden over packed rows (the hidden-state counterpart of
+ * gdn_prefill_varlen): x bf16 [total_T][hidden] holds N rows, row n the
+ * tokens [cu[n], cu[n+1]); cu_seqlens_host / cu_seqlens_dev, state, history
+ * and output layouts, aliasing and NULL rules as for gdn_prefill_varlen
+ * (zero-length rows and rows shorter than the conv window are legal).  The
+ * same bits as gdn_in_proj followed by gdn_prefill_varlen.  workspace:
+ * gdn_prefill_hidden_varlen_workspace_size(dims, N, total_T) bytes.
+ */
+size_t gdn_prefill_hidden_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T);
+int gdn_prefill_hidden_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N,
+                              const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int32_t total_T,
+                              int32_t hidden, const uint16_t* x, const uint16_t* w_in, const float* init_state,
+                              const float* init_conv, uint16_t* out, float* final_state, float* final_conv,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * gdn_prefill without a caller-supplied workspace, for callers that cannot

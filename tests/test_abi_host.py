@@ -108,9 +108,19 @@ def test_projection_and_hidden_arguments_checked_on_host(lib):
     # the hidden-state prefill's workspace holds the prefill's, z and the staged histories
     ws = lib.gdn_prefill_hidden_workspace_size(ctypes.byref(d), 2, 1000)
     assert ws >= lib.gdn_prefill_workspace_size(ctypes.byref(d), 2, 1000) + 2000 * 6144 * 2 + 2 * 3 * 10240 * 4
-    # rows shorter than the conv window take the unfused launches: room for qkv, z, a, b as well
-    assert lib.gdn_prefill_hidden_workspace_size(ctypes.byref(d), 4, 2) >= \
-        lib.gdn_prefill_workspace_size(ctypes.byref(d), 4, 2) + 8 * (10240 + 6144 + 96) * 2
+    # head counts the fused tiles do not cover (odd value-head count) take the unfused launches:
+    # room for qkv, z, a, b as well
+    d_odd = _dims(kh=1, vh=3)
+    C_odd = (2 + 3) * 128
+    assert lib.gdn_prefill_hidden_workspace_size(ctypes.byref(d_odd), 4, 2) >= \
+        lib.gdn_prefill_workspace_size(ctypes.byref(d_odd), 4, 2) + 8 * (C_odd + 3 * 128 + 6) * 2
+    # packed rows: the packed prefill's workspace, z and the staged histories
+    assert lib.gdn_prefill_hidden_varlen_workspace_size(ctypes.byref(d), 3, 1000) >= \
+        lib.gdn_prefill_varlen_workspace_size(ctypes.byref(d), 3, 1000) + 1000 * 6144 * 2 + 3 * 3 * 10240 * 4
+    for cu, total in (([1, 5], 5), ([0, 5, 3], 3), ([0, 4], 5)):
+        arr = (ctypes.c_int32 * len(cu))(*cu)
+        assert lib.gdn_prefill_hidden_varlen(ctypes.byref(d), ctypes.byref(w), len(cu) - 1, arr, 16, total, 128,
+                                             16, 16, None, None, 16, None, None, 16, 1 << 30, None) == -1
     # the schedule query: null outputs, negative sizes
     seg, lau = ctypes.c_int32(-7), ctypes.c_int32(-7)
     assert lib.gdn_prefill_schedule(ctypes.byref(d), 1, 8192, 0, None, None) == -1

@@ -7,8 +7,9 @@ multiply-adds, silu, the L2 norm summed in the order of the load stage's warp
 reduction, the f16 hi/lo split, the gates), so outputs, final states and
 histories must be bit-identical: across the fused tiles' 125-token steps, rows
 that start and end inside a tile, rows with and without a history, in place,
-and the short-row path (rows of fewer than 3 tokens take the unfused launches).
-One small case also goes through the oracle (projection, then the mixer).
+rows shorter than the conv window, and packed rows (prefill_hidden_varlen against
+in_proj + prefill_varlen).  One small case also goes through the oracle (projection,
+then the mixer).
 """
 import numpy as np
 import pytest
@@ -54,7 +55,7 @@ def _unfused(dev, w, x, w_in, st, cv):
     (1, 300, 256, False),   # three fused tiles, ragged last one, zero history
     (3, 130, 128, True),    # rows start and end inside tiles (tiles step 125 tokens)
     (5, 3, 64, True),       # rows of exactly the conv window
-    (2, 2, 64, True),       # rows shorter than the window: the unfused launches
+    (2, 2, 64, True),       # rows shorter than the conv window: history partly the initial one
     (1, 1, 64, False),
     (2, 1000, 512, True),   # several 64-token chunks per row; overlapped schedule
 ])
@@ -83,6 +84,39 @@ def test_in_place_states(dev):
     torch.cuda.synchronize(dev)
     assert fs.data_ptr() == std.data_ptr() and fc.data_ptr() == cvd.data_ptr()
     assert torch.equal(out, ref[0]) and torch.equal(std, ref[1]) and torch.equal(cvd, ref[2])
+
+
+@pytest.mark.parametrize("lengths,init", [
+    ([0, 1, 2, 3, 130, 300, 5], True),     # empty and short rows, rows across tiles
+    ([64, 200, 1], False),
+    ([700, 0, 450], True),
+])
+def test_varlen_bit_identical_to_unfused(dev, lengths, init):
+    hidden = 256
+    total = sum(lengths)
+    w, x, w_in, st, cv = _case(sum(lengths) + len(lengths), 1, total, hidden, False)
+    gen = torch.Generator().manual_seed(len(lengths) * 7)
+    N = len(lengths)
+    st = synth.draw_state(gen, N, synth.MODEL) if init else None
+    cv = synth.draw_history(gen, N, synth.MODEL) if init else None
+    cu = torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32)
+    wd = gdn.weights_to(w, dev)
+    xd, wid = x[0].to(dev), w_in.to(dev)
+    std = st.to(dev) if st is not None else None
+    cvd = cv.to(dev) if cv is not None else None
+    qkv, z, a, b = gdn.in_proj(xd, wid)
+    ref = gdn.prefill_varlen(cu, qkv, z, a, b, wd, std, cvd)
+    got = gdn.prefill_hidden_varlen(cu, xd, wid, wd, std, cvd)
+    torch.cuda.synchronize(dev)
+    for g, r, name in zip(got, ref, ("out", "final_state", "final_conv")):
+        assert torch.equal(g, r), f"{name} differs from in_proj + prefill_varlen"
+    # in place
+    std2, cvd2 = (st.to(dev), cv.to(dev)) if init else (None, None)
+    if init:
+        gdn.prefill_hidden_varlen(cu, xd, wid, wd, std2, cvd2, in_place=True)
+        torch.cuda.synchronize(dev)
+        assert torch.equal(std2, ref[1]) and torch.equal(cvd2, ref[2])
+    assert gdn.last_device_error() == 0
 
 
 def test_layer_shape_bit_identical(dev):

@@ -21,12 +21,12 @@ def test_schedule():
     assert gdn.prefill_schedule(0, 100) == (0, 0)
     assert gdn.prefill_schedule(1, 0) == (0, 0)
     assert gdn.prefill_schedule(1, 15 * 64) == (1, 4)          # under 16 chunks: plain schedule
-    assert gdn.prefill_schedule(1, 15 * 64, True) == (1, 3)    # fused load stage, history copied
-    assert gdn.prefill_schedule(1, 2, True) == (1, 5)          # too short to fuse: in_proj + 4
+    assert gdn.prefill_schedule(1, 15 * 64, True) == (1, 4)    # fused in_proj GEMM, history, WY, recurrence
+    assert gdn.prefill_schedule(1, 2, True) == (1, 4)          # short rows fuse too
     s1, l1 = gdn.prefill_schedule(1, 8192)
     assert 2 <= s1 <= 8 and l1 == 2 + 2 * s1
     s2, l2 = gdn.prefill_schedule(1, 8192, True)
-    assert 2 <= s2 <= 8 and l2 == 1 + 2 * s2
+    assert 2 <= s2 <= 8 and l2 == 2 + 2 * s2
     s3, l3 = gdn.prefill_schedule(2, 65536)
     assert 2 <= s3 <= 8 and l3 == 2 + 2 * s3
     rows = (nsm - 32) // 48 + 1                                # the recurrence would take too many SMs
