@@ -557,21 +557,33 @@ def bench_long_context(args, local, line):
     dq = {k: case["decode"][k].to(dev) for k in ("qkv", "z", "a", "b")}
     dout = torch.empty((steps, B, 6144), dtype=torch.bfloat16, device=dev)
     st, cv = fs.clone(), fc.clone()
-    with torch.cuda.stream(stream):
+
+    def steps_pass():
         for s in range(steps):
             gdn.decode(dq["qkv"][s], dq["z"][s], dq["a"][s], dq["b"][s], w, st, cv, out=dout[s])
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
+
+    # the 256 launches as one captured graph (as a serving loop would replay them), from the
+    # prefill's states each time
+    with torch.cuda.stream(stream):
+        steps_pass()
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        steps_pass()
+    with torch.cuda.stream(stream):
         st.copy_(fs)
         cv.copy_(fc)
+        graph.replay()
+        st.copy_(fs)
+        cv.copy_(fc)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for s in range(steps):
-            gdn.decode(dq["qkv"][s], dq["z"][s], dq["a"][s], dq["b"][s], w, st, cv, out=dout[s])
+        graph.replay()
         e1.record(stream)
     torch.cuda.synchronize(dev)
     td = e0.elapsed_time(e1) / 1000.0
-    res["decode_after"] = {"workload": f"{steps} decode steps x {B} rows from the prefill's states",
+    res["decode_after"] = {"workload": f"{steps} decode steps x {B} rows from the prefill's states (CUDA graph)",
                            "value": B * steps / td, "unit": "row-tokens/s", "us_per_step": td / steps * 1e6,
                            "gpu_launches": steps}
     return res
