@@ -625,22 +625,33 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
         (st = smem_optin(reinterpret_cast<const void*>(gdn_decode_kernel<dec::kMaxTokens>), dec::kSmemLimit)) !=
             GDN_OK)
         return st;
-    const dec::Plan dplan = dec::plan(p.Vh / p.Kh, ntok);
-    if (dplan.stages < 2) return GDN_ERR_UNSUPPORTED;  // the group's inputs of ntok tokens leave no room
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
-    // persistent grid: one CTA per SM walking (row, q/k head) items round-robin
-    p.nitems = rows * p.Kh;
-    const int grid = p.nitems < nsm ? p.nitems : nsm;
+    // Work item = (row, q/k head) with its value heads, persistent CTAs walking the items.  A batch
+    // small enough that one CTA per value head still fits in one wave splits each q/k group over a
+    // cluster of Vh/Kh CTAs, one value head each (one item per CTA): 1 row 9.6 -> 6.8 us, 2 rows
+    // 9.9 -> 7.3 us; with more than one wave the persistent grouping is faster.
+    const int Gfull = p.Vh / p.Kh;
+    const bool split = Gfull > 1 && rows * p.Kh * Gfull <= nsm;
+    p.hpi = split ? 1 : Gfull;
+    const dec::Plan dplan = dec::plan(p.hpi, ntok);
+    if (dplan.stages < 2) return GDN_ERR_UNSUPPORTED;  // the group's inputs of ntok tokens leave no room
+    p.nitems = rows * p.Kh * (split ? Gfull : 1);
+    const int grid = split ? p.nitems : (p.nitems < nsm ? p.nitems : nsm);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(dec::kThreads);
     cfg.dynamicSmemBytes = dplan.smem_bytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = Gfull;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = split ? attr : nullptr;
+    cfg.numAttrs = split ? 1 : 0;
     return cuda_status(ntok == 1 ? cudaLaunchKernelEx(&cfg, gdn_decode_kernel<1>, p)
                                  : cudaLaunchKernelEx(&cfg, gdn_decode_kernel<dec::kMaxTokens>, p));
 }

@@ -40,6 +40,7 @@ namespace gdn {
 struct DecodeParams {
     int Kh, Vh, C, rows, nitems;
     int ntok;                // tokens per row (1 .. the kernel's maximum)
+    int hpi;                 // value heads per item: Vh / Kh, or 1 (a q/k group split over a cluster of CTAs)
     const uint16_t* qkv;     // bf16 [rows][ntok][C]
     const uint16_t* z;       // bf16 [rows][ntok][Vh*128]
     const uint16_t* a;       // bf16 [rows][ntok][Vh]
@@ -123,7 +124,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int G = p.Vh / p.Kh;
+    const int Gfull = p.Vh / p.Kh;         // value heads per q/k head
+    const int G = p.hpi;                   // value heads of one item
+    const int ns = Gfull / G;              // items per q/k group (> 1: one cluster of ns CTAs, one item each)
     const int nt = KMAX == 1 ? 1 : p.ntok;  // tokens per row
     const Plan pl = plan(G, nt);
     const int nst = pl.stages;
@@ -131,6 +134,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     uint64_t* empty = full + kMaxStages;
     uint64_t* auxfull = empty + kMaxStages;
     uint64_t* auxempty = auxfull + 2;
+    uint64_t* qkfree = auxempty + 2;  // split groups: the peers have read the q/k history (rank 0's copy)
     float* scratch = reinterpret_cast<float*>(smem + pl.off_misc + 256);
     float* s_q = scratch + pl.m_q;        // [nt][128]
     float* s_k = scratch + pl.m_k;        // [nt][128]
@@ -158,16 +162,26 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
             mbar_init(&auxfull[s], 1);
             mbar_init(&auxempty[s], kComputeThreads / 32);
         }
+        if (ns > 1) mbar_init(qkfree, ns - 1);
         fence_barrier_init();
     }
     __syncthreads();
+    if (ns > 1) cluster_sync();  // the cluster's barriers are initialised before any remote arrive
+
+    // item it -> batch row, q/k head, first value head (within the group) of the item
+    auto item = [&](int it, int& row, int& kap, int& hoff) {
+        const int rk = it / ns;
+        row = rk / p.Kh;
+        kap = rk - row * p.Kh;
+        hoff = (it - rk * ns) * G;
+    };
 
     // unit u of this CTA: item u / (2G), value head (u % 2G) / 2 of its group, half u % 2
     auto unit_ptr = [&](int u) -> float* {
-        const int it = blockIdx.x + (u / units_per_item) * gridDim.x;
-        const int row = it / p.Kh, kap = it % p.Kh;
+        int row, kap, hoff;
+        item(blockIdx.x + (u / units_per_item) * gridDim.x, row, kap, hoff);
         const int r = u % units_per_item;
-        const int head = kap * G + (r >> 1);
+        const int head = kap * Gfull + hoff + (r >> 1);
         return p.state + (((size_t)decode_slot(p, row) * p.Vh + head) * 128 + (r & 1) * 64) * 128;
     };
 
@@ -175,12 +189,12 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         // ---------------- producer warp: per-item inputs one item ahead, state half-tiles in a ring
         if (lane == 0) {
             auto aux_load = [&](int m) {
-                const int it = blockIdx.x + m * gridDim.x;
-                const int row = it / p.Kh, kap = it % p.Kh;
+                int row, kap, hoff;
+                item(blockIdx.x + m * gridDim.x, row, kap, hoff);
                 uint8_t* ax = smem + pl.off_aux + (m & 1) * pl.aux_bytes;
                 uint64_t* bar = &auxfull[m & 1];
                 mbar_arrive_expect_tx(bar, pl.aux_load_bytes);
-                const int chq = kap * 128, chk = p.Kh * 128 + kap * 128, chv = 2 * p.Kh * 128 + kap * G * 128;
+                const int chq = kap * 128, chk = p.Kh * 128 + kap * 128, chv = 2 * p.Kh * 128 + (kap * Gfull + hoff) * 128;
                 const int srow = decode_slot(p, row);
                 for (int r = 0; r < 3; ++r) {
                     const float* hrow = p.conv + ((size_t)srow * 3 + r) * p.C;
@@ -195,8 +209,8 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                     bulk_load(dx, xrow + chq, 256, bar);
                     bulk_load(dx + 128, xrow + chk, 256, bar);
                     bulk_load(dx + 256, xrow + chv, G * 256, bar);
-                    bulk_load(ax + pl.aux_z + j * G * 256, p.z + (((size_t)row * nt + j) * p.Vh + kap * G) * 128,
-                              G * 256, bar);
+                    bulk_load(ax + pl.aux_z + j * G * 256,
+                              p.z + (((size_t)row * nt + j) * p.Vh + kap * Gfull + hoff) * 128, G * 256, bar);
                 }
                 uint16_t* dw = reinterpret_cast<uint16_t*>(ax + pl.aux_w);
                 bulk_load(dw, p.conv_w + (size_t)chq * 4, 1024, bar);
@@ -227,8 +241,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     // gate inputs of the next item, loaded one item ahead (thread tid < G * nt: token tid / G, head tid % G)
     float ga = 0.f, gb = 0.f, gA = 0.f, gdt = 0.f;
     auto gate_prefetch = [&](int m) {
-        const int it = blockIdx.x + m * gridDim.x;
-        const int row = it / p.Kh, head = (it % p.Kh) * G + tid % G, j = tid / G;
+        int row, kap, hoff;
+        item(blockIdx.x + m * gridDim.x, row, kap, hoff);
+        const int head = kap * Gfull + hoff + tid % G, j = tid / G;
         ga = bf16_bits_to_float(p.a[((size_t)row * nt + j) * p.Vh + head]);
         gb = bf16_bits_to_float(p.b[((size_t)row * nt + j) * p.Vh + head]);
         gA = p.A_log[head];
@@ -237,12 +252,15 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     if (tid < G * nt && nmine > 0) gate_prefetch(0);
     int u = 0;
     for (int m = 0; m < nmine; ++m) {
-        const int it = blockIdx.x + m * gridDim.x;
-        const int row = it / p.Kh, kap = it % p.Kh;
+        int row, kap, hoff;
+        item(blockIdx.x + m * gridDim.x, row, kap, hoff);
         const int srow = decode_slot(p, row);
         const uint8_t* ax = smem + pl.off_aux + (m & 1) * pl.aux_bytes;
         named_barrier_sync(1, kComputeThreads);  // previous item's readers of the scratch are done
         bounded_wait(&auxfull[m & 1], (m >> 1) & 1, broken);
+        // split group: the q/k history is shifted by the group's first CTA once the others hold it
+        const bool qk_writer = ns == 1 || hoff == 0;
+        if (ns > 1 && hoff != 0 && tid == 0) mbar_arrive_remote(qkfree, 0);
 
         // ---- conv + silu of the item's channels over the nt tokens; shift their history in place
         const float* ah = reinterpret_cast<const float*>(ax);
@@ -255,7 +273,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 const int grp = idx >> 7, c = idx & 127;
                 const int ch = (grp == 0) ? kap * 128 + c
                              : (grp == 1) ? p.Kh * 128 + kap * 128 + c
-                                          : 2 * p.Kh * 128 + (kap * G + grp - 2) * 128 + c;
+                                          : 2 * p.Kh * 128 + (kap * Gfull + hoff + grp - 2) * 128 + c;
                 float h0 = ah[idx], h1 = ah[nch + idx], h2 = ah[2 * nch + idx];
                 const uint2 wb = aw[idx];
                 const float t0 = __uint_as_float(wb.x << 16), t1 = __uint_as_float(wb.x & 0xffff0000u);
@@ -273,10 +291,16 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                         h2 = x;
                     }
                 }
-                float* hr = p.conv + (size_t)srow * 3 * p.C + ch;
-                hr[0] = h0;
-                hr[p.C] = h1;
-                hr[2 * p.C] = h2;
+                if (grp >= 2 || qk_writer) {
+                    if (grp < 2 && ns > 1) {
+                        bounded_wait(qkfree, 0, broken);
+                        fence_acq_rel_cluster();
+                    }
+                    float* hr = p.conv + (size_t)srow * 3 * p.C + ch;
+                    hr[0] = h0;
+                    hr[p.C] = h1;
+                    hr[2 * p.C] = h2;
+                }
             }
         }
         if (tid < G * nt) {
@@ -381,7 +405,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                     for (int hh = 0; hh < G; ++hh) {
                         const float* r4 = s_red + j * nred + 8 + hh * 8;
                         const float ms = (r4[0] + r4[1] + r4[2] + r4[3]) * (1.0f / 128.0f);
-                        const int head = kap * G + hh;
+                        const int head = kap * Gfull + hoff + hh;
                         const float zv = bf16_bits_to_float(az[(j * G + hh) * 128 + tid]);
                         const float y = s_o[(j * G + hh) * 128 + tid] * rsqrtf(ms + kEps) * w_n * silu_f(zv);
                         p.out[(((size_t)row * nt + j) * p.Vh + head) * 128 + tid] = float_to_bf16_bits(y);

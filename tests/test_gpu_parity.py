@@ -82,6 +82,26 @@ def test_decode_batch_shape_sampled_heads():
     assert conv_exact(cv, cv_ref)
 
 
+def test_decode_split_groups_bit_identical():
+    """Batches small enough for one CTA per value head in one wave (at most 3 rows here) run
+    each q/k group as a cluster of one-value-head CTAs (the first shifts the shared q/k
+    history once the others hold it); the results are the same bits as the persistent
+    grouping: 6 rows at once against 3 + 2 + 1, over 3 steps."""
+    case = synth.decode_case(777, rows=6, steps=3)
+    w, _, st, cv = to_dev(case)
+    st2, cv2 = st.clone(), cv.clone()
+    for s in range(3):
+        acts = [case[k][s].cuda() for k in ("qkv", "z", "a", "b")]
+        o_all = gdn.decode(*acts, w, st, cv)
+        parts = []
+        for lo, hi in ((0, 3), (3, 5), (5, 6)):
+            parts.append(gdn.decode(*(t[lo:hi] for t in acts), w, st2[lo:hi], cv2[lo:hi]))
+        torch.cuda.synchronize()
+        assert torch.equal(o_all, torch.cat(parts))
+    assert torch.equal(st, st2) and torch.equal(cv, cv2)
+    assert gdn.last_device_error() == 0
+
+
 def test_decode_zero_rows_is_noop():
     case = synth.decode_case(3, rows=1, steps=1)
     w, _, st, cv = to_dev(case)
