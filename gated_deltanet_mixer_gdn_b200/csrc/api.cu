@@ -621,22 +621,23 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
     p.out = out;
     p.slots = slots;
     p.ntok = ntok;
-    if ((st = smem_optin(reinterpret_cast<const void*>(gdn_decode_kernel<1>), dec::kSmemLimit)) != GDN_OK ||
-        (st = smem_optin(reinterpret_cast<const void*>(gdn_decode_kernel<dec::kMaxTokens>), dec::kSmemLimit)) !=
-            GDN_OK)
-        return st;
+    const void* kernels[4] = {reinterpret_cast<const void*>(gdn_decode_kernel<1, false>),
+                              reinterpret_cast<const void*>(gdn_decode_kernel<dec::kMaxTokens, false>),
+                              reinterpret_cast<const void*>(gdn_decode_kernel<1, true>),
+                              reinterpret_cast<const void*>(gdn_decode_kernel<dec::kMaxTokens, true>)};
+    for (const void* k : kernels)
+        if ((st = smem_optin(k, dec::kSmemLimit)) != GDN_OK) return st;
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
     // Work item = (row, q/k head) with its value heads, persistent CTAs walking the items.  A batch
     // small enough that one CTA per value head still fits in one wave splits each q/k group over a
-    // cluster of Vh/Kh CTAs, one value head each (one item per CTA): 1 row 9.6 -> 6.8 us, 2 rows
-    // 9.9 -> 7.3 us; with more than one wave the persistent grouping is faster.
+    // cluster of Vh/Kh CTAs, one value head each (one item per CTA): 1 row 9.6 -> 6.3 us, 2 rows
+    // 9.9 -> 6.5 us; with more than one wave the persistent grouping is faster.
     const int Gfull = p.Vh / p.Kh;
     const bool split = Gfull > 1 && rows * p.Kh * Gfull <= nsm;
-    p.hpi = split ? 1 : Gfull;
-    const dec::Plan dplan = dec::plan(p.hpi, ntok);
+    const dec::Plan dplan = dec::plan(split ? 1 : Gfull, ntok);
     if (dplan.stages < 2) return GDN_ERR_UNSUPPORTED;  // the group's inputs of ntok tokens leave no room
     p.nitems = rows * p.Kh * (split ? Gfull : 1);
     const int grid = split ? p.nitems : (p.nitems < nsm ? p.nitems : nsm);
@@ -652,8 +653,11 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = split ? attr : nullptr;
     cfg.numAttrs = split ? 1 : 0;
-    return cuda_status(ntok == 1 ? cudaLaunchKernelEx(&cfg, gdn_decode_kernel<1>, p)
-                                 : cudaLaunchKernelEx(&cfg, gdn_decode_kernel<dec::kMaxTokens>, p));
+    if (split)
+        return cuda_status(ntok == 1 ? cudaLaunchKernelEx(&cfg, gdn_decode_kernel<1, true>, p)
+                                     : cudaLaunchKernelEx(&cfg, gdn_decode_kernel<dec::kMaxTokens, true>, p));
+    return cuda_status(ntok == 1 ? cudaLaunchKernelEx(&cfg, gdn_decode_kernel<1, false>, p)
+                                 : cudaLaunchKernelEx(&cfg, gdn_decode_kernel<dec::kMaxTokens, false>, p));
 }
 
 

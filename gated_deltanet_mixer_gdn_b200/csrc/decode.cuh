@@ -40,7 +40,6 @@ namespace gdn {
 struct DecodeParams {
     int Kh, Vh, C, rows, nitems;
     int ntok;                // tokens per row (1 .. the kernel's maximum)
-    int hpi;                 // value heads per item: Vh / Kh, or 1 (a q/k group split over a cluster of CTAs)
     const uint16_t* qkv;     // bf16 [rows][ntok][C]
     const uint16_t* z;       // bf16 [rows][ntok][Vh*128]
     const uint16_t* a;       // bf16 [rows][ntok][Vh]
@@ -119,14 +118,17 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, boo
     return true;
 }
 
-template <int KMAX>
+// SPLIT = false: an item is a q/k group (all its value heads), persistent CTAs walk the items.
+// SPLIT = true: an item is one value head; the Vh / Kh items of a group are the CTAs of one
+// thread-block cluster (one item each), launched with that cluster size.
+template <int KMAX, bool SPLIT>
 __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const DecodeParams p) {
     using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int Gfull = p.Vh / p.Kh;         // value heads per q/k head
-    const int G = p.hpi;                   // value heads of one item
-    const int ns = Gfull / G;              // items per q/k group (> 1: one cluster of ns CTAs, one item each)
+    const int G = SPLIT ? 1 : Gfull;       // value heads of one item
+    const int ns = SPLIT ? Gfull : 1;      // items per q/k group
     const int nt = KMAX == 1 ? 1 : p.ntok;  // tokens per row
     const Plan pl = plan(G, nt);
     const int nst = pl.stages;
@@ -162,18 +164,18 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
             mbar_init(&auxfull[s], 1);
             mbar_init(&auxempty[s], kComputeThreads / 32);
         }
-        if (ns > 1) mbar_init(qkfree, ns - 1);
+        if (SPLIT) mbar_init(qkfree, ns - 1);
         fence_barrier_init();
     }
     __syncthreads();
-    if (ns > 1) cluster_sync();  // the cluster's barriers are initialised before any remote arrive
+    if (SPLIT) cluster_sync();  // the cluster's barriers are initialised before any remote arrive
 
     // item it -> batch row, q/k head, first value head (within the group) of the item
     auto item = [&](int it, int& row, int& kap, int& hoff) {
-        const int rk = it / ns;
+        const int rk = SPLIT ? it / ns : it;
         row = rk / p.Kh;
         kap = rk - row * p.Kh;
-        hoff = (it - rk * ns) * G;
+        hoff = SPLIT ? it - rk * ns : 0;
     };
 
     // unit u of this CTA: item u / (2G), value head (u % 2G) / 2 of its group, half u % 2
@@ -259,8 +261,8 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         named_barrier_sync(1, kComputeThreads);  // previous item's readers of the scratch are done
         bounded_wait(&auxfull[m & 1], (m >> 1) & 1, broken);
         // split group: the q/k history is shifted by the group's first CTA once the others hold it
-        const bool qk_writer = ns == 1 || hoff == 0;
-        if (ns > 1 && hoff != 0 && tid == 0) mbar_arrive_remote(qkfree, 0);
+        const bool qk_writer = !SPLIT || hoff == 0;
+        if (SPLIT && hoff != 0 && tid == 0) mbar_arrive_remote(qkfree, 0);
 
         // ---- conv + silu of the item's channels over the nt tokens; shift their history in place
         const float* ah = reinterpret_cast<const float*>(ax);
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                     }
                 }
                 if (grp >= 2 || qk_writer) {
-                    if (grp < 2 && ns > 1) {
+                    if (SPLIT && grp < 2) {
                         bounded_wait(qkfree, 0, broken);
                         fence_acq_rel_cluster();
                     }
