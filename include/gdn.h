@@ -89,6 +89,13 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
  * T = 0 is legal: states and histories are copied through.
  * The prefill computes the recurrence in chunks of 64 tokens (WY form) on
  * tensor cores with f16 operands and f32 accumulation.
+ * When the recurrence leaves most SMs idle (few rows of at least 16 chunks;
+ * gdn_prefill_schedule reports the plan) the call forks onto two internal
+ * streams of the device (created on first use) through events recorded on
+ * `stream`, and joins back onto `stream` before returning: the work stays
+ * ordered on `stream` and can be captured into a CUDA graph.  Concurrent
+ * calls from several host threads share those internal streams and run one
+ * after the other there.
  */
 int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T,
                 const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
