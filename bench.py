@@ -185,6 +185,15 @@ def cpu_baseline_line(case, budget_s: float = 15.0):
             "sample": f"{rows} rows x {steps} decode tokens of the 64x128 decode batch (all 48 heads), f64"}
 
 
+DECODE_METRIC = "GDN decode row-tokens/s (64-row batch, 128 steps)"
+
+
+def decode_config(world):
+    return {"workload": "decode 64 rows x 128 steps, Qwen3.8-27B GDN layer shapes (16 qk / 48 v heads, dim 128), "
+                        "per-row f32 state", "rows": ROWS, "tokens_per_row": DECODE_STEPS,
+            "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (402.7 MB of state per step)"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -198,11 +207,11 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         t += oracle_decode_sample(case, steps, rows)
     value = rows * steps * args.steps / t
-    line = {"impl": "reference", "metric": "GDN decode row-tokens/s (64-row batch)", "value": value,
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value,
             "unit": "row-tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * t / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "decode 64 rows x 128 steps, Qwen3.8-27B GDN shapes (oracle sample)"},
+            "config": decode_config(1),
             "cpu_baseline": {"value": value, "unit": "row-tokens/s", "cores": oracle.max_threads(),
                              "kind": "oracle", "sample": f"{rows} rows x {steps} tokens per step, all 48 heads"},
             "e2e": {"value": value, "unit": "row-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -322,14 +331,11 @@ def run_ours(args, world, rank, local):
     line = None
     if rank == 0:
         line = {
-            "metric": "GDN decode row-tokens/s (64-row batch, 128 steps)",
+            "metric": DECODE_METRIC,
             "value": value, "unit": "row-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "decode 64 rows x 128 steps, Qwen3.8-27B GDN layer shapes (16 qk / 48 v heads, "
-                                   "dim 128), per-row f32 state", "rows": ROWS, "tokens_per_row": DECODE_STEPS,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (402.7 MB of state per step)"},
+            "config": decode_config(world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": decode_traffic(),
                          "kernel": "gdn_decode_kernel", "peak_source": peaks["source"],
