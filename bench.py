@@ -437,6 +437,12 @@ def prefill_launches(B, T, from_hidden=False):
     return gdn.prefill_schedule(B, T, from_hidden)[1]
 
 
+def prefill_launches_varlen():
+    """Kernels one packed (varlen) prefill call launches: load stage, history writer, chunk
+    offsets and row order, WY records, recurrence."""
+    return 5
+
+
 def bench_hidden(args, local, T=8192):
     """Prefill of one row of T tokens from the layer's hidden states [T,5120]: the load
     stage inside the in_proj GEMM (gdn_prefill_hidden) against in_proj followed by the
@@ -494,13 +500,121 @@ def _time_prefill(call, dev, stream, warmup, reps):
     return statistics.median(pt), len(pt)
 
 
-def bench_prefill(args, world, rank, local, T):
-    """Chunked prefill: one row of T tokens from zero state, and the 8-row varlen
-    workload (lengths U[512,16384] from the seed, random initial state and history)."""
+def prefill_line(tokens, sec, workload, launches, peaks):
+    tf = tokens * PREFILL_FLOP_PER_TOKEN / sec / 1e12
+    return {"workload": workload, "value": tokens / sec, "unit": "tokens/s", "ms": sec * 1000.0,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"],
+                         "scope": "whole call (every kernel of the prefill)",
+                         "algorithmic_flop_per_token": PREFILL_FLOP_PER_TOKEN},
+            "l2": "flushed (256 MiB write) before each timed call", "gpu_launches": launches}
+
+
+def oracle_prefill_sample(case, rows, tokens):
+    """Seconds the float64 oracle takes for the first `tokens` tokens of each of the given rows
+    (all 48 heads, the rows' initial state and history)."""
+    import numpy as np
+    import oracle
+    f = synth.to_f64
+    w = case["weights"]
+    if "cu_seqlens" in case:
+        cu = case["cu_seqlens"].tolist()
+        spans = [(cu[r], min(cu[r + 1], cu[r] + tokens)) for r in rows]
+        take = lambda t: torch.cat([t[a:b] for a, b in spans])  # noqa: E731
+    else:
+        spans = [(0, tokens)] * len(rows)
+        take = lambda t: t[list(rows), :tokens].reshape(-1, t.shape[-1])  # noqa: E731
+    lens = [b - a for a, b in spans]
+    cu_s = np.concatenate([[0], np.cumsum(lens)])
+    st = None if case["init_state"] is None else f(case["init_state"][list(rows)])
+    cv = None if case["init_conv"] is None else f(case["init_conv"][list(rows)])
+    acts = {k: f(take(case[k])) for k in ("qkv", "z", "a", "b")}
+    t0 = time.perf_counter()
+    oracle.mixer(case["dims"], cu_s, acts["qkv"], acts["z"], acts["a"], acts["b"], f(w["conv_w"]), f(w["A_log"]),
+                 f(w["dt_bias"]), f(w["norm_w"]), st, cv)
+    return time.perf_counter() - t0, int(sum(lens))
+
+
+def prefill_cpu_baseline(case, rows, tokens, what):
+    import oracle
+    oracle.build()
+    dt, n = oracle_prefill_sample(case, rows, tokens)
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{what}: the first {tokens} tokens of {len(rows)} row(s), all 48 heads, f64 ({dt:.1f} s)"}
+
+
+def prefill_e2e(args, dev, case, w, seg=2048):
+    """One row of T tokens through the public API from pinned host buffers, as a serving loop
+    streams a long prompt: the row is cut into segments of `seg` tokens; segment k+1's inputs
+    go host -> device on a copy stream while segment k runs (each segment's prefill continues
+    from the state and history the previous one left), and each segment's output goes back on
+    another stream; the final state and history come back after the last segment.  Every input
+    and output byte crosses inside the timed region."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    T = case["qkv"].shape[1]
+    nseg = T // seg
+    pin = {k: case[k][0].pin_memory() for k in ("qkv", "z", "a", "b")}
+    din = {k: torch.empty_like(v, device=dev) for k, v in pin.items()}
+    host_out = torch.empty((T, 6144), dtype=torch.bfloat16).pin_memory()
+    host_st = torch.empty((1, 48, 128, 128), dtype=torch.float32).pin_memory()
+    host_cv = torch.empty((1, 3, 10240), dtype=torch.float32).pin_memory()
+    dout = torch.empty((T, 6144), dtype=torch.bfloat16, device=dev)
+    st = [torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev) for _ in range(2)]
+    cv = [torch.empty((1, 3, 10240), dtype=torch.float32, device=dev) for _ in range(2)]
+    h2d_bytes = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h_bytes = host_out.numel() * 2 + host_st.numel() * 4 + host_cv.numel() * 4
+    comp, h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nseg)]
+    ev_out = [torch.cuda.Event() for _ in range(nseg)]
+
+    def one_pass():
+        h2d.wait_stream(comp)
+        for k in range(nseg):
+            sl = slice(k * seg, (k + 1) * seg)
+            with torch.cuda.stream(h2d):
+                for n in din:
+                    din[n][sl].copy_(pin[n][sl], non_blocking=True)
+                ev_in[k].record(h2d)
+            comp.wait_event(ev_in[k])
+            with torch.cuda.stream(comp):
+                acts = [din[n][sl].unsqueeze(0) for n in ("qkv", "z", "a", "b")]
+                gdn.prefill(*acts, w, None if k == 0 else st[(k - 1) % 2], None if k == 0 else cv[(k - 1) % 2],
+                            out=dout[sl].unsqueeze(0), final_state=st[k % 2], final_conv=cv[k % 2])
+                ev_out[k].record(comp)
+            d2h.wait_event(ev_out[k])
+            with torch.cuda.stream(d2h):
+                host_out[sl].copy_(dout[sl], non_blocking=True)
+        with torch.cuda.stream(d2h):
+            host_st.copy_(st[(nseg - 1) % 2], non_blocking=True)
+            host_cv.copy_(cv[(nseg - 1) % 2], non_blocking=True)
+        comp.wait_stream(d2h)
+
+    one_pass()
+    torch.cuda.synchronize(dev)
+    reps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for _ in range(reps):
+        one_pass()
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    sec = e0.elapsed_time(e1) / 1000.0 / reps
+    return {"value": T / sec, "unit": "tokens/s", "ms": sec * 1000.0, "h2d_bytes_per_step": h2d_bytes,
+            "d2h_bytes_per_step": d2h_bytes, "segments": nseg,
+            "how": f"{nseg} segments of {seg} tokens, copies overlapped with the previous segment's prefill"}
+
+
+def bench_prefill(args, world, rank, local, T, full=True):
+    """Chunked prefill.  Top level: one row of T tokens from zero state (the 8192-token
+    workload), with its roofline, the oracle timed on a sample of it, and the end-to-end number
+    through the public API from host buffers.  Nested beside it (full=True): the 256-token row,
+    the 4096 + 4096 split run carrying state, the 8-row varlen workload and the 2 x 65,536
+    long-context rows."""
     import gated_deltanet_mixer_gdn_b200 as gdn
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     stream = torch.cuda.Stream(dev)
+    warm, reps = max(3, args.warmup), max(5, args.steps)
     pcase = synth.config(2) if T == 8192 else synth.dense_case(1236, 1, T)
     pw = gdn.weights_to(pcase["weights"], dev)
     a1 = {k: pcase[k].to(dev) for k in ("qkv", "z", "a", "b")}
@@ -508,18 +622,46 @@ def bench_prefill(args, world, rank, local, T):
     pst = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
     pcv = torch.empty((1, 3, 10240), dtype=torch.float32, device=dev)
     t1, n1 = _time_prefill(lambda: gdn.prefill(a1["qkv"], a1["z"], a1["a"], a1["b"], pw, out=pout, final_state=pst,
-                                               final_conv=pcv), dev, stream, max(3, args.warmup), max(5, args.steps))
+                                               final_conv=pcv), dev, stream, warm, reps)
+    res = prefill_line(T, t1, f"prefill B=1 T={T}, zero initial state, final state returned",
+                       prefill_launches(1, T) * n1, peaks)
+    res["metric"] = "GDN prefill tokens/s"
+    if T % 2048 == 0:
+        res["e2e"] = prefill_e2e(args, dev, pcase, pw)
+    if not full:
+        return res
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = prefill_cpu_baseline(pcase, [0], 2048, f"prefill B=1 T={T}")
+    configs = {}
+    # 4096 + 4096: the second half continues from the state and history the first half left
+    h = T // 2
+    halves = [{k: a1[k][:, i * h:(i + 1) * h].contiguous() for k in a1} for i in range(2)]
+    sst = torch.empty_like(pst)
+    scv = torch.empty_like(pcv)
 
-    def line(tokens, sec, workload, launches):
-        tf = tokens * PREFILL_FLOP_PER_TOKEN / sec / 1e12
-        return {"workload": workload, "value": tokens / sec, "unit": "tokens/s", "ms": sec * 1000.0,
-                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                             "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"],
-                             "algorithmic_flop_per_token": PREFILL_FLOP_PER_TOKEN},
-                "l2": "flushed (256 MiB write) before each timed call", "gpu_launches": launches}
+    def split():
+        gdn.prefill(halves[0]["qkv"], halves[0]["z"], halves[0]["a"], halves[0]["b"], pw, out=pout[:, :h],
+                    final_state=sst, final_conv=scv)
+        gdn.prefill(halves[1]["qkv"], halves[1]["z"], halves[1]["a"], halves[1]["b"], pw, sst, scv, out=pout[:, h:],
+                    final_state=pst, final_conv=pcv)
 
-    # launches per call: see prefill_launches (packed rows: load stage, history out, chunk offsets, WY, recurrence)
-    out = {"b1": line(T, t1, f"prefill B=1 T={T}, zero initial state", prefill_launches(1, T) * n1)}
+    ts, ns = _time_prefill(split, dev, stream, warm, reps)
+    configs["split"] = prefill_line(T, ts, f"prefill B=1 T={T} as {h} + {h} tokens, state and history carried",
+                                    2 * prefill_launches(1, h) * ns, peaks)
+    # the 256-token row (latency)
+    c0 = synth.config(0)
+    w0 = gdn.weights_to(c0["weights"], dev)
+    a0 = {k: c0[k].to(dev) for k in ("qkv", "z", "a", "b")}
+    o0 = torch.empty((1, 256, 6144), dtype=torch.bfloat16, device=dev)
+    s0 = torch.empty_like(pst)
+    v0 = torch.empty_like(pcv)
+    t0, n0 = _time_prefill(lambda: gdn.prefill(a0["qkv"], a0["z"], a0["a"], a0["b"], w0, out=o0, final_state=s0,
+                                               final_conv=v0), dev, stream, warm, reps)
+    configs["t256"] = prefill_line(256, t0, "prefill B=1 T=256, zero initial state (latency)",
+                                   prefill_launches(1, 256) * n0, peaks)
+    configs["t256"]["us"] = t0 * 1e6
+    if world == 1 and not args.no_cpu_baseline:
+        configs["t256"]["cpu_baseline"] = prefill_cpu_baseline(c0, [0], 256, "prefill B=1 T=256")
     if T == 8192:
         vcase = synth.config(3)
         vw = gdn.weights_to(vcase["weights"], dev)
@@ -533,11 +675,17 @@ def bench_prefill(args, world, rank, local, T):
         t2, n2 = _time_prefill(lambda: gdn.prefill_varlen(cu, av["qkv"], av["z"], av["a"], av["b"], vw, st0, cv0,
                                                           out=vout, final_state=vst, final_conv=vcv,
                                                           cu_seqlens_dev=cud),
-                               dev, stream, max(3, args.warmup), max(5, args.steps))
-        out["varlen8"] = line(total, t2, f"varlen prefill 8 rows ({total} tokens, lengths U[512,16384]), "
-                                         "random initial state and history", 5 * n2)
-        out["long2"] = bench_long_context(args, local, line)
-    return out
+                               dev, stream, warm, reps)
+        configs["varlen8"] = prefill_line(total, t2, f"varlen prefill 8 rows ({total} tokens, lengths "
+                                          "U[512,16384]), random initial state and history",
+                                          prefill_launches_varlen() * n2, peaks)
+        if world == 1 and not args.no_cpu_baseline:
+            configs["varlen8"]["cpu_baseline"] = prefill_cpu_baseline(vcase, list(range(8)), 512,
+                                                                      "varlen prefill 8 rows")
+        del av, st0, cv0, vout, vst, vcv
+        configs["long2"] = bench_long_context(args, local, lambda *a: prefill_line(*a, peaks))
+    res["configs"] = configs
+    return res
 
 
 def bench_long_context(args, local, line):
@@ -558,6 +706,8 @@ def bench_long_context(args, local, line):
                                              final_conv=fc), dev, stream, 3, reps)
     res = line(B * T, t, f"long-context prefill B={B} T={T}, zero initial state, final states returned",
                prefill_launches(B, T) * n)
+    if not args.no_cpu_baseline:
+        res["cpu_baseline"] = prefill_cpu_baseline(case, [0, 1], 1024, f"long-context prefill B={B} T={T}")
     # 256 decode steps per row from the prefill's states (2 rows: launch-latency bound, reported)
     steps = case["decode"]["qkv"].shape[0]
     dq = {k: case["decode"][k].to(dev) for k in ("qkv", "z", "a", "b")}
@@ -606,6 +756,8 @@ def main():
                     help="decode: the 64-row decode batch (default line); prefill: only the chunked prefill; "
                          "hidden: only the prefill from hidden states (fused in_proj + load stage)")
     ap.add_argument("--prefill-T", type=int, default=PREFILL_T, help="tokens of the prefill measurement")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="with --workload prefill: only the one-row prefill (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -619,9 +771,9 @@ def main():
                 print(json.dumps({"metric": "GDN prefill from hidden states tokens/s", **hid}))
             return 0
         if args.workload == "prefill":
-            pre = bench_prefill(args, world, rank, local, args.prefill_T)
+            pre = bench_prefill(args, world, rank, local, args.prefill_T, full=not args.prefill_only)
             if rank == 0:
-                print(json.dumps({"metric": "GDN prefill tokens/s", **pre["b1"], "varlen8": pre.get("varlen8")}))
+                print(json.dumps(pre))
             return 0
         line, case = run_ours(args, world, rank, local)
         pre = bench_prefill(args, world, rank, local, args.prefill_T)

@@ -29,7 +29,7 @@ EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_schedule", 
            "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
            "gdn_in_proj", "gdn_out_proj", "gdn_prefill_hidden_workspace_size", "gdn_prefill_hidden",
            "gdn_prefill_hidden_varlen_workspace_size", "gdn_prefill_hidden_varlen",
-           "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_status_string",
+           "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_set_decode_wait_limit", "gdn_status_string",
            "gdn_version")
 
 GDN_OK = 0
@@ -98,6 +98,8 @@ def load_library() -> ctypes.CDLL:
                                                vp, sz, vp]
         L.gdn_last_device_error.restype = ctypes.c_int
         L.gdn_last_device_error.argtypes = []
+        L.gdn_set_decode_wait_limit.restype = ctypes.c_int
+        L.gdn_set_decode_wait_limit.argtypes = [ctypes.c_uint64]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_version.restype = ctypes.c_int
@@ -463,12 +465,21 @@ def prefill_varlen_slots(cu_seqlens, slots, qkv, z, a, b, weights, state_pool, c
 
 
 def last_device_error() -> int:
+    """The device error word (0, or the code of the first bounded wait that ran out); cleared by reading."""
     return load_library().gdn_last_device_error()
+
+
+DECODE_WAIT_LIMIT_DEFAULT_NS = 2_000_000_000
+
+
+def set_decode_wait_limit(ns: int = DECODE_WAIT_LIMIT_DEFAULT_NS) -> None:
+    """Bound of every wait inside the decode kernels on the current device (default 2 s)."""
+    _check(load_library().gdn_set_decode_wait_limit(int(ns)), "gdn_set_decode_wait_limit")
 
 
 def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tensor]:
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_schedule", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_hidden_varlen", "prefill_varlen_slots", "last_device_error", "status_string", "load_library",
+__all__ = ["prefill", "prefill_schedule", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_hidden_varlen", "prefill_varlen_slots", "last_device_error", "set_decode_wait_limit", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

@@ -565,21 +565,60 @@ int check_io(int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16
 // up once per device below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
 
+// The address is cached per CUDA context (by the driver's unique context id), so a
+// context that replaced an earlier one on the same device (after cudaDeviceReset) gets
+// its own lookup instead of a stale pointer.
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
+struct NoallocEntry {
+    unsigned long long ctx_id;
+    void* addr;
+};
+std::vector<NoallocEntry> g_noalloc_addr;
 
-// Device address of g_noalloc_scratch on the current device (resolved on first use).
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+void* driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return p;
+}
+
+// Unique id of the current context (0 if there is none or the driver cannot say).
+unsigned long long current_ctx_id() {
+    static PfnCtxGetCurrent get_cur = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_cur = reinterpret_cast<PfnCtxGetCurrent>(driver_fn("cuCtxGetCurrent"));
+        get_id = reinterpret_cast<PfnCtxGetId>(driver_fn("cuCtxGetId"));
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_cur == nullptr || get_id == nullptr || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of g_noalloc_scratch in the current context (resolved on first use there;
+// cudaGetSymbolAddress also makes the device's primary context current if it was not).
 int noalloc_scratch(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+    unsigned long long id = current_ctx_id();
+    for (const NoallocEntry& e : g_noalloc_addr)
+        if (id != 0 && e.ctx_id == id) {
+            *out = e.addr;
+            return GDN_OK;
+        }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
+    if (id == 0) id = current_ctx_id();
+    if (id != 0) g_noalloc_addr.push_back(NoallocEntry{id, p});
+    *out = p;
     return GDN_OK;
 }
 
@@ -1009,6 +1048,13 @@ int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, i
     return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, a, b, init_state, init_conv, out,
                         final_state, final_conv, scratch, (size_t)GDN_NOALLOC_SCRATCH_BYTES,
                         static_cast<cudaStream_t>(stream), false);
+}
+
+int gdn_set_decode_wait_limit(uint64_t ns) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    const unsigned long long v = ns;
+    if (cudaMemcpyToSymbol(gdn::g_decode_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return GDN_ERR_CUDA;
+    return cudaDeviceSynchronize() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 int gdn_last_device_error(void) {

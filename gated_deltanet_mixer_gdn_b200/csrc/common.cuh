@@ -28,6 +28,12 @@ constexpr float kEps = 1e-6f;  // eps of the L2 norms and of the gated RMSNorm
 // wait (a chunk step takes microseconds), short enough to return control.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Bound of the decode kernel's waits (settable from the host through
+// gdn_set_decode_wait_limit; the kernels that hold tensor memory keep the fixed
+// bound above).  A wait that runs out sets the error word; the kernel then
+// stops issuing copies, drains the ones in flight and returns.
+__device__ unsigned long long g_decode_wait_limit_ns = kWaitLimitNs;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -64,15 +70,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false after the limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete; false after `limit_ns`.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(a, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
     return true;
+}
+
+// The same with the fixed bound.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -108,9 +108,11 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// Once one of this thread's waits has run out (`broken`), it waits no more: it records
+// the error once, and the caller no longer releases buffers or issues copies.
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, bool& broken) {
     if (broken) return false;
-    if (!mbar_wait(bar, parity)) {
+    if (!mbar_wait_for(bar, parity, g_decode_wait_limit_ns)) {
         broken = true;
         record_error(kErrTimeoutTma);
         return false;
@@ -220,20 +222,36 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 bulk_load(dw + 1024, p.conv_w + (size_t)chv * 4, G * 1024, bar);
             };
             // the next item's inputs are requested once the ring holds this item's first stages,
-            // by which time the item two back has released their buffer
+            // by which time the item two back has released their buffer.  A buffer is only
+            // refilled after every consumer released it, so no phase is armed twice; if a wait
+            // for a release runs out (the consumers stopped releasing after a wait of their own
+            // ran out), no further copy is issued.
             const int lead = nst < units_per_item - 1 ? nst : units_per_item - 1;
-            if (nmine > 0) aux_load(0);
+            int issued = 0, issued_aux = 0;
+            if (nmine > 0) {
+                aux_load(0);
+                issued_aux = 1;
+            }
             for (int u = 0; u < nunits; ++u) {
                 const int m = u / units_per_item, r = u % units_per_item;
                 if (r == lead && m + 1 < nmine) {
-                    if (m >= 1) bounded_wait(&auxempty[(m + 1) & 1], ((m - 1) >> 1) & 1, broken);
+                    if (m >= 1 && !bounded_wait(&auxempty[(m + 1) & 1], ((m - 1) >> 1) & 1, broken)) break;
                     aux_load(m + 1);
+                    issued_aux = m + 2;
                 }
                 const int st = u % nst;
-                if (u >= nst) bounded_wait(&empty[st], ((u / nst) - 1) & 1, broken);
+                if (u >= nst && !bounded_wait(&empty[st], ((u / nst) - 1) & 1, broken)) break;
                 mbar_arrive_expect_tx(&full[st], kTileBytes);
                 bulk_load(smem + st * kTileBytes, unit_ptr(u), kTileBytes, &full[st]);
+                issued = u + 1;
             }
+            // Drain: every copy issued into this CTA's shared memory has landed before the CTA
+            // can exit (on the normal path these phases are complete already).  Only the last
+            // phase armed on each buffer can still be open.
+            for (int v = issued > nst ? issued - nst : 0; v < issued; ++v)
+                mbar_wait(&full[v % nst], (v / nst) & 1);
+            for (int m = issued_aux > 2 ? issued_aux - 2 : 0; m < issued_aux; ++m)
+                mbar_wait(&auxfull[m & 1], (m >> 1) & 1);
         }
         return;
     }
@@ -351,7 +369,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
 #pragma unroll
                 for (int r = 0; r < 8; ++r) s[r] = reinterpret_cast<const float4*>(tile + (warp * 8 + r) * 128)[lane];
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done reading the stage
+                if (lane == 0 && !broken) mbar_arrive(&empty[st]);  // this warp is done reading the stage
                 const int irow = half * 64 + warp * 8 + (lane >> 2);
 #pragma unroll 1
                 for (int j = 0; j < nt; ++j) {
@@ -416,7 +434,15 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&auxempty[m & 1]);  // this warp is done with the item's inputs
+        if (lane == 0 && !broken) mbar_arrive(&auxempty[m & 1]);  // this warp is done with the item's inputs
+    }
+    // Split group: the peers signal rank 0's q/k-history barrier in rank 0's shared memory.  If
+    // rank 0 gave up waiting for them, it still holds until they have signalled (fixed bound),
+    // so no remote arrive reaches a CTA that has exited.
+    if (SPLIT && tid == 0 && nmine > 0) {
+        int row, kap, hoff;
+        item(blockIdx.x, row, kap, hoff);
+        if (hoff == 0) mbar_wait(qkfree, 0);
     }
 }
 

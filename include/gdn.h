@@ -25,9 +25,12 @@
  *
  * Memory: every pointer is DEVICE memory owned by the caller, 16-byte
  * aligned, densely packed in the layouts given.  bf16 tensors are passed as
- * uint16_t bit patterns.  The library allocates nothing and keeps no state
- * between calls other than a per-process cache of driver entry points, a
- * device-side error word, and the fixed scratch array of gdn_prefill_noalloc.
+ * uint16_t bit patterns.  The library allocates no device memory and keeps no
+ * state between calls other than a per-process cache of driver entry points,
+ * two internal streams and a few events per device (created by the first
+ * prefill that overlaps its kernels, see gdn_prefill), a device-side error word
+ * with the decode kernels' wait bound, and the fixed scratch array of
+ * gdn_prefill_noalloc.
  *
  * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  * Every call only enqueues work on it and returns; results are ready when
@@ -297,9 +300,25 @@ int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, i
                         const float* init_state, const float* init_conv,
                         uint16_t* out, float* final_state, float* final_conv, void* stream);
 
-/* Device-side error word of the current device: 0, or the code of the last
- * bounded wait that expired (cleared by reading).  Synchronises the device. */
+/* Device-side error word of the current device: 0, or the code of the first
+ * bounded wait that expired since the last read (GDN_DEVERR_TIMEOUT_COPY: a wait
+ * for a bulk copy or for a buffer to be released; GDN_DEVERR_TIMEOUT_MMA: a wait
+ * for a tensor-core product).  Cleared by reading.  Synchronises the device. */
+#define GDN_DEVERR_TIMEOUT_COPY 1
+#define GDN_DEVERR_TIMEOUT_MMA 2
 int gdn_last_device_error(void);
+
+/* Bound, in nanoseconds, of every wait inside the decode kernels (gdn_decode,
+ * gdn_decode_multi, gdn_decode_slots) on the current device; the default is
+ * GDN_DECODE_WAIT_LIMIT_DEFAULT_NS (2 s).  A wait that runs out sets the error
+ * word above; the kernel then stops issuing copies, waits (up to 2 s) for the
+ * copies it already issued, and returns with its outputs undefined, leaving the
+ * context usable.  A small bound makes waits run out on purpose (the library's
+ * test of that path uses 0); restore the default afterwards.  The kernels that
+ * hold tensor memory (prefill, projections) keep a fixed 2 s bound.
+ * Synchronises the device; not for use during stream capture. */
+#define GDN_DECODE_WAIT_LIMIT_DEFAULT_NS 2000000000ull
+int gdn_set_decode_wait_limit(uint64_t ns);
 
 /* Human-readable text of a gdn_status value (static storage). */
 const char* gdn_status_string(int status);

@@ -6,9 +6,16 @@ each element's error divided by max(|y_ref|, rms(y_ref)) so that elements near
 zero are measured against the output RMS; final states
 ||S - S_ref||_F / ||S_ref||_F <= 1e-3 per row; conv histories bit-exact.
 Two aggregate output checks ride along: rms(y - y_ref) / rms(y_ref) <= 5e-3
-and, reported only, max|y - y_ref| / rms(y_ref) (dominated by the bf16
+and, recorded only, max|y - y_ref| / rms(y_ref) (dominated by the bf16
 rounding of the largest outputs, whose magnitude reaches ~40x the RMS).
+
+With GDN_PARITY_LOG=<path> in the environment, every parity check appends one
+JSON line (test name, the measured errors, the bars) to that file, so the
+margins of each workload can be collected from a GPU run.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -64,6 +71,31 @@ def out_rms_err(y, y_ref):
     return float(np.sqrt(np.mean((y - y_ref) ** 2)) / max(np.sqrt(np.mean(y_ref * y_ref)), 1e-30))
 
 
+def record(name, **values):
+    """Append the measured errors of one parity check to $GDN_PARITY_LOG (if set)."""
+    path = os.environ.get("GDN_PARITY_LOG")
+    if not path:
+        return
+    line = {"check": name, **{k: float(v) if isinstance(v, (float, np.floating)) else v for k, v in values.items()},
+            "bars": {"out": OUT_TOL, "out_rms": OUT_RMS_TOL, "state": STATE_TOL}}
+    with open(path, "a") as f:
+        f.write(json.dumps(line) + "\n")
+
+
+def check_outputs(name, out, ref_out, fs=None, ref_state=None, fc=None, ref_conv=None):
+    """Assert the output, state and history bars; record the measured errors."""
+    e_out, e_rms, e_max = out_err(out, ref_out), out_rms_err(out, ref_out), out_maxabs_over_rms(out, ref_out)
+    e_st = state_err(fs, ref_state) if fs is not None else None
+    record(name, out=e_out, out_rms=e_rms, out_maxabs_over_rms=e_max, state=e_st)
+    assert e_out <= OUT_TOL, f"{name}: output error {e_out:.3e}"
+    assert e_rms <= OUT_RMS_TOL, f"{name}: output rms error {e_rms:.3e}"
+    if fs is not None:
+        assert e_st <= STATE_TOL, f"{name}: state error {e_st:.3e}"
+    if fc is not None:
+        assert conv_exact(fc, ref_conv), f"{name}: conv history not bit-exact"
+    return e_out, e_st
+
+
 def out_maxabs_over_rms(y, y_ref):
     y = _as64(y, y_ref.shape)
     if y_ref.size == 0:
@@ -97,22 +129,24 @@ def to_dev(case, device="cuda"):
 
 
 def group_case(case, kappa):
-    """The sub-problem of q/k head `kappa`: its q and k channels, the channels,
-    z, gates and parameters of its value heads, as a case with one q/k head.
-    The mixer computes each value head from exactly these inputs, so the
-    oracle on this case gives those heads' outputs and states (and the
-    history of these channels) at a fraction of the cost."""
+    """The sub-problem of q/k head(s) `kappa` (an int or a list): their q and k
+    channels, the channels, z, gates and parameters of their value heads, as a
+    case with len(kappa) q/k heads.  The mixer computes each value head from
+    exactly these inputs, so the oracle on this case gives those heads' outputs
+    and states (and the history of these channels) at a fraction of the cost."""
     d = case["dims"]
+    groups = [kappa] if isinstance(kappa, int) else list(kappa)
     G, D = d.num_v_heads // d.num_k_heads, d.head_dim
-    heads = list(range(kappa * G, (kappa + 1) * G))
-    ch = list(range(kappa * D, (kappa + 1) * D)) + list(range(d.num_k_heads * D + kappa * D,
-                                                              d.num_k_heads * D + (kappa + 1) * D))
+    heads = [kp * G + j for kp in groups for j in range(G)]
+    ch = [kp * D + c for kp in groups for c in range(D)]
+    ch += [d.num_k_heads * D + kp * D + c for kp in groups for c in range(D)]
     ch += [2 * d.num_k_heads * D + h * D + c for h in heads for c in range(D)]
     ch = torch.tensor(ch)
     zc = torch.tensor([h * D + c for h in heads for c in range(D)])
     hs = torch.tensor(heads)
     sub = dict(case)
-    sub["dims"] = synth.Dims(num_k_heads=1, num_v_heads=G, head_dim=D, conv_width=d.conv_width)
+    sub["dims"] = synth.Dims(num_k_heads=len(groups), num_v_heads=G * len(groups), head_dim=D,
+                             conv_width=d.conv_width)
     w = case["weights"]
     sub["weights"] = {"conv_w": w["conv_w"][ch], "A_log": w["A_log"][hs], "dt_bias": w["dt_bias"][hs],
                       "norm_w": w["norm_w"]}

@@ -15,8 +15,8 @@ import torch
 import gated_deltanet_mixer_gdn_b200 as gdn
 from gated_deltanet_mixer_gdn_b200 import synth
 
-from _util import (OUT_RMS_TOL, OUT_TOL, STATE_TOL, conv_exact, group_case, oracle_prefill, out_err,
-                   out_rms_err, state_err, to_dev)
+from _util import (OUT_RMS_TOL, OUT_TOL, STATE_TOL, check_outputs, conv_exact, group_case, oracle_prefill,
+                   out_err, out_rms_err, record, state_err, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,17 +28,11 @@ def _gpu():
     gdn.load_library()
 
 
-def _check_prefill(case, res, ref):
+def _check_prefill(case, res, ref, name="prefill"):
     out, fs, fc = res
-    e_out = out_err(out, ref["out"])
-    e_rms = out_rms_err(out, ref["out"])
-    e_st = state_err(fs, ref["state"])
-    assert e_out <= OUT_TOL, f"output error {e_out:.3e}"
-    assert e_rms <= OUT_RMS_TOL, f"output rms error {e_rms:.3e}"
-    assert e_st <= STATE_TOL, f"state error {e_st:.3e}"
-    assert conv_exact(fc, ref["conv"]), "conv history not bit-exact"
+    r = check_outputs(name, out, ref["out"], fs, ref["state"], fc, ref["conv"])
     assert gdn.last_device_error() == 0
-    return e_out, e_st
+    return r
 
 
 # ---------------------------------------------------------------- decode
@@ -58,28 +52,37 @@ def test_decode_small_chain():
     assert gdn.last_device_error() == 0
 
 
-def test_decode_batch_shape_sampled_heads():
-    """64 rows x 16 steps at the decode batch's shapes; oracle on 6 value heads
-    (two whole q/k groups) of every row."""
-    case = synth.decode_case(1235, rows=64, steps=16)
+def test_decode_batch_all_steps_every_group():
+    """The decode batch exactly as benchmarked (64 rows x 128 steps, seed of the decode
+    workload): every step's output, the final states and histories.  Row r is compared on
+    the 3 value heads of q/k head r % 16, so every q/k group of the 64-row persistent grid is
+    checked on 4 rows; the oracle runs each row's 128 tokens as one chain (decode = prefill
+    token by token)."""
+    case = synth.config(1)
+    steps, rows = case["qkv"].shape[0], case["qkv"].shape[1]
     w, _, st, cv = to_dev(case)
-    outs = []
-    for s in range(16):
-        outs.append(gdn.decode(*(case[k][s].cuda() for k in ("qkv", "z", "a", "b")), w, st, cv))
-    heads = (3, 9)
-    st_ref, cv_ref = case["init_state"], case["init_conv"]
-    errs = []
-    for s in range(16):
-        acts = {k: case[k][s] for k in ("qkv", "z", "a", "b")}
-        ref = oracle_prefill(case, cu=np.arange(65), init_state=st_ref, init_conv=cv_ref, acts=acts, heads=heads)
-        full_state = st_ref if isinstance(st_ref, np.ndarray) else st_ref.numpy().astype(np.float64)
-        full_state = full_state.copy()
-        full_state[:, heads[0]:heads[1]] = ref["state"]
-        errs.append(out_err(outs[s][:, heads[0] * 128:heads[1] * 128], ref["out"]))
-        st_ref, cv_ref = full_state, ref["conv"]
-    assert max(errs) <= OUT_TOL
-    assert state_err(st[:, heads[0]:heads[1]], st_ref[:, heads[0]:heads[1]]) <= STATE_TOL
-    assert conv_exact(cv, cv_ref)
+    outs = torch.empty((steps, rows, 6144), dtype=torch.bfloat16, device="cuda")
+    for s in range(steps):
+        gdn.decode(*(case[k][s].cuda() for k in ("qkv", "z", "a", "b")), w, st, cv, out=outs[s])
+    torch.cuda.synchronize()
+    outs, st, cv = outs.cpu(), st.cpu(), cv.cpu()
+    worst = {"out": 0.0, "out_rms": 0.0, "state": 0.0}
+    for kap in range(16):
+        R = [r for r in range(rows) if r % 16 == kap]
+        sub = group_case(case, kap)
+        acts = {k: sub[k][:, R].transpose(0, 1).reshape(len(R) * steps, -1) for k in ("qkv", "z", "a", "b")}
+        ref = oracle_prefill(sub, cu=np.arange(len(R) + 1) * steps, init_state=sub["init_state"][R],
+                             init_conv=sub["init_conv"][R], acts=acts)
+        y = outs[:, R].index_select(2, sub["z_channels"]).transpose(0, 1).reshape(len(R) * steps, -1)
+        e_out, e_rms = out_err(y, ref["out"]), out_rms_err(y, ref["out"])
+        e_st = state_err(st[R].index_select(1, sub["heads"]), ref["state"])
+        worst = {"out": max(worst["out"], e_out), "out_rms": max(worst["out_rms"], e_rms),
+                 "state": max(worst["state"], e_st)}
+        assert e_out <= OUT_TOL and e_rms <= OUT_RMS_TOL, f"group {kap}: output {e_out:.3e} / rms {e_rms:.3e}"
+        assert e_st <= STATE_TOL, f"group {kap}: state {e_st:.3e}"
+        assert conv_exact(cv[R].index_select(2, sub["channels"]), ref["conv"]), f"group {kap}: history"
+    record("decode batch 64x128, all groups", **worst)
+    assert gdn.last_device_error() == 0
 
 
 def test_decode_split_groups_bit_identical():
@@ -118,7 +121,7 @@ def test_prefill_small_config():
     w, acts, _, _ = to_dev(case)
     res = gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w)
     torch.cuda.synchronize()
-    _check_prefill(case, res, oracle_prefill(case))
+    _check_prefill(case, res, oracle_prefill(case), "prefill B=1 T=256 (all heads)")
 
 
 @pytest.mark.parametrize("T", [1, 2, 3, 63, 64, 65, 127, 200])
@@ -136,7 +139,7 @@ def test_prefill_long_memory_family():
     w, acts, st, cv = to_dev(case)
     res = gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w, st, cv)
     torch.cuda.synchronize()
-    _check_prefill(case, res, oracle_prefill(case))
+    _check_prefill(case, res, oracle_prefill(case), "prefill long-memory T=600")
 
 
 def test_prefill_in_place_state():
@@ -241,57 +244,57 @@ def test_chunked_prefill_8192_and_split():
     w, acts, _, _ = to_dev(case)
     res = gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w)
     torch.cuda.synchronize()
-    _check_prefill(case, res, ref)
+    _check_prefill(case, res, ref, "prefill B=1 T=8192 (all heads)")
     o1, s1, c1 = gdn.prefill(*(acts[k][:, :4096].contiguous() for k in ("qkv", "z", "a", "b")), w)
     o2, s2, c2 = gdn.prefill(*(acts[k][:, 4096:].contiguous() for k in ("qkv", "z", "a", "b")), w, s1, c1)
     torch.cuda.synchronize()
-    _check_prefill(case, (torch.cat([o1, o2], 1), s2, c2), ref)
+    _check_prefill(case, (torch.cat([o1, o2], 1), s2, c2), ref, "prefill 4096+4096 split (all heads)")
 
 
-def test_varlen_benchmark_rows_sampled_group():
-    """The 8-row varlen workload (lengths U[512,16384]); oracle on the 3 value
-    heads of q/k head 7."""
+GROUPS = (0, 5, 10, 15)
+
+
+def test_varlen_benchmark_rows_sampled_groups():
+    """The 8-row varlen workload (lengths U[512,16384]); oracle on the 12 value heads of
+    q/k heads 0, 5, 10 and 15."""
     case = synth.config(3)
-    sub = group_case(case, 7)
+    sub = group_case(case, GROUPS)
     ref = oracle_prefill(sub)
     w, acts, st, cv = to_dev(case)
     out, fs, fc = gdn.prefill_varlen(case["cu_seqlens"], acts["qkv"], acts["z"], acts["a"], acts["b"], w, st, cv)
     torch.cuda.synchronize()
     zc, hs, ch = sub["z_channels"].cuda(), sub["heads"].cuda(), sub["channels"].cuda()
-    assert out_err(out.index_select(1, zc), ref["out"]) <= OUT_TOL
-    assert out_rms_err(out.index_select(1, zc), ref["out"]) <= OUT_RMS_TOL
-    assert state_err(fs.index_select(1, hs), ref["state"]) <= STATE_TOL
-    assert conv_exact(fc.index_select(2, ch), ref["conv"])
+    check_outputs("varlen 8 rows (groups 0,5,10,15)", out.index_select(1, zc), ref["out"], fs.index_select(1, hs),
+                  ref["state"], fc.index_select(2, ch), ref["conv"])
+    assert gdn.last_device_error() == 0
 
 
-def test_long_context_two_rows_then_decode_sampled_group():
-    """Two rows of 65,536 tokens from zero state, returning final states, then
-    256 decode steps per row from those states; oracle on the 3 value heads of
-    q/k head 15 (and the history of their channels)."""
+def test_long_context_two_rows_then_decode_sampled_groups():
+    """Two rows of 65,536 tokens from zero state, returning final states, then 256 decode
+    steps per row from those states; oracle on the 12 value heads of q/k heads 0, 5, 10 and
+    15 (and the history of their channels).  The oracle continues from its own states."""
     case = synth.config(4)
-    sub = group_case(case, 15)
+    sub = group_case(case, GROUPS)
     w, acts, _, _ = to_dev(case)
     out, fs, fc = gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w)
     torch.cuda.synchronize()
     ref = oracle_prefill(sub)
     zc, hs, ch = sub["z_channels"].cuda(), sub["heads"].cuda(), sub["channels"].cuda()
     o2 = out.reshape(2 * 65536, -1).index_select(1, zc)
-    assert out_err(o2, ref["out"]) <= OUT_TOL
-    assert out_rms_err(o2, ref["out"]) <= OUT_RMS_TOL
-    assert state_err(fs.index_select(1, hs), ref["state"]) <= STATE_TOL
-    assert conv_exact(fc.index_select(2, ch), ref["conv"])
-    # 256 decode steps from the GPU's final state; the oracle continues from its own
+    check_outputs("long context 2x65536 (groups 0,5,10,15)", o2, ref["out"], fs.index_select(1, hs), ref["state"],
+                  fc.index_select(2, ch), ref["conv"])
+    # 256 decode steps from the GPU's final state; the oracle runs them as one 256-token chain per row
     dec = case["decode"]
-    outs = [gdn.decode(*(dec[k][s].cuda() for k in ("qkv", "z", "a", "b")), w, fs, fc) for s in range(256)]
+    steps = dec["qkv"].shape[0]
+    outs = torch.empty((steps, 2, 6144), dtype=torch.bfloat16, device="cuda")
+    for s in range(steps):
+        gdn.decode(*(dec[k][s].cuda() for k in ("qkv", "z", "a", "b")), w, fs, fc, out=outs[s])
     torch.cuda.synchronize()
-    st_ref, cv_ref = ref["state"], ref["conv"]
-    errs = []
-    for s in range(256):
-        step = {"qkv": dec["qkv"][s].index_select(-1, sub["channels"]), "z": dec["z"][s].index_select(-1, sub["z_channels"]),
-                "a": dec["a"][s].index_select(-1, sub["heads"]), "b": dec["b"][s].index_select(-1, sub["heads"])}
-        r = oracle_prefill(sub, cu=np.arange(3), init_state=st_ref, init_conv=cv_ref, acts=step)
-        errs.append(out_err(outs[s].index_select(1, zc), r["out"]))
-        st_ref, cv_ref = r["state"], r["conv"]
-    assert max(errs) <= OUT_TOL
-    assert state_err(fs.index_select(1, hs), st_ref) <= STATE_TOL
-    assert conv_exact(fc.index_select(2, ch), cv_ref)
+    idx = {"qkv": sub["channels"], "z": sub["z_channels"], "a": sub["heads"], "b": sub["heads"]}
+    chain = {k: dec[k].index_select(-1, idx[k]).transpose(0, 1).reshape(2 * steps, -1) for k in idx}
+    r = oracle_prefill(sub, cu=np.array([0, steps, 2 * steps]), init_state=ref["state"], init_conv=ref["conv"],
+                       acts=chain)
+    y = outs.index_select(2, zc).transpose(0, 1).reshape(2 * steps, -1)
+    check_outputs("decode 256 steps after long context (groups 0,5,10,15)", y, r["out"], fs.index_select(1, hs),
+                  r["state"], fc.index_select(2, ch), r["conv"])
+    assert gdn.last_device_error() == 0

@@ -3,8 +3,8 @@
 must not take an allocation's implicit device synchronisation).  Its scratch is
 a fixed device array inside the library, so the test checks that two calls in
 a row, with different inputs, give the same results as gdn_prefill with a
-caller-allocated workspace, and that a request beyond the fixed capacity is
-refused.  The file sorts last so that a run stopping at the first failure has
+caller-allocated workspace, that each call leaves the device's free memory
+unchanged, and that a request beyond the fixed capacity is refused.  The file sorts last so that a run stopping at the first failure has
 already run every other test; it also passes alone in a fresh process.
 """
 import ctypes
@@ -59,9 +59,14 @@ def test_noalloc_two_calls_match_workspace_entry_point(dev):
         out = torch.empty_like(ref_out)
         fs = torch.empty_like(ref_st)
         fc = torch.empty_like(ref_cv)
+        # the library is loaded (the reference call above ran the same kernels), so the call
+        # itself must leave the device's free memory exactly as it was
+        torch.cuda.synchronize(dev)
+        free_before = torch.cuda.mem_get_info(dev)[0]
         status = _call_noalloc(fn, B, T, w, acts, st, cv, out, fs, fc)
         assert status == 0, gdn.status_string(status)
         torch.cuda.synchronize(dev)
+        assert torch.cuda.mem_get_info(dev)[0] == free_before, f"call {call} changed the free device memory"
         ref64 = ref_out.double().cpu().numpy()
         assert out_err(out, ref64) <= OUT_TOL, f"call {call}"
         assert out_rms_err(out, ref64) <= OUT_RMS_TOL, f"call {call}"
