@@ -480,6 +480,40 @@ def bench_hidden(args, local, T=8192):
             "l2": "flushed (256 MiB write) before each timed call"}
 
 
+def bench_prefill_out(args, local, T=8192):
+    """The mixer followed by out_proj (hidden 5120) for one row of T tokens: gdn_prefill_out (each
+    segment's projection overlapped with the later segments' recurrence) against gdn_prefill
+    followed by gdn_out_proj (bit-identical results)."""
+    import gated_deltanet_mixer_gdn_b200 as gdn
+    dev = torch.device("cuda", local)
+    case = synth.config(2) if T == 8192 else synth.dense_case(1236, 1, T)
+    w = gdn.weights_to(case["weights"], dev)
+    acts = {k: case[k].to(dev) for k in ("qkv", "z", "a", "b")}
+    g = torch.Generator(device=dev).manual_seed(13)
+    w_out = (torch.randn((5120, 6144), generator=g, device=dev) * 6144 ** -0.5).to(torch.bfloat16)
+    out = torch.empty((1, T, 5120), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((1, T, 6144), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
+    fc = torch.empty((1, 3, 10240), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    warm, reps = max(3, args.warmup), max(5, args.steps)
+    tf, nf = _time_prefill(lambda: gdn.prefill_out(acts["qkv"], acts["z"], acts["a"], acts["b"], w, w_out, out=out,
+                                                   final_state=fs, final_conv=fc), dev, stream, warm, reps)
+
+    def pair():
+        gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w, out=y, final_state=fs, final_conv=fc)
+        gdn.out_proj(y[0], w_out, out=out[0])
+
+    tu, nu = _time_prefill(pair, dev, stream, warm, reps)
+    segs = gdn.prefill_schedule(1, T)[0]
+    return {"workload": f"prefill B=1 T={T} then out_proj [{T},6144] x [5120,6144]^T, zero initial state",
+            "fused": {"value": T / tf, "unit": "tokens/s", "ms": tf * 1000.0,
+                      "gpu_launches": (prefill_launches(1, T) + segs) * nf},
+            "unfused": {"value": T / tu, "unit": "tokens/s", "ms": tu * 1000.0,
+                        "gpu_launches": (prefill_launches(1, T) + 1) * nu},
+            "l2": "flushed (256 MiB write) before each timed call"}
+
+
 def _time_prefill(call, dev, stream, warmup, reps):
     """Median seconds of `call` (CUDA events on `stream`), L2 flushed before each timed call."""
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > L2, written between iterations
@@ -540,7 +574,8 @@ def prefill_cpu_baseline(case, rows, tokens, what):
     oracle.build()
     dt, n = oracle_prefill_sample(case, rows, tokens)
     return {"value": n / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"{what}: the first {tokens} tokens of {len(rows)} row(s), all 48 heads, f64 ({dt:.1f} s)"}
+            "sample": f"{what}: {n} tokens ({len(rows)} row(s), up to {tokens} tokens each), all 48 heads, f64 "
+                      f"({dt:.1f} s)"}
 
 
 def prefill_e2e(args, dev, case, w, seg=2048):
@@ -631,7 +666,7 @@ def bench_prefill(args, world, rank, local, T, full=True):
     if not full:
         return res
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = prefill_cpu_baseline(pcase, [0], 2048, f"prefill B=1 T={T}")
+        res["cpu_baseline"] = prefill_cpu_baseline(pcase, [0], T, f"prefill B=1 T={T}")
     configs = {}
     # 4096 + 4096: the second half continues from the state and history the first half left
     h = T // 2
@@ -680,7 +715,7 @@ def bench_prefill(args, world, rank, local, T, full=True):
                                           "U[512,16384]), random initial state and history",
                                           prefill_launches_varlen() * n2, peaks)
         if world == 1 and not args.no_cpu_baseline:
-            configs["varlen8"]["cpu_baseline"] = prefill_cpu_baseline(vcase, list(range(8)), 512,
+            configs["varlen8"]["cpu_baseline"] = prefill_cpu_baseline(vcase, list(range(8)), 16384,
                                                                       "varlen prefill 8 rows")
         del av, st0, cv0, vout, vst, vcv
         configs["long2"] = bench_long_context(args, local, lambda *a: prefill_line(*a, peaks))
@@ -707,7 +742,7 @@ def bench_long_context(args, local, line):
     res = line(B * T, t, f"long-context prefill B={B} T={T}, zero initial state, final states returned",
                prefill_launches(B, T) * n)
     if not args.no_cpu_baseline:
-        res["cpu_baseline"] = prefill_cpu_baseline(case, [0, 1], 1024, f"long-context prefill B={B} T={T}")
+        res["cpu_baseline"] = prefill_cpu_baseline(case, [0, 1], T, f"long-context prefill B={B} T={T}")
     # 256 decode steps per row from the prefill's states (2 rows: launch-latency bound, reported)
     steps = case["decode"]["qkv"].shape[0]
     dq = {k: case["decode"][k].to(dev) for k in ("qkv", "z", "a", "b")}
@@ -780,8 +815,10 @@ def main():
         multi = bench_decode_multi(args, local)
         proj = bench_projections(args, local)
         hid = bench_hidden(args, local)
+        pout = bench_prefill_out(args, local)
         if rank == 0:
             line["prefill"] = pre
+            line["prefill_out_proj"] = pout
             line["decode_multi"] = multi
             line["projections"] = proj
             line["prefill_from_hidden"] = hid

@@ -25,11 +25,13 @@ from .synth import Dims, MODEL
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
-EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_schedule", "gdn_prefill_varlen_workspace_size",
+EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_out_workspace_size", "gdn_prefill_out",
+           "gdn_prefill_schedule", "gdn_prefill_varlen_workspace_size",
            "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
            "gdn_in_proj", "gdn_out_proj", "gdn_prefill_hidden_workspace_size", "gdn_prefill_hidden",
            "gdn_prefill_hidden_varlen_workspace_size", "gdn_prefill_hidden_varlen",
-           "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_set_decode_wait_limit", "gdn_status_string",
+           "gdn_prefill_noalloc", "gdn_last_device_error", "gdn_set_decode_wait_limit", "gdn_test_decode_stop_copies_at",
+           "gdn_status_string",
            "gdn_version")
 
 GDN_OK = 0
@@ -69,6 +71,10 @@ def load_library() -> ctypes.CDLL:
         L.gdn_prefill_varlen_workspace_size.restype = sz
         L.gdn_prefill_varlen_workspace_size.argtypes = [dp, i32, i32]
         L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_prefill_out_workspace_size.restype = sz
+        L.gdn_prefill_out_workspace_size.argtypes = [dp, i32, i32]
+        L.gdn_prefill_out.restype = ctypes.c_int
+        L.gdn_prefill_out.argtypes = [dp, wp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_prefill_schedule.restype = ctypes.c_int
         L.gdn_prefill_schedule.argtypes = [dp, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
         L.gdn_prefill.argtypes = [dp, wp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -100,6 +106,8 @@ def load_library() -> ctypes.CDLL:
         L.gdn_last_device_error.argtypes = []
         L.gdn_set_decode_wait_limit.restype = ctypes.c_int
         L.gdn_set_decode_wait_limit.argtypes = [ctypes.c_uint64]
+        L.gdn_test_decode_stop_copies_at.restype = ctypes.c_int
+        L.gdn_test_decode_stop_copies_at.argtypes = [ctypes.c_int32]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_version.restype = ctypes.c_int
@@ -189,6 +197,44 @@ def prefill(qkv, z, a, b, weights, init_state=None, init_conv=None, *, out=None,
                        _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(init_state), _ptr(init_conv),
                        _ptr(out), _ptr(final_state), _ptr(final_conv), _ptr(ws), ws_bytes, _stream(dev))
     _check(st, "gdn_prefill")
+    return out, final_state, final_conv
+
+
+def prefill_out(qkv, z, a, b, weights, w_out, init_state=None, init_conv=None, *, out=None, final_state=None,
+                final_conv=None, dims: Dims = MODEL, in_place: bool = False):
+    """Dense prefill followed by out_proj in one call: qkv [B,T,C], z [B,T,Vh*D], a/b [B,T,Vh] bf16,
+    w_out bf16 [hidden, Vh*D].  Returns (out bf16 [B,T,hidden], final_state, final_conv); the same
+    bits as prefill followed by out_proj."""
+    dev = _device_of(qkv)
+    L = load_library()
+    B, T = int(qkv.shape[0]), int(qkv.shape[1])
+    C, VD, Vh, D, Wm = dims.conv_channels, dims.value_width, dims.num_v_heads, dims.head_dim, dims.conv_width - 1
+    for t, dt, nm in ((qkv, torch.bfloat16, "qkv"), (z, torch.bfloat16, "z"), (a, torch.bfloat16, "a"),
+                      (b, torch.bfloat16, "b"), (w_out, torch.bfloat16, "w_out")):
+        _need(t, dt, nm, dev)
+    hidden = int(w_out.shape[0])
+    if tuple(qkv.shape) != (B, T, C) or tuple(z.shape) != (B, T, VD) or tuple(a.shape) != (B, T, Vh) \
+            or tuple(b.shape) != (B, T, Vh) or tuple(w_out.shape) != (hidden, VD):
+        raise ValueError("prefill_out: shape mismatch")
+    if init_state is not None:
+        _need(init_state, torch.float32, "init_state", dev)
+    if init_conv is not None:
+        _need(init_conv, torch.float32, "init_conv", dev)
+    if out is None:
+        out = torch.empty((B, T, hidden), dtype=torch.bfloat16, device=dev)
+    if final_state is None:
+        final_state = init_state if (in_place and init_state is not None) else \
+            torch.empty((B, Vh, D, D), dtype=torch.float32, device=dev)
+    if final_conv is None:
+        final_conv = init_conv if (in_place and init_conv is not None) else \
+            torch.empty((B, Wm, C), dtype=torch.float32, device=dev)
+    dc = _dims_c(dims)
+    ws_bytes = L.gdn_prefill_out_workspace_size(ctypes.byref(dc), B, T)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    st = L.gdn_prefill_out(ctypes.byref(dc), ctypes.byref(_weights_c(weights, dev)), B, T, hidden,
+                           _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), _ptr(init_state), _ptr(init_conv), _ptr(w_out),
+                           _ptr(out), _ptr(final_state), _ptr(final_conv), _ptr(ws), ws_bytes, _stream(dev))
+    _check(st, "gdn_prefill_out")
     return out, final_state, final_conv
 
 
@@ -481,5 +527,5 @@ def weights_to(weights: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tens
     return {k: v.to(device).contiguous() for k, v in weights.items()}
 
 
-__all__ = ["prefill", "prefill_schedule", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_hidden_varlen", "prefill_varlen_slots", "last_device_error", "set_decode_wait_limit", "status_string", "load_library",
+__all__ = ["prefill", "prefill_out", "prefill_schedule", "prefill_varlen", "decode", "decode_multi", "decode_slots", "in_proj", "out_proj", "prefill_hidden", "prefill_hidden_varlen", "prefill_varlen_slots", "last_device_error", "set_decode_wait_limit", "status_string", "load_library",
            "GdnError", "Dims", "MODEL", "LIB_PATH", "EXPORTS", "weights_to"]

@@ -122,7 +122,8 @@ struct SideStreams {
     bool ready = false;
     cudaStream_t prod = nullptr, chain = nullptr;
     cudaEvent_t fork = nullptr, prod_done = nullptr, chain_done = nullptr;
-    cudaEvent_t seg[kMaxSegments] = {};
+    cudaEvent_t seg[kMaxSegments] = {};   // WY records of a segment written (prod -> chain)
+    cudaEvent_t rec[kMaxSegments] = {};   // recurrence of a segment done (chain -> prod)
 };
 std::mutex g_side_mu;
 SideStreams g_side[kMaxDevices];
@@ -140,6 +141,8 @@ int side_streams(int dev, SideStreams** out) {
         for (cudaEvent_t* e : evs)
             if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
         for (auto& e : st.seg)
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
+        for (auto& e : st.rec)
             if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
         st.ready = true;
     }
@@ -173,6 +176,28 @@ struct FusedLoad {
     uint16_t* z;           // bf16 [total][Vh*128]
     float* conv_last;      // f32 [N][3][C]
 };
+
+// out_proj after the mixer (gdn_prefill_out): out[t] = y[t] w_out^T for every token t,
+// y being the mixer's gated-norm output.
+struct OutProjTail {
+    const uint16_t* w_out;  // bf16 [hidden][Vh*128]
+    int hidden;
+    uint16_t* out;          // bf16 [tokens][hidden]
+};
+
+int gemm_launch(const uint16_t* A, const uint16_t* W, struct GemmParams gp, cudaStream_t stream);
+
+// out_proj of tokens [t0, t1) of the call (rows of y and of out).
+int out_proj_range(const OutProjTail& op, const uint16_t* y, int VD, int64_t t0, int64_t t1, cudaStream_t st) {
+    if (t1 <= t0) return GDN_OK;
+    GemmParams gp{};
+    gp.M = (int)(t1 - t0);
+    gp.N = op.hidden;
+    gp.K = VD;
+    gp.nseg = 1;
+    gp.seg[0] = GemmSegment{0, op.hidden, op.out + t0 * op.hidden};
+    return gemm_launch(y + t0 * VD, op.w_out, gp, st);
+}
 
 // Segment plan of the overlapped dense prefill.  The load stage runs over all
 // tokens first; segment 0's WY records run on every SM; after that, the recurrence
@@ -414,7 +439,8 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                  int32_t total, int64_t nchunks, int64_t nchunks_planned, const uint16_t* qkv, const uint16_t* z,
                  const uint16_t* a, const uint16_t* b, const float* init_state, const float* init_conv, uint16_t* out,
                  float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-                 bool may_overlap, const int32_t* slots_dev = nullptr, const FusedLoad* fused = nullptr) {
+                 bool may_overlap, const int32_t* slots_dev = nullptr, const FusedLoad* fused = nullptr,
+                 const OutProjTail* op = nullptr) {
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
     const int C = (2 * Kh + Vh) * 128;
     const size_t state_bytes = (size_t)N * Vh * 128 * 128 * 4;
@@ -524,6 +550,17 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
             if ((st = P.recurrence(cs[k], k + 1 < S ? cs[k + 1] : -1, k == 0 ? init_state : final_state, final_state,
                                    ss->chain)) != GDN_OK)
                 return st;
+            if (op != nullptr && cudaEventRecord(ss->rec[k], ss->chain) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        // out_proj of each segment's tokens, behind every WY launch on the low-priority stream,
+        // as soon as that segment's recurrence has written them
+        for (int k = 0; op != nullptr && k < S; ++k) {
+            if (cudaStreamWaitEvent(ss->prod, ss->rec[k], 0) != cudaSuccess) return GDN_ERR_CUDA;
+            const int64_t a0 = (int64_t)cs[k] * 64, a1 = k + 1 < S ? (int64_t)cs[k + 1] * 64 : uniform_T;
+            for (int n = 0; n < N; ++n)
+                if ((st = out_proj_range(*op, out, Vh * 128, (int64_t)n * uniform_T + a0,
+                                         (int64_t)n * uniform_T + (a1 < uniform_T ? a1 : uniform_T), ss->prod)) != GDN_OK)
+                    return st;
         }
         if (cudaEventRecord(ss->prod_done, ss->prod) != cudaSuccess ||
             cudaEventRecord(ss->chain_done, ss->chain) != cudaSuccess ||
@@ -542,7 +579,8 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     if ((st = P.wy_records(nchunks, 0, 0, nsm, stream)) != GDN_OK) return st;  // 4. WY records, all chunks
-    return P.recurrence(0, -1, init_state, final_state, stream);              // 5. recurrence + gated norm
+    if ((st = P.recurrence(0, -1, init_state, final_state, stream)) != GDN_OK) return st;  // 5. recurrence + gated norm
+    return op != nullptr ? out_proj_range(*op, out, Vh * 128, 0, total, stream) : GDN_OK;  // 6. out_proj
 }
 
 int check_io(int32_t total, const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
@@ -916,6 +954,40 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
     return plan_workspace(dims, total, B, (int64_t)B * ((T + 63) / 64)).bytes;
 }
 
+size_t gdn_prefill_out_workspace_size(const gdn_dims* dims, int32_t B, int32_t T) {
+    if (check_dims(dims) != GDN_OK || B < 0 || T < 0) return 0;
+    const int64_t total = (int64_t)B * T;
+    if (total > INT32_MAX) return 0;
+    return plan_workspace(dims, total, B, (int64_t)B * ((T + 63) / 64)).bytes +
+           align_up((size_t)total * dims->num_v_heads * 128 * 2);
+}
+
+int gdn_prefill_out(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, int32_t hidden,
+                    const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                    const float* init_state, const float* init_conv, const uint16_t* w_out, uint16_t* out,
+                    float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, void* stream) {
+    int st = check_dims(dims);
+    if (st != GDN_OK) return st;
+    if ((st = check_weights(w)) != GDN_OK) return st;
+    if (B < 0 || T < 0 || B > 65535 || hidden <= 0) return GDN_ERR_INVALID_ARG;
+    if (hidden % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    const int64_t total = (int64_t)B * T;
+    if (total > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if ((st = check_io((int32_t)total, qkv, z, a, b, out, init_state, init_conv, final_state, final_conv)) != GDN_OK)
+        return st;
+    if (total > 0 && (w_out == nullptr || !aligned16(w_out))) return GDN_ERR_INVALID_ARG;
+    if ((st = check_device()) != GDN_OK) return st;
+    const int64_t nch = (int64_t)B * ((T + 63) / 64);
+    const size_t ws_mixer = plan_workspace(dims, total, B, nch).bytes;
+    if (total > 0 && (workspace == nullptr || workspace_bytes < gdn_prefill_out_workspace_size(dims, B, T)))
+        return GDN_ERR_WORKSPACE;
+    uint16_t* y = total > 0 ? reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + ws_mixer) : nullptr;
+    const OutProjTail op{w_out, hidden, out};
+    return prefill_impl(dims, w, B, nullptr, T, (int32_t)total, nch, nch, qkv, z, a, b, init_state, init_conv, y,
+                        final_state, final_conv, workspace, ws_mixer, static_cast<cudaStream_t>(stream), true, nullptr,
+                        nullptr, &op);
+}
+
 size_t gdn_prefill_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T) {
     if (check_dims(dims) != GDN_OK || N < 0 || total_T < 0) return 0;
     return plan_workspace(dims, total_T, N, chunk_bound(N, total_T)).bytes;
@@ -1054,6 +1126,14 @@ int gdn_set_decode_wait_limit(uint64_t ns) {
     if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
     const unsigned long long v = ns;
     if (cudaMemcpyToSymbol(gdn::g_decode_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return GDN_ERR_CUDA;
+    return cudaDeviceSynchronize() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_test_decode_stop_copies_at(int32_t unit) {
+    if (unit < -1) return GDN_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    const int v = unit;
+    if (cudaMemcpyToSymbol(gdn::g_decode_stop_copies_at, &v, sizeof(v)) != cudaSuccess) return GDN_ERR_CUDA;
     return cudaDeviceSynchronize() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -34,6 +34,11 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // stops issuing copies, drains the ones in flight and returns.
 __device__ unsigned long long g_decode_wait_limit_ns = kWaitLimitNs;
 
+// Test hook of the decode kernels (gdn_test_decode_stop_copies_at): when >= 0, each
+// CTA's copy producer issues no state copy from this unit of its work on, so the
+// consumers' wait for that unit runs out.  -1 (the default): off.
+__device__ int g_decode_stop_copies_at = -1;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
             // for a release runs out (the consumers stopped releasing after a wait of their own
             // ran out), no further copy is issued.
             const int lead = nst < units_per_item - 1 ? nst : units_per_item - 1;
+            const int stop_at = g_decode_stop_copies_at;  // test hook, -1 normally
             int issued = 0, issued_aux = 0;
             if (nmine > 0) {
                 aux_load(0);
@@ -240,6 +241,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                     issued_aux = m + 2;
                 }
                 const int st = u % nst;
+                if (u == stop_at) break;
                 if (u >= nst && !bounded_wait(&empty[st], ((u / nst) - 1) & 1, broken)) break;
                 mbar_arrive_expect_tx(&full[st], kTileBytes);
                 bulk_load(smem + st * kTileBytes, unit_ptr(u), kTileBytes, &full[st]);

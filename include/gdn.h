@@ -107,6 +107,26 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Dense prefill followed by the layer's output projection, in one call: the
+ * mixer's gated-norm output y (bf16, kept in the workspace) times out_proj
+ * (Qwen/Qwen3.8-27B architecture page, module tree: out_proj 5120x6144):
+ *   out[b][t][:] = y[b][t][:] w_out^T      w_out bf16 [hidden][Vh*D], out bf16 [B][T][hidden]
+ * Arguments and results otherwise as gdn_prefill (hidden % 8 == 0, else
+ * GDN_ERR_UNSUPPORTED).  Workspace: gdn_prefill_out_workspace_size(dims, B, T)
+ * bytes (the prefill's workspace plus y).  When the prefill overlaps its
+ * kernels (see gdn_prefill_schedule), the projection of each recurrence
+ * segment's tokens starts on the internal low-priority stream as soon as that
+ * segment's outputs are written, while the later segments' recurrence runs;
+ * otherwise it runs after the recurrence on `stream`.  The result is the same,
+ * bit for bit, as gdn_prefill followed by gdn_out_proj.
+ */
+size_t gdn_prefill_out_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
+int gdn_prefill_out(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, int32_t hidden,
+                    const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
+                    const float* init_state, const float* init_conv, const uint16_t* w_out, uint16_t* out,
+                    float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Schedule of a dense prefill of B rows x T tokens that returns its final
  * state, on the current device: gdn_prefill (from_hidden = 0) or
  * gdn_prefill_hidden (from_hidden = 1).  *segments = S, the number of
@@ -313,12 +333,19 @@ int gdn_last_device_error(void);
  * GDN_DECODE_WAIT_LIMIT_DEFAULT_NS (2 s).  A wait that runs out sets the error
  * word above; the kernel then stops issuing copies, waits (up to 2 s) for the
  * copies it already issued, and returns with its outputs undefined, leaving the
- * context usable.  A small bound makes waits run out on purpose (the library's
- * test of that path uses 0); restore the default afterwards.  The kernels that
- * hold tensor memory (prefill, projections) keep a fixed 2 s bound.
- * Synchronises the device; not for use during stream capture. */
+ * context usable.  The kernels that hold tensor memory (prefill, projections)
+ * keep a fixed 2 s bound.  Synchronises the device; not for use during stream
+ * capture. */
 #define GDN_DECODE_WAIT_LIMIT_DEFAULT_NS 2000000000ull
 int gdn_set_decode_wait_limit(uint64_t ns);
+
+/* Test hook of the failure path above.  unit >= 0: from then on, in every
+ * decode launch on the current device, each CTA's copy producer issues no
+ * state copy from the unit-th half-tile of its work onward, so the consumers'
+ * wait for that half-tile runs out (after the bound set above) with no copy
+ * in flight; -1 (the default) switches it off.  Used with a short bound by the
+ * library's tests; never needed otherwise.  Synchronises the device. */
+int gdn_test_decode_stop_copies_at(int32_t unit);
 
 /* Human-readable text of a gdn_status value (static storage). */
 const char* gdn_status_string(int status);

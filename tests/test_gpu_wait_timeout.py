@@ -2,8 +2,10 @@
 hanging the GPU.
 
 Every wait inside the decode kernels polls its mbarrier against a wall-clock
-bound.  With that bound set to 0, waits that are not already satisfied run out
-at once: the kernel must record the timeout in the device error word, stop
+bound.  The test shortens that bound to 1 ms and switches on the library's test
+hook that makes each CTA's copy producer stop issuing state copies from its
+second half-tile on, so the consumers' wait for that half-tile can only run
+out.  The kernel must record the timeout in the device error word, stop
 releasing and refilling its shared-memory buffers, wait for the bulk copies it
 already issued, and return.  The test then checks that the error is reported
 (and cleared by reading), and that the same context still computes a correct
@@ -40,12 +42,14 @@ def test_decode_wait_runs_out_reports_and_returns(rows):
     acts = [case[k][0].cuda() for k in ("qkv", "z", "a", "b")]
     assert gdn.last_device_error() == 0
     st, cv = st0.clone(), cv0.clone()
-    gdn.set_decode_wait_limit(0)
+    lib = gdn.load_library()
+    gdn.set_decode_wait_limit(1_000_000)
+    assert lib.gdn_test_decode_stop_copies_at(1) == 0
     try:
-        for _ in range(3):
-            gdn.decode(*acts, w, st, cv)
+        gdn.decode(*acts, w, st, cv)
         torch.cuda.synchronize()
     finally:
+        assert lib.gdn_test_decode_stop_copies_at(-1) == 0
         gdn.set_decode_wait_limit()
     assert gdn.last_device_error() == GDN_DEVERR_TIMEOUT_COPY
     assert gdn.last_device_error() == 0  # cleared by the read
