@@ -718,7 +718,8 @@ def bench_prefill(args, world, rank, local, T, full=True):
             configs["varlen8"]["cpu_baseline"] = prefill_cpu_baseline(vcase, list(range(8)), 16384,
                                                                       "varlen prefill 8 rows")
         del av, st0, cv0, vout, vst, vcv
-        configs["long2"] = bench_long_context(args, local, lambda *a: prefill_line(*a, peaks))
+        if not args.no_long:
+            configs["long2"] = bench_long_context(args, local, lambda *a: prefill_line(*a, peaks))
     res["configs"] = configs
     return res
 
@@ -791,6 +792,8 @@ def main():
                     help="decode: the 64-row decode batch (default line); prefill: only the chunked prefill; "
                          "hidden: only the prefill from hidden states (fused in_proj + load stage)")
     ap.add_argument("--prefill-T", type=int, default=PREFILL_T, help="tokens of the prefill measurement")
+    ap.add_argument("--no-long", action="store_true",
+                    help="with --workload prefill: skip the 2 x 65,536-token leg")
     ap.add_argument("--prefill-only", action="store_true",
                     help="with --workload prefill: only the one-row prefill (a small case for profiling)")
     args = ap.parse_args()
