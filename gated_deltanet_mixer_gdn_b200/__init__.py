@@ -23,7 +23,8 @@ import torch
 from .synth import Dims, MODEL
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
+# GDN_B200_LIBRARY selects another build of the library (the debug build, libgdn_b200_debug.so)
+LIB_PATH = os.environ.get("GDN_B200_LIBRARY") or os.path.join(_PKG, "libgdn_b200.so")
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_out_workspace_size", "gdn_prefill_out",
            "gdn_prefill_schedule", "gdn_prefill_varlen_workspace_size",

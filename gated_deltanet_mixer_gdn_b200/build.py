@@ -1,4 +1,6 @@
-"""Build libgdn_b200.so (sm_100a) in-tree with nvcc."""
+"""Build libgdn_b200.so (sm_100a) in-tree with nvcc, and its debug variant
+libgdn_b200_debug.so (-DGDN_DEBUG: the kernels check the indices of their
+global-memory accesses and record a failed check in the device error word)."""
 from __future__ import annotations
 
 import glob
@@ -8,6 +10,7 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libgdn_b200.so")
+DEBUG_LIB = os.path.join(PKG, "libgdn_b200_debug.so")
 SOURCES = sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu")) + glob.glob(os.path.join(PKG, "csrc", "*.cuh"))
                  + [os.path.join(ROOT, "include", "gdn.h")])
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -21,24 +24,26 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in SOURCES)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, os.path.join(PKG, "csrc", "api.cu"), "-o", tmp]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DGDN_DEBUG"] if debug else []), os.path.join(PKG, "csrc", "api.cu"), "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     print(build(force=True, verbose=True))
+    print(build(force=True, debug=True))

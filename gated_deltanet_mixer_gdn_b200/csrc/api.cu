@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <climits>
 #include <cstdint>
@@ -22,6 +23,15 @@
 namespace {
 
 using namespace gdn;
+
+// An NVTX range over one ABI call (named after the entry point), so host timelines of a
+// profiler show each call and the launches it enqueued; free when no tool is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
@@ -298,6 +308,8 @@ struct PrefillPlan {
     int* chunk_base;
     int* order;  // recurrence row order (packed rows), or nullptr
     uint8_t* rec;
+    int rec_chunks;  // chunks the record array holds
+    int state_rows;  // rows of the state / history arrays (the pool's, with slots)
     CUtensorMap mK, mQ, mKl, mQl, mV, mZ, mO;
 
     int prep(int tok_begin, int tok_end, cudaStream_t st) const {
@@ -378,6 +390,7 @@ struct PrefillPlan {
         ConvOutParams cp{};
         cp.C = C;
         cp.N = N;
+        cp.total = total;
         cp.seq = seq;
         cp.qkv = qkv;
         cp.init_conv = init_conv;
@@ -402,6 +415,7 @@ struct PrefillPlan {
         wp.Gs = Gs;
         wp.Bs = Bs;
         wp.rec = rec;
+        wp.rec_chunks = rec_chunks;
         int rc = smem_optin(reinterpret_cast<const void*>(gdn_wy_kernel), wy::SMEM_BYTES);
         if (rc != GDN_OK) return rc;
         const int ratio = Vh / Kh;
@@ -427,6 +441,8 @@ struct PrefillPlan {
         cp.c0 = c0;
         cp.c1 = c1;
         cp.slots = slots;
+        cp.rec_chunks = rec_chunks;
+        cp.state_rows = state_rows;
         int rc = smem_optin(reinterpret_cast<const void*>(gdn_chunk_kernel), chunk::SMEM_BYTES);
         if (rc != GDN_OK) return rc;
         dim3 grid(Vh, N);
@@ -440,7 +456,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                  const uint16_t* a, const uint16_t* b, const float* init_state, const float* init_conv, uint16_t* out,
                  float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, cudaStream_t stream,
                  bool may_overlap, const int32_t* slots_dev = nullptr, const FusedLoad* fused = nullptr,
-                 const OutProjTail* op = nullptr) {
+                 const OutProjTail* op = nullptr, int32_t pool_rows = 0) {
     const int Kh = d->num_k_heads, Vh = d->num_v_heads;
     const int C = (2 * Kh + Vh) * 128;
     const size_t state_bytes = (size_t)N * Vh * 128 * 128 * 4;
@@ -502,6 +518,8 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     P.chunk_base = cu_dev ? reinterpret_cast<int*>(wsb + ws.off_cb) : nullptr;
     P.order = cu_dev ? P.chunk_base + N + 1 : nullptr;
     P.rec = wsb + ws.off_rec;
+    P.rec_chunks = (int)nchunks_planned;
+    P.state_rows = slots_dev != nullptr ? pool_rows : N;
     if (!make_map(&P.mK, P.Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&P.mKl, P.Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
@@ -675,7 +693,7 @@ int check_slots(const int32_t* slots_host, int32_t rows, int32_t pool_rows) {
 // The decode launch: rows batch rows, state / history rows through slots (or nullptr).
 int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const uint16_t* qkv, const uint16_t* z,
                 const uint16_t* a, const uint16_t* b, float* state, float* conv, uint16_t* out, const int32_t* slots,
-                int32_t ntok, void* stream) {
+                int32_t ntok, void* stream, int32_t pool_rows) {
     int st = GDN_OK;
     if (!state || !conv || !aligned16(state) || !aligned16(conv)) return GDN_ERR_INVALID_ARG;
     if ((st = check_io(rows, qkv, z, a, b, out, nullptr, nullptr, nullptr, nullptr)) != GDN_OK) return st;
@@ -697,6 +715,7 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
     p.conv = conv;
     p.out = out;
     p.slots = slots;
+    p.pool_rows = pool_rows;
     p.ntok = ntok;
     const void* kernels[4] = {reinterpret_cast<const void*>(gdn_decode_kernel<1, false>),
                               reinterpret_cast<const void*>(gdn_decode_kernel<dec::kMaxTokens, false>),
@@ -844,6 +863,7 @@ extern "C" {
 
 int gdn_in_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t* x, const uint16_t* w_in,
                 uint16_t* qkv, uint16_t* z, uint16_t* b, uint16_t* a, void* stream) {
+    NvtxRange nvtx_range("gdn_in_proj");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if (T < 0 || hidden <= 0) return GDN_ERR_INVALID_ARG;
@@ -864,6 +884,7 @@ int gdn_in_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t*
 
 int gdn_out_proj(const gdn_dims* dims, int32_t T, int32_t hidden, const uint16_t* y, const uint16_t* w_out,
                  uint16_t* out, void* stream) {
+    NvtxRange nvtx_range("gdn_out_proj");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if (T < 0 || hidden <= 0) return GDN_ERR_INVALID_ARG;
@@ -889,6 +910,7 @@ int gdn_prefill_hidden(const gdn_dims* dims, const gdn_weights* w, int32_t B, in
                        const uint16_t* x, const uint16_t* w_in, const float* init_state, const float* init_conv,
                        uint16_t* out, float* final_state, float* final_conv, void* workspace, size_t workspace_bytes,
                        void* stream) {
+    NvtxRange nvtx_range("gdn_prefill_hidden");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
@@ -910,6 +932,7 @@ int gdn_prefill_hidden_varlen(const gdn_dims* dims, const gdn_weights* w, int32_
                               const uint16_t* w_in, const float* init_state, const float* init_conv, uint16_t* out,
                               float* final_state, float* final_conv, void* workspace, size_t workspace_bytes,
                               void* stream) {
+    NvtxRange nvtx_range("gdn_prefill_hidden_varlen");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
@@ -966,6 +989,7 @@ int gdn_prefill_out(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32
                     const uint16_t* qkv, const uint16_t* z, const uint16_t* a, const uint16_t* b,
                     const float* init_state, const float* init_conv, const uint16_t* w_out, uint16_t* out,
                     float* final_state, float* final_conv, void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("gdn_prefill_out");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
@@ -997,6 +1021,7 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
                 const uint16_t* z, const uint16_t* a, const uint16_t* b, const float* init_state,
                 const float* init_conv, uint16_t* out, float* final_state, float* final_conv, void* workspace,
                 size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("gdn_prefill");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
@@ -1016,6 +1041,7 @@ int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, co
                        const uint16_t* a, const uint16_t* b, const float* init_state, const float* init_conv,
                        uint16_t* out, float* final_state, float* final_conv, void* workspace, size_t workspace_bytes,
                        void* stream) {
+    NvtxRange nvtx_range("gdn_prefill_varlen");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
@@ -1037,24 +1063,26 @@ int gdn_prefill_varlen(const gdn_dims* dims, const gdn_weights* w, int32_t N, co
 
 int gdn_decode(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const uint16_t* qkv, const uint16_t* z,
                const uint16_t* a, const uint16_t* b, float* state, float* conv, uint16_t* out, void* stream) {
+    NvtxRange nvtx_range("gdn_decode");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
     if (rows < 0 || rows > 65535) return GDN_ERR_INVALID_ARG;
     if (rows == 0) return GDN_OK;
-    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, 1, stream);
+    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, 1, stream, rows);
 }
 
 int gdn_decode_multi(const gdn_dims* dims, const gdn_weights* w, int32_t rows, int32_t ntok, const uint16_t* qkv,
                      const uint16_t* z, const uint16_t* a, const uint16_t* b, float* state, float* conv, uint16_t* out,
                      void* stream) {
+    NvtxRange nvtx_range("gdn_decode_multi");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
     if (rows < 0 || rows > 65535 || ntok < 1) return GDN_ERR_INVALID_ARG;
     if (ntok > dec::kMaxTokens) return GDN_ERR_UNSUPPORTED;
     if (rows == 0) return GDN_OK;
-    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, ntok, stream);
+    return decode_impl(dims, w, rows, qkv, z, a, b, state, conv, out, nullptr, ntok, stream, rows);
 }
 
 
@@ -1062,6 +1090,7 @@ int gdn_decode_slots(const gdn_dims* dims, const gdn_weights* w, int32_t rows, c
                      const int32_t* slots_dev, int32_t pool_rows, const uint16_t* qkv, const uint16_t* z,
                      const uint16_t* a, const uint16_t* b, float* state_pool, float* conv_pool, uint16_t* out,
                      void* stream) {
+    NvtxRange nvtx_range("gdn_decode_slots");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
@@ -1069,7 +1098,7 @@ int gdn_decode_slots(const gdn_dims* dims, const gdn_weights* w, int32_t rows, c
     if (rows == 0) return GDN_OK;
     if ((st = check_slots(slots_host, rows, pool_rows)) != GDN_OK) return st;
     if (slots_dev == nullptr || (reinterpret_cast<uintptr_t>(slots_dev) & 3u)) return GDN_ERR_INVALID_ARG;
-    return decode_impl(dims, w, rows, qkv, z, a, b, state_pool, conv_pool, out, slots_dev, 1, stream);
+    return decode_impl(dims, w, rows, qkv, z, a, b, state_pool, conv_pool, out, slots_dev, 1, stream, pool_rows);
 }
 
 int gdn_prefill_varlen_slots(const gdn_dims* dims, const gdn_weights* w, int32_t N, const int32_t* cu_host,
@@ -1077,6 +1106,7 @@ int gdn_prefill_varlen_slots(const gdn_dims* dims, const gdn_weights* w, int32_t
                              const int32_t* slots_dev, int32_t pool_rows, const uint16_t* qkv, const uint16_t* z,
                              const uint16_t* a, const uint16_t* b, float* state_pool, float* conv_pool,
                              uint16_t* out, void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("gdn_prefill_varlen_slots");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;
@@ -1098,12 +1128,13 @@ int gdn_prefill_varlen_slots(const gdn_dims* dims, const gdn_weights* w, int32_t
     for (int32_t i = 0; i < N; ++i) nch += (cu_host[i + 1] - cu_host[i] + 63) / 64;
     return prefill_impl(dims, w, N, cu_dev, 0, total_T, nch, chunk_bound(N, total_T), qkv, z, a, b, state_pool,
                         conv_pool, out, state_pool, conv_pool, workspace, workspace_bytes,
-                        static_cast<cudaStream_t>(stream), false, slots_dev);
+                        static_cast<cudaStream_t>(stream), false, slots_dev, nullptr, nullptr, pool_rows);
 }
 
 int gdn_prefill_noalloc(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, const uint16_t* qkv,
                         const uint16_t* z, const uint16_t* a, const uint16_t* b, const float* init_state,
                         const float* init_conv, uint16_t* out, float* final_state, float* final_conv, void* stream) {
+    NvtxRange nvtx_range("gdn_prefill_noalloc");
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if ((st = check_weights(w)) != GDN_OK) return st;

@@ -48,6 +48,8 @@ struct ChunkParams {
     int c0, c1;               // chunk window [c0, c1) of every row (c1 < 0: to the end of the row)
     const int* slots;         // [N] state row of each packed row (validated by the host), or nullptr
     const int* order;         // [N] packed row of each grid row (longest first), or nullptr: grid row = row
+    int rec_chunks;           // chunks the record array holds  } the index checks of
+    int state_rows;           // rows of the state arrays       } the debug build
 };
 
 namespace chunk {
@@ -161,11 +163,16 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
 
     auto buf = [&](int c) { return smem + ((c & 1) ? OFF_BUF1 : OFF_BUF0); };
     auto dacc = [&](int c) { return tbase + ((c & 1) ? T_D1 : T_D0); };
-    auto rec_of = [&](int c) { return p.rec + ((size_t)(cbase + c) * p.Vh + h) * wy::REC_BYTES; };
+    // (debug build: a record index out of range is recorded and record 0 is read instead)
+    auto rec_of = [&](int c) {
+        const bool ok = GDN_CHECK(cbase + c >= 0 && cbase + c < p.rec_chunks);
+        return p.rec + (ok ? ((size_t)(cbase + c) * p.Vh + h) * wy::REC_BYTES : 0);
+    };
     auto load_chunk = [&](int c) {
         uint8_t* B = buf(c);
         uint64_t* bar = &bars[B_LD + (c & 1)];
         const int y = start + c * C;
+        (void)GDN_CHECK(y >= 0 && y < p.total);
         mbar_arrive_expect_tx(bar, LD_BYTES);
         tma_load_2d(B + BUF_V, &tmV, h * 128, y, bar);
         tma_load_2d(B + BUF_V + 8192, &tmV, h * 128 + 64, y, bar);
@@ -295,8 +302,9 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                 wait(B_LD, 0);
                 gC = reinterpret_cast<const float*>(buf(0) + BUF_DEC)[128];
             }
-            const float* src =
-                p.init_state ? p.init_state + (((size_t)srow * p.Vh + h) * 128 + row) * 128 + 64 * hf : nullptr;
+            const float* src = p.init_state && GDN_CHECK(srow >= 0 && srow < p.state_rows)
+                                   ? p.init_state + (((size_t)srow * p.Vh + h) * 128 + row) * 128 + 64 * hf
+                                   : nullptr;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];
@@ -382,7 +390,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
             }
         }
 
-        if (!broken && p.final_state != nullptr) {
+        if (!broken && p.final_state != nullptr && GDN_CHECK(srow >= 0 && srow < p.state_rows)) {
             float* dst = p.final_state + (((size_t)srow * p.Vh + h) * 128 + row) * 128 + 64 * hf;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -475,7 +483,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1)
                 const int nt = nv - 16 * qt;  // tokens of this quarter inside the row
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj)
-                    if (jj < nt)
+                    if (jj < nt && GDN_CHECK(tok0 + 16 * qt + jj < p.total))
                         op[(size_t)jj * p.Vh * 128] = static_cast<uint16_t>((jj & 1) ? (yb[jj >> 1] >> 16) : yb[jj >> 1]);
             }
             named_barrier_sync(3, kEThreads);

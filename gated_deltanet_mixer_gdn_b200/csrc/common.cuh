@@ -19,6 +19,7 @@ enum DeviceError : int {
     kErrNone = 0,
     kErrTimeoutTma = 1,
     kErrTimeoutMma = 2,
+    kErrIndex = 3,  // an index check of the GDN_DEBUG build failed
 };
 
 constexpr int kD = 128;        // head width (the only supported value)
@@ -381,5 +382,19 @@ __device__ __forceinline__ float warp_transpose_sum16(float (&v)[16], int lane) 
 }
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_error, 0, code); }
+
+// Index checks of the debug build (-DGDN_DEBUG): GDN_CHECK(cond) guards a global-memory
+// access whose address the kernel computed; a false condition records kErrIndex in the
+// error word and the caller skips the access (nothing traps).  In the release build the
+// condition is not evaluated and the guard is always true.
+__device__ __forceinline__ bool debug_check(bool ok) {
+    if (!ok) record_error(kErrIndex);
+    return ok;
+}
+#ifdef GDN_DEBUG
+#define GDN_CHECK(cond) (::gdn::debug_check(cond))
+#else
+#define GDN_CHECK(cond) (true)
+#endif
 
 }  // namespace gdn

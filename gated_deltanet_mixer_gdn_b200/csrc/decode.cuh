@@ -52,10 +52,15 @@ struct DecodeParams {
     float* conv;             // f32 [rows or pool][3][C], in place
     uint16_t* out;           // bf16 [rows][ntok][Vh*128]
     const int* slots;        // [rows] state / history row of each batch row (validated by the host), or nullptr
+    int pool_rows;           // rows of the state and history arrays (the index checks of the debug build)
 };
 
-// State and history row of batch row r.
-__device__ __forceinline__ int decode_slot(const DecodeParams& p, int r) { return p.slots ? __ldg(p.slots + r) : r; }
+// State and history row of batch row r (debug build: a row out of range is recorded and row
+// 0 is used instead).
+__device__ __forceinline__ int decode_slot(const DecodeParams& p, int r) {
+    const int s = p.slots ? __ldg(p.slots + r) : r;
+    return GDN_CHECK(r >= 0 && r < p.rows && s >= 0 && s < p.pool_rows) ? s : 0;
+}
 
 namespace dec {
 constexpr int kMaxStages = GDN_DECODE_STAGES;

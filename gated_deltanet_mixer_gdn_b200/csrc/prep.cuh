@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
             }
         }
     }
-    if (is_v && lane < nt) {  // gates of this value head: one token per lane
+    if (is_v && lane < nt && GDN_CHECK(t0 + lane < p.total && vh < p.Vh)) {  // gates: one token per lane
         const int t = t0 + lane;
         const float av = bf16_bits_to_float(p.a[(size_t)t * p.Vh + vh]);
         const float bv = bf16_bits_to_float(p.b[(size_t)t * p.Vh + vh]);
@@ -141,8 +141,9 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
     float w0[4], w1[4], w2[4];
     auto fetch_xbar = [&](int nn, int xi, int tok, float (&x)[4]) {
         if (xi >= 3) {
-            unpack4(__ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)tok * p.C + ch0)), x);
-        } else if (p.init_conv != nullptr) {
+            if (GDN_CHECK(tok >= 0 && tok < p.total && ch0 + 4 <= p.C))
+                unpack4(__ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)tok * p.C + ch0)), x);
+        } else if (p.init_conv != nullptr && GDN_CHECK(nn >= 0 && nn < p.seq.N && xi >= 0)) {
             const int sr = p.slots ? __ldg(p.slots + nn) : nn;
             const float4 h = __ldg(reinterpret_cast<const float4*>(p.init_conv + ((size_t)sr * 3 + xi) * p.C + ch0));
             x[0] = h.x; x[1] = h.y; x[2] = h.z; x[3] = h.w;
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
         for (int tt = 0; tt < kPrepTokens; ++tt) {
             if (!FAST && tt >= nt) break;
             const int t = t0 + tt;
+            if (!GDN_CHECK(t < p.total)) break;
             float xn[4];
             unpack4(ahead[tt % kPrepAhead], xn);
             if (FAST ? (tt + kPrepAhead < kPrepTokens) : (tt + kPrepAhead < nt))
@@ -238,7 +240,7 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
 
 
 struct ConvOutParams {
-    int C, N;
+    int C, N, total;
     SeqIndex seq;
     const uint16_t* qkv;     // bf16 [total][C]
     const float* init_conv;  // f32 [N or pool][3][C] or nullptr
@@ -255,12 +257,13 @@ __global__ void __launch_bounds__(256) gdn_conv_out_kernel(const ConvOutParams p
     if (ch >= p.C) return;
     int start, len;
     p.seq.bounds(n, start, len);
+    if (!GDN_CHECK(n < p.N && start >= 0 && len >= 0)) return;
     const size_t sr = p.slots ? (size_t)__ldg(p.slots + n) : (size_t)n;
 #pragma unroll
     for (int r = 0; r < 3; ++r) {
         const int e = len + r;
         float v;
-        if (e >= 3) v = bf16_bits_to_float(p.qkv[(size_t)(start + e - 3) * p.C + ch]);
+        if (e >= 3) v = GDN_CHECK(start + e - 3 < p.total) ? bf16_bits_to_float(p.qkv[(size_t)(start + e - 3) * p.C + ch]) : 0.f;
         else v = p.init_conv ? p.init_conv[(sr * 3 + e) * p.C + ch] : 0.f;
         p.final_conv[(sr * 3 + r) * p.C + ch] = v;
     }

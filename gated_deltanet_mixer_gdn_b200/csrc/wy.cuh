@@ -37,6 +37,7 @@ struct WyParams {
     const float* Gs;        // f32 [Vh][total] log-decay
     const float* Bs;        // f32 [Vh][total] write rate
     uint8_t* rec;           // records [nchunks][Vh] of wy::REC_BYTES
+    int rec_chunks;         // chunks the record array holds (the index checks of the debug build)
 };
 
 namespace wy {
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         if (hslot >= ratio) return;
         int start, len;
         p.seq.bounds(n, start, len);
-        if (wt < min(C, len - c * C)) {
+        if (wt < min(C, len - c * C) && GDN_CHECK(start + c * C + wt < p.total && kap * ratio + hslot < p.Vh)) {
             const size_t off = (size_t)(kap * ratio + hslot) * p.total + start + c * C + wt;
             gv = __ldg(p.Gs + off);
             bv = __ldg(p.Bs + off);
@@ -485,7 +486,9 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
         const int hslot = sub * kHeads + wg;
         const bool active = hslot < ratio;
         const int h = kap * ratio + hslot;
-        uint8_t* rec = p.rec + ((size_t)g * p.Vh + h) * REC_BYTES;
+        // (debug build: a record index out of range is recorded and the task writes record 0)
+        const bool rec_ok = !active || GDN_CHECK(g >= 0 && g < p.rec_chunks && h < p.Vh);
+        uint8_t* rec = p.rec + (rec_ok ? ((size_t)g * p.Vh + h) * REC_BYTES : 0);
 
         const float gv = gv_next, bv = bv_next;
         load_gates(task + gridDim.x, gv_next, bv_next);
