@@ -130,8 +130,8 @@ Workspace plan_workspace(const gdn_dims* d, int64_t total, int64_t N, int64_t nc
 constexpr int kMaxSegments = 8;
 struct SideStreams {
     bool ready = false;
-    cudaStream_t prod = nullptr, chain = nullptr;
-    cudaEvent_t fork = nullptr, prod_done = nullptr, chain_done = nullptr;
+    cudaStream_t prod = nullptr, chain = nullptr, tail = nullptr;  // priorities: chain > prod > tail
+    cudaEvent_t fork = nullptr, prod_done = nullptr, chain_done = nullptr, tail_done = nullptr;
     cudaEvent_t seg[kMaxSegments] = {};   // WY records of a segment written (prod -> chain)
     cudaEvent_t rec[kMaxSegments] = {};   // recurrence of a segment done (chain -> prod)
 };
@@ -144,10 +144,13 @@ int side_streams(int dev, SideStreams** out) {
     if (!st.ready) {
         int least = 0, greatest = 0;
         if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GDN_ERR_CUDA;
-        if (cudaStreamCreateWithPriority(&st.prod, cudaStreamNonBlocking, least) != cudaSuccess ||
-            cudaStreamCreateWithPriority(&st.chain, cudaStreamNonBlocking, greatest) != cudaSuccess)
+        // (numerically lower is higher priority; with a single level all three are equal)
+        const int middle = greatest < least ? greatest + 1 : greatest;
+        if (cudaStreamCreateWithPriority(&st.prod, cudaStreamNonBlocking, middle) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&st.chain, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&st.tail, cudaStreamNonBlocking, least) != cudaSuccess)
             return GDN_ERR_CUDA;
-        cudaEvent_t* evs[3] = {&st.fork, &st.prod_done, &st.chain_done};
+        cudaEvent_t* evs[4] = {&st.fork, &st.prod_done, &st.chain_done, &st.tail_done};
         for (cudaEvent_t* e : evs)
             if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GDN_ERR_CUDA;
         for (auto& e : st.seg)
@@ -570,20 +573,23 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                 return st;
             if (op != nullptr && cudaEventRecord(ss->rec[k], ss->chain) != cudaSuccess) return GDN_ERR_CUDA;
         }
-        // out_proj of each segment's tokens, behind every WY launch on the low-priority stream,
-        // as soon as that segment's recurrence has written them
+        // out_proj of each segment's tokens on the lowest-priority stream, as soon as that
+        // segment's recurrence has written them (it takes the SMs the WY records leave)
         for (int k = 0; op != nullptr && k < S; ++k) {
-            if (cudaStreamWaitEvent(ss->prod, ss->rec[k], 0) != cudaSuccess) return GDN_ERR_CUDA;
+            if (cudaStreamWaitEvent(ss->tail, ss->rec[k], 0) != cudaSuccess) return GDN_ERR_CUDA;
             const int64_t a0 = (int64_t)cs[k] * 64, a1 = k + 1 < S ? (int64_t)cs[k + 1] * 64 : uniform_T;
             for (int n = 0; n < N; ++n)
                 if ((st = out_proj_range(*op, out, Vh * 128, (int64_t)n * uniform_T + a0,
-                                         (int64_t)n * uniform_T + (a1 < uniform_T ? a1 : uniform_T), ss->prod)) != GDN_OK)
+                                         (int64_t)n * uniform_T + (a1 < uniform_T ? a1 : uniform_T), ss->tail)) != GDN_OK)
                     return st;
         }
         if (cudaEventRecord(ss->prod_done, ss->prod) != cudaSuccess ||
             cudaEventRecord(ss->chain_done, ss->chain) != cudaSuccess ||
             cudaStreamWaitEvent(stream, ss->prod_done, 0) != cudaSuccess ||
             cudaStreamWaitEvent(stream, ss->chain_done, 0) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        if (op != nullptr && (cudaEventRecord(ss->tail_done, ss->tail) != cudaSuccess ||
+                              cudaStreamWaitEvent(stream, ss->tail_done, 0) != cudaSuccess))
             return GDN_ERR_CUDA;
         return GDN_OK;
     }

@@ -93,8 +93,8 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
  * The prefill computes the recurrence in chunks of 64 tokens (WY form) on
  * tensor cores with f16 operands and f32 accumulation.
  * When the recurrence leaves most SMs idle (few rows of at least 16 chunks;
- * gdn_prefill_schedule reports the plan) the call forks onto two internal
- * streams of the device (created on first use) through events recorded on
+ * gdn_prefill_schedule reports the plan) the call forks onto internal streams
+ * of the device (created on first use) through events recorded on
  * `stream`, and joins back onto `stream` before returning: the work stays
  * ordered on `stream` and can be captured into a CUDA graph.  Concurrent
  * calls from several host threads share those internal streams and run one
@@ -115,9 +115,9 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
  * GDN_ERR_UNSUPPORTED).  Workspace: gdn_prefill_out_workspace_size(dims, B, T)
  * bytes (the prefill's workspace plus y).  When the prefill overlaps its
  * kernels (see gdn_prefill_schedule), the projection of each recurrence
- * segment's tokens starts on the internal low-priority stream as soon as that
- * segment's outputs are written, while the later segments' recurrence runs;
- * otherwise it runs after the recurrence on `stream`.  The result is the same,
+ * segment's tokens starts on an internal stream of the lowest priority as soon
+ * as that segment's outputs are written, while the later segments' recurrence
+ * runs; otherwise it runs after the recurrence on `stream`.  The result is the same,
  * bit for bit, as gdn_prefill followed by gdn_out_proj.
  */
 size_t gdn_prefill_out_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
