@@ -792,6 +792,8 @@ def main():
                     help="decode: the 64-row decode batch (default line); prefill: only the chunked prefill; "
                          "hidden: only the prefill from hidden states (fused in_proj + load stage)")
     ap.add_argument("--prefill-T", type=int, default=PREFILL_T, help="tokens of the prefill measurement")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="only the decode batch line (headline and e2e; a small case for profiling)")
     ap.add_argument("--no-long", action="store_true",
                     help="with --workload prefill: skip the 2 x 65,536-token leg")
     ap.add_argument("--prefill-only", action="store_true",
@@ -814,6 +816,10 @@ def main():
                 print(json.dumps(pre))
             return 0
         line, case = run_ours(args, world, rank, local)
+        if args.headline_only:
+            if rank == 0:
+                print(json.dumps(line))
+            return 0
         pre = bench_prefill(args, world, rank, local, args.prefill_T)
         multi = bench_decode_multi(args, local)
         proj = bench_projections(args, local)
