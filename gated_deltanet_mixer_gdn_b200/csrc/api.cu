@@ -14,6 +14,7 @@
 
 #include "../../include/gdn.h"
 #include "chunk.cuh"
+#include "chunk_pair.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "gemm.cuh"
@@ -227,7 +228,19 @@ int out_proj_range(const OutProjTail& op, const uint16_t* y, int VD, int64_t t0,
 // (Running the load stage per segment on the WY stream as well was measured no
 // faster at one row and slower at two.)
 namespace seg_model {
-constexpr double kWaveUs = 11.2, kWyFixedUs = 4.0, kChainFixedUs = 9.5, kChainChunkUs = 2.3;
+constexpr double kWaveUs = 11.2, kWyFixedUs = 4.0, kChainFixedUs = 9.5;
+constexpr double kChainChunkUs = 2.3, kPairChainChunkUs = 1.9;  // one CTA per head; CTA pairs
+}
+
+// The recurrence runs on CTA pairs (each 64 of a head's value channels, half the
+// per-chunk chain) unless that needs more than one wave of SMs.
+#ifndef GDN_PAIR_RULE
+#define GDN_PAIR_RULE 2
+#endif
+bool use_pair(int N, int Vh, int nsm) {
+    if (GDN_PAIR_RULE == 0) return false;
+    if (GDN_PAIR_RULE == 1) return true;
+    return 2 * (int64_t)N * Vh <= nsm;
 }
 
 struct SegPlan {
@@ -236,7 +249,7 @@ struct SegPlan {
 };
 
 // Time from the end of the load stage to the end of the last recurrence launch.
-double simulate_plan(const SegPlan& pl, int tasks_per_chunk, int nsm, int chain_ctas) {
+double simulate_plan(const SegPlan& pl, int tasks_per_chunk, int nsm, int chain_ctas, double chunk_us) {
     using namespace seg_model;
     const int P = pl.S > 1 ? nsm - chain_ctas : nsm;  // SMs of the WY stream beside a running recurrence
     auto wy_us = [&](int chunks, int sms) {
@@ -246,7 +259,7 @@ double simulate_plan(const SegPlan& pl, int tasks_per_chunk, int nsm, int chain_
     double wy_end = wy_us(pl.cs[1], nsm), chain_end = 0.0;
     for (int k = 0; k < pl.S; ++k) {
         const double start = chain_end > wy_end ? chain_end : wy_end;
-        chain_end = start + kChainFixedUs + kChainChunkUs * (pl.cs[k + 1] - pl.cs[k]);
+        chain_end = start + kChainFixedUs + chunk_us * (pl.cs[k + 1] - pl.cs[k]);
         if (k + 1 < pl.S) wy_end += wy_us(pl.cs[k + 2] - pl.cs[k + 1], P);
     }
     return chain_end;
@@ -254,14 +267,15 @@ double simulate_plan(const SegPlan& pl, int tasks_per_chunk, int nsm, int chain_
 
 // The plan for N dense rows of T tokens: overlap needs a recurrence that leaves at least
 // 32 SMs to the WY records and rows of at least 16 chunks.
-SegPlan dense_plan(int Kh, int Vh, int N, int T, int nsm) {
+SegPlan dense_plan(int Kh, int Vh, int N, int T, int nsm, bool pair) {
     const int per = (T + 63) / 64;
     SegPlan best;
     best.cs[1] = per;
-    if (N * Vh + 32 > nsm || per < 16) return best;
+    const int chain_ctas = (pair ? 2 : 1) * N * Vh;
+    const double chunk_us = pair ? seg_model::kPairChainChunkUs : seg_model::kChainChunkUs;
+    if (chain_ctas + 32 > nsm || per < 16) return best;
     const int tasks_per_chunk = N * Kh * ((Vh / Kh + wy::kHeads - 1) / wy::kHeads);
-    const int chain_ctas = N * Vh;
-    double best_t = simulate_plan(best, tasks_per_chunk, nsm, chain_ctas);
+    double best_t = simulate_plan(best, tasks_per_chunk, nsm, chain_ctas, chunk_us);
     static const double kRho[] = {0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8, 0.9, 1.0, 1.1, 1.2, 1.35, 1.5, 1.75, 2.0};
     const int max_S = per < kMaxSegments ? per : kMaxSegments;
     for (int S = 2; S <= max_S; ++S) {
@@ -279,7 +293,7 @@ SegPlan dense_plan(int Kh, int Vh, int N, int T, int nsm) {
                 c.cs[k] = v < lo ? lo : (v > hi ? hi : v);
             }
             c.cs[S] = per;
-            const double t = simulate_plan(c, tasks_per_chunk, nsm, chain_ctas);
+            const double t = simulate_plan(c, tasks_per_chunk, nsm, chain_ctas, chunk_us);
             if (t < best_t) {
                 best_t = t;
                 best = c;
@@ -313,6 +327,7 @@ struct PrefillPlan {
     uint8_t* rec;
     int rec_chunks;  // chunks the record array holds
     int state_rows;  // rows of the state / history arrays (the pool's, with slots)
+    bool pair;       // recurrence on CTA pairs (64 value channels each), else one CTA per head
     CUtensorMap mK, mQ, mKl, mQl, mV, mZ, mO;
 
     int prep(int tok_begin, int tok_end, cudaStream_t st) const {
@@ -446,6 +461,23 @@ struct PrefillPlan {
         cp.slots = slots;
         cp.rec_chunks = rec_chunks;
         cp.state_rows = state_rows;
+        if (pair) {
+            int rc = smem_optin(reinterpret_cast<const void*>(gdn_chunk_pair_kernel), pair::SMEM_BYTES);
+            if (rc != GDN_OK) return rc;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3(2 * Vh, N);
+            cfg.blockDim = dim3(pair::kThreads);
+            cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            return cuda_status(cudaLaunchKernelEx(&cfg, gdn_chunk_pair_kernel, mV, mQ, mK, mZ, mO, cp));
+        }
         int rc = smem_optin(reinterpret_cast<const void*>(gdn_chunk_kernel), chunk::SMEM_BYTES);
         if (rc != GDN_OK) return rc;
         dim3 grid(Vh, N);
@@ -523,6 +555,7 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     P.rec = wsb + ws.off_rec;
     P.rec_chunks = (int)nchunks_planned;
     P.state_rows = slots_dev != nullptr ? pool_rows : N;
+    P.pair = use_pair(N, Vh, nsm);
     if (!make_map(&P.mK, P.Ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&P.mKl, P.Kl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Kh * 128, total, 64, 64,
@@ -533,10 +566,10 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&P.mV, P.Vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)Vh * 128, total, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&P.mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&P.mO, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, 128, 64,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
+        !make_map(&P.mZ, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, P.pair ? 64 : 128, 64,
+                  P.pair ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&P.mO, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)Vh * 128, total, P.pair ? 64 : 128, 64,
+                  P.pair ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
         return GDN_ERR_CUDA;
 
     // Overlapped schedule (dense rows that leave most SMs idle during the recurrence):
@@ -545,10 +578,10 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
     // persistent grid that leaves the recurrence its SMs) while the recurrence of
     // segment s runs on the high-priority one, each segment's recurrence starting from
     // the state the previous one left in final_state.
-    const int chain_ctas = N * Vh;
+    const int chain_ctas = (P.pair ? 2 : 1) * N * Vh;
     SegPlan plan;
     if (may_overlap && cu_dev == nullptr && final_state != nullptr)
-        plan = dense_plan(Kh, Vh, N, uniform_T, nsm);
+        plan = dense_plan(Kh, Vh, N, uniform_T, nsm, P.pair);
     const int S = plan.S;
     const int* cs = plan.cs;
     if (S > 1) {
@@ -970,7 +1003,8 @@ int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t fro
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
     const bool fused = from_hidden != 0 && fused_load_ok(dims);
-    const SegPlan pl = dense_plan(dims->num_k_heads, dims->num_v_heads, B, T, nsm);
+    const SegPlan pl =
+        dense_plan(dims->num_k_heads, dims->num_v_heads, B, T, nsm, use_pair(B, dims->num_v_heads, nsm));
     *segments = pl.S;
     *launches = plan_launches(pl) + (from_hidden != 0 && !fused ? 1 : 0);  // + the unfused in_proj
     return GDN_OK;

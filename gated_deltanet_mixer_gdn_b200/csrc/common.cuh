@@ -174,6 +174,48 @@ __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank)
 
 __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Asynchronous store of v to the shared-memory location of `local` in CTA `rank` of this
+// thread's cluster; its 4 bytes count towards the transaction count of the mbarrier at the
+// location of `local_bar` in that CTA (which must expect them).
+__device__ __forceinline__ void st_async_remote_f32(const float* local, const uint64_t* local_bar, uint32_t rank,
+                                                    float v) {
+    uint32_t rdst, rbar;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rdst) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(smem_u32(local_bar)), "r"(rank));
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(rdst),
+                 "r"(__float_as_uint(v)), "r"(rbar)
+                 : "memory");
+}
+
+// mbarrier wait with acquire at cluster scope (for phases completed from another CTA),
+// false after the fixed bound.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    auto try_once = [&]() {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(a), "r"(parity)
+            : "memory");
+        return ok != 0;
+    };
+    if (try_once()) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!try_once()) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (tensor-core operand reads, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -298,6 +340,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
     d |= static_cast<uint64_t>(1) << 46;  // descriptor version of sm_100
     d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
     return d;
+}
+
+// The descriptor of shared-memory address `saddr` from the one of address 0 with the same
+// strides (`tmpl` = sw128_desc(0, lbo, sbo)): the address field is the low 14 bits.
+__device__ __forceinline__ uint64_t desc_at(uint64_t tmpl, uint32_t saddr) {
+    return tmpl + static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
 }
 
 // Instruction descriptor of kind::f16 with f16 A/B and an f32 accumulator.
