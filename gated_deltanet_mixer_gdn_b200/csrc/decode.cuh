@@ -107,6 +107,17 @@ __host__ __device__ inline Plan plan(int G, int n) {
 }
 }  // namespace dec
 
+// The row arithmetic, with every fused multiply-add written out, so that the one-token and
+// the several-token kernels round identically whatever the compiler would contract.
+__device__ __forceinline__ float dot4(const float4 a, const float4 b) {
+    return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, a.x * b.x)));
+}
+// alpha s + u k
+__device__ __forceinline__ float4 decay_add(const float4 s, float alpha, float u, const float4 k) {
+    return make_float4(fmaf(u, k.x, alpha * s.x), fmaf(u, k.y, alpha * s.y), fmaf(u, k.z, alpha * s.z),
+                       fmaf(u, k.w, alpha * s.w));
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -387,21 +398,18 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                         float vals[16];
 #pragma unroll
                         for (int r = 0; r < 8; ++r) {
-                            vals[2 * r] = s[r].x * kf.x + s[r].y * kf.y + s[r].z * kf.z + s[r].w * kf.w;
-                            vals[2 * r + 1] = s[r].x * qf.x + s[r].y * qf.y + s[r].z * qf.z + s[r].w * qf.w;
+                            vals[2 * r] = dot4(s[r], kf);
+                            vals[2 * r + 1] = dot4(s[r], qf);
                         }
                         // lane l: row l >> 2 of the warp's 8, S.k if bit 1 of l is clear, else S.q
                         const float tot = warp_transpose_sum16(vals, lane);
-                        const float u_k = beta * (s_v[(j * G + hh) * 128 + irow] - alpha * tot);  // lanes 4r, 4r+1
+                        const float u_k = beta * fmaf(-alpha, tot, s_v[(j * G + hh) * 128 + irow]);  // lanes 4r, 4r+1
                         const float u_r = __shfl_sync(0xffffffffu, u_k, lane & ~3);
-                        if ((lane & 3) == 2) s_o[(j * G + hh) * 128 + irow] = alpha * tot + u_r * s_kq[j];
+                        if ((lane & 3) == 2) s_o[(j * G + hh) * 128 + irow] = fmaf(u_r, s_kq[j], alpha * tot);
 #pragma unroll
                         for (int r = 0; r < 8; ++r) {
                             const float ur = __shfl_sync(0xffffffffu, u_k, 4 * r);
-                            s[r].x = alpha * s[r].x + ur * kf.x;
-                            s[r].y = alpha * s[r].y + ur * kf.y;
-                            s[r].z = alpha * s[r].z + ur * kf.z;
-                            s[r].w = alpha * s[r].w + ur * kf.w;
+                            s[r] = decay_add(s[r], alpha, ur, kf);
                         }
                     }
                 }

@@ -602,13 +602,6 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             __syncwarp();
         }
 
-        // ---- once every slot is done with this buffer, fill it with the task after next
-        if (tid == 0) {
-            wait1(B_FREE + buf, pb);
-            if (task + 2 * (int)gridDim.x < ntasks) issue_loads(task + 2 * gridDim.x, buf);
-        }
-        __syncwarp();
-
         // ---- -W to the record: TMEM lane k holds column k of W (64 tokens)
         if (active) {
             wait(B_W + wg, ph);
@@ -633,6 +626,14 @@ __global__ void __launch_bounds__(wy::kThreads, 1)
             }
             tc_fence_before();
         }
+
+        // ---- once every slot is done with this buffer, fill it with the task after next
+        // (after this warpgroup's own record, so its thread 0 does not wait for the others first)
+        if (tid == 0) {
+            wait1(B_FREE + buf, pb);
+            if (task + 2 * (int)gridDim.x < ntasks) issue_loads(task + 2 * gridDim.x, buf);
+        }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
