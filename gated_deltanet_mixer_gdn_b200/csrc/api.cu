@@ -772,13 +772,14 @@ int decode_impl(const gdn_dims* dims, const gdn_weights* w, int32_t rows, const 
     // 9.9 -> 6.5 us; with more than one wave the persistent grouping is faster.
     const int Gfull = p.Vh / p.Kh;
     const bool split = Gfull > 1 && rows * p.Kh * Gfull <= nsm;
-    const dec::Plan dplan = dec::plan(split ? 1 : Gfull, ntok);
+    const int kmax = ntok == 1 ? 1 : dec::kMaxTokens;  // the kernel instantiation
+    const dec::Plan dplan = dec::plan(split ? 1 : Gfull, ntok, dec::groups(kmax));
     if (dplan.stages < 2) return GDN_ERR_UNSUPPORTED;  // the group's inputs of ntok tokens leave no room
     p.nitems = rows * p.Kh * (split ? Gfull : 1);
     const int grid = split ? p.nitems : (p.nitems < nsm ? p.nitems : nsm);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(dec::kThreads);
+    cfg.blockDim = dim3(dec::threads(kmax));
     cfg.dynamicSmemBytes = dplan.smem_bytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];

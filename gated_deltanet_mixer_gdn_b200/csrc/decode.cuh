@@ -66,8 +66,11 @@ namespace dec {
 constexpr int kMaxStages = GDN_DECODE_STAGES;
 constexpr int kMaxGroup = 8;                     // value heads per q/k head (Vh / Kh)
 constexpr uint32_t kTileBytes = 64 * 128 * 4;   // half of a head's state
-constexpr int kComputeThreads = 256;
-constexpr int kThreads = kComputeThreads + 32;  // + producer warp
+constexpr int kComputeThreads = 256;            // one group of compute warps
+// Groups of compute warps: with several tokens per row, two groups take alternate items, so
+// that one group's conv, norms and output of an item overlap the other's state stream.
+__host__ __device__ constexpr int groups(int kmax) { return kmax > 1 ? 2 : 1; }
+__host__ __device__ constexpr int threads(int kmax) { return groups(kmax) * kComputeThreads + 32; }  // + producer
 constexpr int kSlots = (2 + kMaxGroup) * 128 / kComputeThreads;  // conv channels per thread (max)
 constexpr uint32_t kSmemLimit = 232448;         // opt-in shared memory per block on sm_100
 constexpr int kMaxTokens = 8;                   // tokens per row of the multi-token kernel
@@ -81,8 +84,9 @@ struct Plan {
     int stages;
     uint32_t aux_x, aux_w, aux_z, aux_bytes, aux_load_bytes, off_aux, off_misc, misc_bytes, smem_bytes;
     uint32_t m_q, m_k, m_v, m_o, m_red, m_gate;  // float offsets of the scratch arrays (from off_misc + 256)
+    uint32_t group_floats;                        // scratch of one group of compute warps
 };
-__host__ __device__ inline Plan plan(int G, int n) {
+__host__ __device__ inline Plan plan(int G, int n, int ngroups) {
     Plan pl{};
     const uint32_t nch = (2 + G) * 128;
     pl.aux_x = 3 * nch * 4;
@@ -96,7 +100,8 @@ __host__ __device__ inline Plan plan(int G, int n) {
     pl.m_o = pl.m_v + n * G * 128;
     pl.m_red = pl.m_o + n * G * 128;
     pl.m_gate = pl.m_red + n * (8 + 8 * G);
-    pl.misc_bytes = 256 + ((pl.m_gate + n * G * 2 + n) * 4 + 127) / 128 * 128;  // gates, then k.q [n]
+    pl.group_floats = (pl.m_gate + n * G * 2 + n + 31) / 32 * 32;  // gates, then k.q [n]
+    pl.misc_bytes = 256 + ngroups * pl.group_floats * 4;
     const uint32_t rest = 2 * pl.aux_bytes + pl.misc_bytes + 1024;
     int st = (int)((kSmemLimit - rest) / kTileBytes);
     pl.stages = st > kMaxStages ? kMaxStages : st;
@@ -111,6 +116,31 @@ __host__ __device__ inline Plan plan(int G, int n) {
 // the several-token kernels round identically whatever the compiler would contract.
 __device__ __forceinline__ float dot4(const float4 a, const float4 b) {
     return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, a.x * b.x)));
+}
+// sum of the products of 16 columns (4 chunks of 4), in a fixed order
+__device__ __forceinline__ float dot16(const float4 (&a)[4], const float4 (&b)[4]) {
+    float acc = a[0].x * b[0].x;
+    acc = fmaf(a[0].y, b[0].y, acc);
+    acc = fmaf(a[0].z, b[0].z, acc);
+    acc = fmaf(a[0].w, b[0].w, acc);
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+        acc = fmaf(a[i].x, b[i].x, acc);
+        acc = fmaf(a[i].y, b[i].y, acc);
+        acc = fmaf(a[i].z, b[i].z, acc);
+        acc = fmaf(a[i].w, b[i].w, acc);
+    }
+    return acc;
+}
+// Four values per lane, summed over each aligned group of 8 lanes: lane l ends with the sum of
+// value ((l >> 2) & 1) * 2 + ((l >> 1) & 1).
+__device__ __forceinline__ float group8_transpose_sum4(const float (&v)[4], int lane) {
+    const bool up4 = (lane & 4) != 0;
+    const float w0 = (up4 ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, up4 ? v[0] : v[2], 4);
+    const float w1 = (up4 ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, up4 ? v[1] : v[3], 4);
+    const bool up2 = (lane & 2) != 0;
+    const float x = (up2 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, up2 ? w0 : w1, 2);
+    return x + __shfl_xor_sync(0xffffffffu, x, 1);
 }
 // alpha s + u k
 __device__ __forceinline__ float4 decay_add(const float4 s, float alpha, float u, const float4 k) {
@@ -140,7 +170,7 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, boo
 // SPLIT = true: an item is one value head; the Vh / Kh items of a group are the CTAs of one
 // thread-block cluster (one item each), launched with that cluster size.
 template <int KMAX, bool SPLIT>
-__global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(dec::threads(KMAX), 1) gdn_decode_kernel(const DecodeParams p) {
     using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -148,7 +178,8 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
     const int G = SPLIT ? 1 : Gfull;       // value heads of one item
     const int ns = SPLIT ? Gfull : 1;      // items per q/k group
     const int nt = KMAX == 1 ? 1 : p.ntok;  // tokens per row
-    const Plan pl = plan(G, nt);
+    constexpr int NG = groups(KMAX);
+    const Plan pl = plan(G, nt, NG);
     const int nst = pl.stages;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.off_misc);
     uint64_t* empty = full + kMaxStages;
@@ -205,7 +236,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         return p.state + (((size_t)decode_slot(p, row) * p.Vh + head) * 128 + (r & 1) * 64) * 128;
     };
 
-    if (warp == kComputeThreads / 32) {
+    if (warp == NG * kComputeThreads / 32) {
         // ---------------- producer warp: per-item inputs one item ahead, state half-tiles in a ring
         if (lane == 0) {
             auto aux_load = [&](int m) {
@@ -274,31 +305,41 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         return;
     }
 
-    // ---------------- compute warps (tid < 256)
-    const float w_n = (tid < 128) ? 1.0f + p.norm_w[tid] : 0.f;
-    // gate inputs of the next item, loaded one item ahead (thread tid < G * nt: token tid / G, head tid % G)
+    // ---------------- compute warps: group cg of NG takes this CTA's items cg, cg + NG, ...
+    const int cg = warp / (kComputeThreads / 32);
+    const int ctid = tid - cg * kComputeThreads, cwarp = ctid >> 5;
+    const uint32_t gbar = 1 + cg;  // named barrier of the group
+    s_q += cg * pl.group_floats;
+    s_k += cg * pl.group_floats;
+    s_v += cg * pl.group_floats;
+    s_o += cg * pl.group_floats;
+    s_red += cg * pl.group_floats;
+    s_gate += cg * pl.group_floats;
+    s_kq += cg * pl.group_floats;
+    const float w_n = (ctid < 128) ? 1.0f + p.norm_w[ctid] : 0.f;
+    // gate inputs of the next item, loaded one item ahead (thread ctid < G * nt: token ctid / G, head ctid % G)
     float ga = 0.f, gb = 0.f, gA = 0.f, gdt = 0.f;
     auto gate_prefetch = [&](int m) {
         int row, kap, hoff;
         item(blockIdx.x + m * gridDim.x, row, kap, hoff);
-        const int head = kap * Gfull + hoff + tid % G, j = tid / G;
+        const int head = kap * Gfull + hoff + ctid % G, j = ctid / G;
         ga = bf16_bits_to_float(p.a[((size_t)row * nt + j) * p.Vh + head]);
         gb = bf16_bits_to_float(p.b[((size_t)row * nt + j) * p.Vh + head]);
         gA = p.A_log[head];
         gdt = p.dt_bias[head];
     };
-    if (tid < G * nt && nmine > 0) gate_prefetch(0);
-    int u = 0;
-    for (int m = 0; m < nmine; ++m) {
+    if (ctid < G * nt && cg < nmine) gate_prefetch(cg);
+    for (int m = cg; m < nmine; m += NG) {
+        int u = m * units_per_item;  // first state unit of the item
         int row, kap, hoff;
         item(blockIdx.x + m * gridDim.x, row, kap, hoff);
         const int srow = decode_slot(p, row);
         const uint8_t* ax = smem + pl.off_aux + (m & 1) * pl.aux_bytes;
-        named_barrier_sync(1, kComputeThreads);  // previous item's readers of the scratch are done
+        named_barrier_sync(gbar, kComputeThreads);  // previous item's readers of the scratch are done
         bounded_wait(&auxfull[m & 1], (m >> 1) & 1, broken);
         // split group: the q/k history is shifted by the group's first CTA once the others hold it
         const bool qk_writer = !SPLIT || hoff == 0;
-        if (SPLIT && hoff != 0 && tid == 0) mbar_arrive_remote(qkfree, 0);
+        if (SPLIT && hoff != 0 && ctid == 0) mbar_arrive_remote(qkfree, 0);
 
         // ---- conv + silu of the item's channels over the nt tokens; shift their history in place
         const float* ah = reinterpret_cast<const float*>(ax);
@@ -306,7 +347,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
         const uint2* aw = reinterpret_cast<const uint2*>(ax + pl.aux_w);
 #pragma unroll
         for (int s = 0; s < kSlots; ++s) {
-            const int idx = tid + s * kComputeThreads;
+            const int idx = ctid + s * kComputeThreads;
             if (idx < nch) {
                 const int grp = idx >> 7, c = idx & 127;
                 const int ch = (grp == 0) ? kap * 128 + c
@@ -341,39 +382,39 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                 }
             }
         }
-        if (tid < G * nt) {
-            s_gate[2 * tid] = expf(-expf(gA) * softplus_f(ga + gdt));  // alpha of (token tid / G, head tid % G)
-            s_gate[2 * tid + 1] = sigmoid_f(gb);                        // beta
-            if (m + 1 < nmine) gate_prefetch(m + 1);
+        if (ctid < G * nt) {
+            s_gate[2 * ctid] = expf(-expf(gA) * softplus_f(ga + gdt));  // alpha of (token ctid / G, head ctid % G)
+            s_gate[2 * ctid + 1] = sigmoid_f(gb);                        // beta
+            if (m + NG < nmine) gate_prefetch(m + NG);
         }
-        named_barrier_sync(1, kComputeThreads);
+        named_barrier_sync(gbar, kComputeThreads);
         // ---- L2 norms per token: q in warps 0-3, k in warps 4-7
 #pragma unroll 1
         for (int j = 0; j < nt; ++j) {
             {
-                const float x = (tid < 128) ? s_q[j * 128 + tid] : s_k[j * 128 + tid - 128];
+                const float x = (ctid < 128) ? s_q[j * 128 + ctid] : s_k[j * 128 + ctid - 128];
                 const float ss = warp_sum(x * x);
-                if (lane == 0) s_red[j * nred + warp] = ss;
+                if (lane == 0) s_red[j * nred + cwarp] = ss;
             }
         }
-        named_barrier_sync(1, kComputeThreads);
-        // q / (|q| sqrt(128)), k / |k| in place; then k.q per token (warp j)
+        named_barrier_sync(gbar, kComputeThreads);
+        // q / (|q| sqrt(128)), k / |k| in place; then k.q per token (warp j of the group)
 #pragma unroll 1
         for (int j = 0; j < nt; ++j) {
             {
                 const float* r8 = s_red + j * nred;
-                if (tid < 128) s_q[j * 128 + tid] *= rsqrtf(r8[0] + r8[1] + r8[2] + r8[3] + kEps) * rsqrtf(128.0f);
-                else s_k[j * 128 + tid - 128] *= rsqrtf(r8[4] + r8[5] + r8[6] + r8[7] + kEps);
+                if (ctid < 128) s_q[j * 128 + ctid] *= rsqrtf(r8[0] + r8[1] + r8[2] + r8[3] + kEps) * rsqrtf(128.0f);
+                else s_k[j * 128 + ctid - 128] *= rsqrtf(r8[4] + r8[5] + r8[6] + r8[7] + kEps);
             }
         }
-        named_barrier_sync(1, kComputeThreads);
-        if (warp < nt) {
-            const float4 qf = reinterpret_cast<const float4*>(s_q + warp * 128)[lane];
-            const float4 kf = reinterpret_cast<const float4*>(s_k + warp * 128)[lane];
+        named_barrier_sync(gbar, kComputeThreads);
+        if (cwarp < nt) {
+            const float4 qf = reinterpret_cast<const float4*>(s_q + cwarp * 128)[lane];
+            const float4 kf = reinterpret_cast<const float4*>(s_k + cwarp * 128)[lane];
             const float kq = warp_sum(kf.x * qf.x + kf.y * qf.y + kf.z * qf.z + kf.w * qf.w);
-            if (lane == 0) s_kq[warp] = kq;
+            if (lane == 0) s_kq[cwarp] = kq;
         }
-        named_barrier_sync(1, kComputeThreads);
+        named_barrier_sync(gbar, kComputeThreads);
 
         // ---- stream the G value heads' states, two half-tiles each; nt updates per row in registers
 #pragma unroll 1
@@ -382,57 +423,67 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
             for (int half = 0; half < 2; ++half, ++u) {
                 const int st = u % nst;
                 bounded_wait(&full[st], (u / nst) & 1, broken);
-                const float* tile = reinterpret_cast<const float*>(smem + st * kTileBytes);
-                float4 s[8];
+                // the warp's 8 rows: lanes 8 g .. 8 g + 7 hold rows 2 g and 2 g + 1, lane l the
+                // 16-byte column chunks (l & 7) + 8 i, i < 4 (eight lanes read 128 contiguous bytes)
+                const float4* tile = reinterpret_cast<const float4*>(smem + st * kTileBytes);
+                const int r0 = cwarp * 8 + 2 * (lane >> 3), sl = lane & 7;
+                float4 s[2][4];
 #pragma unroll
-                for (int r = 0; r < 8; ++r) s[r] = reinterpret_cast<const float4*>(tile + (warp * 8 + r) * 128)[lane];
+                for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) s[rr][i] = tile[(r0 + rr) * 32 + sl + 8 * i];
                 __syncwarp();
                 if (lane == 0 && !broken) mbar_arrive(&empty[st]);  // this warp is done reading the stage
-                const int irow = half * 64 + warp * 8 + (lane >> 2);
+                // after the reduction lane l holds row r0 + ((l >> 2) & 1), S.k if bit 1 of l is clear, else S.q
+                const int irow = half * 64 + r0 + ((lane >> 2) & 1);
 #pragma unroll 1
                 for (int j = 0; j < nt; ++j) {
                     {
                         const float alpha = s_gate[2 * (j * G + hh)], beta = s_gate[2 * (j * G + hh) + 1];
-                        const float4 qf = reinterpret_cast<const float4*>(s_q + j * 128)[lane];
-                        const float4 kf = reinterpret_cast<const float4*>(s_k + j * 128)[lane];
-                        float vals[16];
+                        const float4* q4 = reinterpret_cast<const float4*>(s_q + j * 128) + sl;
+                        const float4* k4 = reinterpret_cast<const float4*>(s_k + j * 128) + sl;
+                        float4 kf[4], qf[4];
 #pragma unroll
-                        for (int r = 0; r < 8; ++r) {
-                            vals[2 * r] = dot4(s[r], kf);
-                            vals[2 * r + 1] = dot4(s[r], qf);
+                        for (int i = 0; i < 4; ++i) {
+                            kf[i] = k4[8 * i];
+                            qf[i] = q4[8 * i];
                         }
-                        // lane l: row l >> 2 of the warp's 8, S.k if bit 1 of l is clear, else S.q
-                        const float tot = warp_transpose_sum16(vals, lane);
-                        const float u_k = beta * fmaf(-alpha, tot, s_v[(j * G + hh) * 128 + irow]);  // lanes 4r, 4r+1
-                        const float u_r = __shfl_sync(0xffffffffu, u_k, lane & ~3);
-                        if ((lane & 3) == 2) s_o[(j * G + hh) * 128 + irow] = fmaf(u_r, s_kq[j], alpha * tot);
+                        float v[4] = {dot16(s[0], kf), dot16(s[0], qf), dot16(s[1], kf), dot16(s[1], qf)};
+                        const float tot = group8_transpose_sum4(v, lane);
+                        const float u_k = beta * fmaf(-alpha, tot, s_v[(j * G + hh) * 128 + irow]);  // lanes with bit 1 clear
+                        const float u0 = __shfl_sync(0xffffffffu, u_k, lane & ~7);        // row r0
+                        const float u1 = __shfl_sync(0xffffffffu, u_k, (lane & ~7) | 4);  // row r0 + 1
+                        if ((lane & 3) == 2)
+                            s_o[(j * G + hh) * 128 + irow] = fmaf((lane & 4) ? u1 : u0, s_kq[j], alpha * tot);
 #pragma unroll
-                        for (int r = 0; r < 8; ++r) {
-                            const float ur = __shfl_sync(0xffffffffu, u_k, 4 * r);
-                            s[r] = decay_add(s[r], alpha, ur, kf);
+                        for (int i = 0; i < 4; ++i) {
+                            s[0][i] = decay_add(s[0][i], alpha, u0, kf[i]);
+                            s[1][i] = decay_add(s[1][i], alpha, u1, kf[i]);
                         }
                     }
                 }
-                float* gdst = unit_ptr(u) + (warp * 8) * 128;
+                float4* gdst = reinterpret_cast<float4*>(unit_ptr(u));
 #pragma unroll
-                for (int r = 0; r < 8; ++r) __stcs(reinterpret_cast<float4*>(gdst + r * 128) + lane, s[r]);
+                for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) __stcs(gdst + (r0 + rr) * 32 + sl + 8 * i, s[rr][i]);
             }
         }
 
         // ---- gated RMSNorm of the G heads' 128 outputs of every token
-        named_barrier_sync(1, kComputeThreads);
+        named_barrier_sync(gbar, kComputeThreads);
 #pragma unroll 1
         for (int j = 0; j < nt; ++j) {
             {
                 for (int hh = 0; hh < G; ++hh) {
-                    const float o = (tid < 128) ? s_o[(j * G + hh) * 128 + tid] : 0.f;
+                    const float o = (ctid < 128) ? s_o[(j * G + hh) * 128 + ctid] : 0.f;
                     const float ss = warp_sum(o * o);
-                    if (lane == 0) s_red[j * nred + 8 + hh * 8 + warp] = ss;
+                    if (lane == 0) s_red[j * nred + 8 + hh * 8 + cwarp] = ss;
                 }
             }
         }
-        named_barrier_sync(1, kComputeThreads);
-        if (tid < 128) {
+        named_barrier_sync(gbar, kComputeThreads);
+        if (ctid < 128) {
             const uint16_t* az = reinterpret_cast<const uint16_t*>(ax + pl.aux_z);
 #pragma unroll 1
             for (int j = 0; j < nt; ++j) {
@@ -441,9 +492,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) gdn_decode_kernel(const Deco
                         const float* r4 = s_red + j * nred + 8 + hh * 8;
                         const float ms = (r4[0] + r4[1] + r4[2] + r4[3]) * (1.0f / 128.0f);
                         const int head = kap * Gfull + hoff + hh;
-                        const float zv = bf16_bits_to_float(az[(j * G + hh) * 128 + tid]);
-                        const float y = s_o[(j * G + hh) * 128 + tid] * rsqrtf(ms + kEps) * w_n * silu_f(zv);
-                        p.out[(((size_t)row * nt + j) * p.Vh + head) * 128 + tid] = float_to_bf16_bits(y);
+                        const float zv = bf16_bits_to_float(az[(j * G + hh) * 128 + ctid]);
+                        const float y = s_o[(j * G + hh) * 128 + ctid] * rsqrtf(ms + kEps) * w_n * silu_f(zv);
+                        p.out[(((size_t)row * nt + j) * p.Vh + head) * 128 + ctid] = float_to_bf16_bits(y);
                     }
                 }
             }
