@@ -22,11 +22,14 @@
 // reader and writer, and the in-place history shift needs no cross-CTA sync.
 // Persistent CTAs (one per SM) walk items round-robin.  A producer warp
 // streams each state in 32 KiB half-tiles (64 state rows) with bulk copies
-// into a ring of shared-memory stages, running up to a full item ahead; eight
-// compute warps read a half-tile (8 rows per warp, one 128-bit load per lane
-// per row), reduce the 16 dot products of a warp with one transposed shuffle
-// reduction, and write the updated rows straight back to HBM with coalesced
-// 128-bit stores.
+// into a ring of shared-memory stages, running up to a full item ahead; a
+// group of eight compute warps reads a half-tile (8 rows per warp: each lane
+// holds 16 columns of 2 rows, eight lanes reading 128 contiguous bytes), sums
+// each row's two dot products over its eight lanes with one transposed
+// shuffle reduction, and writes the updated rows straight back to HBM with
+// coalesced 128-bit stores.  With several tokens per row two such groups take
+// alternate items, so that one group's conv, norms and output overlap the
+// other's state stream.
 #pragma once
 
 #include "common.cuh"
