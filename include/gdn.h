@@ -114,11 +114,12 @@ int gdn_prefill(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T
  * Arguments and results otherwise as gdn_prefill (hidden % 8 == 0, else
  * GDN_ERR_UNSUPPORTED).  Workspace: gdn_prefill_out_workspace_size(dims, B, T)
  * bytes (the prefill's workspace plus y).  When the prefill overlaps its
- * kernels (see gdn_prefill_schedule), the projection of each recurrence
- * segment's tokens starts on an internal stream of the lowest priority as soon
- * as that segment's outputs are written, while the later segments' recurrence
- * runs; otherwise it runs after the recurrence on `stream`.  The result is the same,
- * bit for bit, as gdn_prefill followed by gdn_out_proj.
+ * kernels (see gdn_prefill_schedule) and its recurrence occupies at most half
+ * the SMs, the projection of each recurrence segment's tokens starts on an
+ * internal stream of the lowest priority as soon as that segment's outputs are
+ * written, while the later segments' recurrence runs; otherwise it runs after
+ * the recurrence.  The result is the same, bit for bit, as gdn_prefill followed
+ * by gdn_out_proj.
  */
 size_t gdn_prefill_out_workspace_size(const gdn_dims* dims, int32_t B, int32_t T);
 int gdn_prefill_out(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32_t T, int32_t hidden,
