@@ -425,7 +425,11 @@ def bench_projections(args, local, T=8192):
         tf = flop / t / 1e12
         res[name] = {"workload": shape + " bf16, f32 accumulation", "ms": t * 1000.0, "tflops": tf,
                      "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                  "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"]},
+                                  "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"],
+                                  # the launches run back to back for several ms, under the power cap:
+                                  # against the seconds-long cuBLAS figure as well
+                                  "peak_sustained": peaks["bf16_tflops_sustained"],
+                                  "frac_sustained": tf / peaks["bf16_tflops_sustained"]},
                      "gpu_launches": n}
     return res
 
