@@ -588,7 +588,6 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
             cudaStreamWaitEvent(ss->chain, ss->fork, 0) != cudaSuccess)
             return GDN_ERR_CUDA;
         if ((st = P.prep(0, total, ss->prod)) != GDN_OK) return st;
-        if ((st = P.conv_out(ss->prod)) != GDN_OK) return st;  // after the load stage read the history
         for (int k = 0; k < S; ++k) {
             const int win = cs[k + 1] - cs[k];
             const int cap = k == 0 ? nsm : nsm - chain_ctas;  // leave the recurrence its SMs
@@ -616,6 +615,9 @@ int prefill_impl(const gdn_dims* d, const gdn_weights* w, int32_t N, const int32
                                          (int64_t)n * uniform_T + (a1 < uniform_T ? a1 : uniform_T), ss->tail)) != GDN_OK)
                     return st;
         }
+        // the final histories: after the load stage has read the old ones, off the path to the
+        // first recurrence segment (beside the last one)
+        if ((st = P.conv_out(ss->prod)) != GDN_OK) return st;
         if (cudaEventRecord(ss->prod_done, ss->prod) != cudaSuccess ||
             cudaEventRecord(ss->chain_done, ss->chain) != cudaSuccess ||
             cudaStreamWaitEvent(stream, ss->prod_done, 0) != cudaSuccess ||
