@@ -351,8 +351,12 @@ struct PrefillPlan {
         pp.Vs = Vs;
         pp.Gs = Gs;
         pp.Bs = Bs;
+        CUtensorMap mX;  // the CTAs' input rows x 256-channel boxes (rows outside the tensor read as zero)
+        if (!make_map(&mX, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)C, (uint64_t)total, kPrepBox, kPrepRows,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return GDN_ERR_CUDA;
         dim3 grid((tok_end - tok_begin + kPrepTokens - 1) / kPrepTokens, (2 * Kh + Vh + kPrepSlots - 1) / kPrepSlots);
-        gdn_prep_kernel<<<grid, 256, 0, st>>>(pp);
+        gdn_prep_kernel<<<grid, 256, kPrepSmem, st>>>(mX, pp);
         return cuda_status(cudaGetLastError());
     }
     // in_proj + load stage over all tokens: 128-row tiles advancing by 125 tokens

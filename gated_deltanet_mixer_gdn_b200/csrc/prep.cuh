@@ -77,8 +77,14 @@ struct Flag {
 };
 
 constexpr int kPrepTokens = 16;  // consecutive tokens per thread
-constexpr int kPrepAhead = 4;    // rows loaded ahead of the token being computed
 constexpr int kPrepSlots = 8;    // head slots (warps) per CTA
+// The CTA's input rows (3 before its first token, for the conv window, then its tokens) x its
+// 1024 channels, staged in shared memory by TMA at the start: 4 boxes of 256 channels.
+constexpr int kPrepRows = kPrepTokens + 3;
+constexpr int kPrepBox = 256;
+constexpr uint32_t kPrepBlockBytes = kPrepRows * kPrepBox * 2;               // 9,728
+constexpr uint32_t kPrepTileBytes = (kPrepSlots * kD / kPrepBox) * kPrepBlockBytes;  // 38,912
+constexpr uint32_t kPrepSmem = kPrepTileBytes + 16 + 128;                   // + barrier, alignment
 
 __device__ __forceinline__ void unpack4(const uint2 v, float (&x)[4]) {
     x[0] = __uint_as_float(v.x << 16);
@@ -88,29 +94,41 @@ __device__ __forceinline__ void unpack4(const uint2 v, float (&x)[4]) {
 }
 
 // A CTA covers 8 head slots (one warp each, 4 channels per lane) for
-// kPrepTokens consecutive tokens.  Each thread keeps its taps unpacked and the
-// last three inputs of its channels in registers (a rolling window that
-// restarts from the row's history at every row start), and loads the next
-// inputs kPrepAhead tokens ahead: per token one 8-byte load and a short
+// kPrepTokens consecutive tokens.  Its input rows arrive in shared memory by TMA
+// all at once (about 38 KB in flight per CTA, rows outside the tensor read as
+// zero); each thread keeps its taps unpacked and the last three inputs of its
+// channels in registers (a rolling window that restarts from the row's history
+// at every row start): per token one 8-byte shared-memory read and a short
 // instruction chain per thread, with many warps resident per SM.
-__global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
+__global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const __grid_constant__ CUtensorMap tmX, const PrepParams p) {
     const int lane = threadIdx.x & 31;
     const int nheads = 2 * p.Kh + p.Vh;
-    const int slot = blockIdx.y * kPrepSlots + (threadIdx.x >> 5);
+    const int wslot = threadIdx.x >> 5;
+    const int slot = blockIdx.y * kPrepSlots + wslot;
+    const int t0 = p.tok_begin + blockIdx.x * kPrepTokens;
+    const int nt = min(kPrepTokens, p.tok_end - t0);
+    if (nt <= 0) return;  // whole CTA
+
+    extern __shared__ uint8_t prep_smem_raw[];
+    uint8_t* tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(prep_smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(tile + kPrepTileBytes);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(bar, kPrepTileBytes);
+#pragma unroll
+        for (int i = 0; i < (int)(kPrepSlots * kD / kPrepBox); ++i)
+            tma_load_2d(tile + i * kPrepBlockBytes, &tmX, blockIdx.y * kPrepSlots * kD + i * kPrepBox, t0 - 3, bar);
+    }
+    __syncthreads();  // the barrier is initialised before anyone waits on it
     if (slot >= nheads) return;  // whole warp
     const int ch0 = slot * kD + lane * 4;
     const bool is_q = slot < p.Kh;
     const bool is_v = slot >= 2 * p.Kh;
     const int vh = slot - 2 * p.Kh;
-    const int t0 = p.tok_begin + blockIdx.x * kPrepTokens;
-    const int nt = min(kPrepTokens, p.tok_end - t0);
-    if (nt <= 0) return;  // whole CTA
-
-    uint2 ahead[kPrepAhead];
-#pragma unroll
-    for (int i = 0; i < kPrepAhead; ++i)
-        ahead[i] = (i < nt) ? __ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)(t0 + i) * p.C + ch0))
-                            : make_uint2(0u, 0u);
+    // this lane's 4 channels in input row r of the tile (r = token - t0 + 3)
+    const uint8_t* xcol = tile + (wslot >> 1) * kPrepBlockBytes + ((wslot & 1) * kD + lane * 4) * 2;
+    auto xrow = [&](int r) { return *reinterpret_cast<const uint2*>(xcol + r * kPrepBox * 2); };
     float w[4][4];  // w[j][e]: tap j of channel ch0 + e
     {
         const uint4* wp = reinterpret_cast<const uint4*>(p.conv_w + (size_t)ch0 * 4);
@@ -135,14 +153,17 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
         p.Bs[(size_t)vh * p.total + t] = sigmoid_f(bv);
     }
 
+    if (!mbar_wait(bar, 0)) {  // the tile never landed: recorded, nothing written
+        record_error(kErrTimeoutTma);
+        return;
+    }
     int n, start, len;
     p.seq.locate(t0, n, start, len);
     // window: w0 = index s, w1 = s + 1, w2 = s + 2 of [history (3 rows); tokens of the row]
     float w0[4], w1[4], w2[4];
     auto fetch_xbar = [&](int nn, int xi, int tok, float (&x)[4]) {
-        if (xi >= 3) {
-            if (GDN_CHECK(tok >= 0 && tok < p.total && ch0 + 4 <= p.C))
-                unpack4(__ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)tok * p.C + ch0)), x);
+        if (xi >= 3) {  // a token of the row: one of the tile's three rows before t0
+            if (GDN_CHECK(tok >= t0 - 3 && tok < t0 && tok >= 0 && ch0 + 4 <= p.C)) unpack4(xrow(tok - t0 + 3), x);
         } else if (p.init_conv != nullptr && GDN_CHECK(nn >= 0 && nn < p.seq.N && xi >= 0)) {
             const int sr = p.slots ? __ldg(p.slots + nn) : nn;
             const float4 h = __ldg(reinterpret_cast<const float4*>(p.init_conv + ((size_t)sr * 3 + xi) * p.C + ch0));
@@ -171,10 +192,7 @@ __global__ void __launch_bounds__(256, 4) gdn_prep_kernel(const PrepParams p) {
             const int t = t0 + tt;
             if (!GDN_CHECK(t < p.total)) break;
             float xn[4];
-            unpack4(ahead[tt % kPrepAhead], xn);
-            if (FAST ? (tt + kPrepAhead < kPrepTokens) : (tt + kPrepAhead < nt))
-                ahead[tt % kPrepAhead] =
-                    __ldg(reinterpret_cast<const uint2*>(p.qkv + (size_t)(t + kPrepAhead) * p.C + ch0));
+            unpack4(xrow(tt + 3), xn);
             if (!FAST && t == start + len) {  // a new row starts here (skip empty rows): restart from its history
                 if (p.seq.cu == nullptr) {
                     ++n;
