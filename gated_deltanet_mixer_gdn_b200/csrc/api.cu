@@ -355,6 +355,8 @@ struct PrefillPlan {
         if (!make_map(&mX, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)C, (uint64_t)total, kPrepBox, kPrepRows,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
             return GDN_ERR_CUDA;
+        int rc = smem_optin(reinterpret_cast<const void*>(gdn_prep_kernel), kPrepSmem);
+        if (rc != GDN_OK) return rc;
         dim3 grid((tok_end - tok_begin + kPrepTokens - 1) / kPrepTokens, (2 * Kh + Vh + kPrepSlots - 1) / kPrepSlots);
         gdn_prep_kernel<<<grid, 256, kPrepSmem, st>>>(mX, pp);
         return cuda_status(cudaGetLastError());
