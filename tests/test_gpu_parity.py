@@ -124,9 +124,12 @@ def test_prefill_small_config():
     _check_prefill(case, res, oracle_prefill(case), "prefill B=1 T=256 (all heads)")
 
 
+# one row: the recurrence on CTA pairs (each 64 of a head's value channels); two rows: one CTA
+# per (row, value head)
+@pytest.mark.parametrize("B", [1, 2])
 @pytest.mark.parametrize("T", [1, 2, 3, 63, 64, 65, 127, 200])
-def test_prefill_ragged_lengths_with_state(T):
-    case = synth.dense_case(500 + T, B=2, T=T, init=True)
+def test_prefill_ragged_lengths_with_state(T, B):
+    case = synth.dense_case(500 + T + (1000 if B == 1 else 0), B=B, T=T, init=True)
     w, acts, st, cv = to_dev(case)
     res = gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w, st, cv)
     torch.cuda.synchronize()
@@ -142,8 +145,9 @@ def test_prefill_long_memory_family():
     _check_prefill(case, res, oracle_prefill(case), "prefill long-memory T=600")
 
 
-def test_prefill_in_place_state():
-    case = synth.dense_case(78, B=2, T=130, init=True)
+@pytest.mark.parametrize("B", [1, 2])
+def test_prefill_in_place_state(B):
+    case = synth.dense_case(78 if B == 2 else 178, B=B, T=130, init=True)
     ref = oracle_prefill(case)
     w, acts, st, cv = to_dev(case)
     out, fs, fc = gdn.prefill(acts["qkv"], acts["z"], acts["a"], acts["b"], w, st, cv, in_place=True)
