@@ -278,13 +278,20 @@ __global__ void __launch_bounds__(pair::kThreads, 1)
         if (lane == 0 && nchunks > 0) {
             load_chunk(0);
             if (nchunks > 1) load_chunk(1);
+            int issued = nchunks > 1 ? 2 : 1;  // chunks whose inputs were requested
             for (int c = 2; c < nchunks && c < 4; ++c) prefetch_chunk(c);
             // a buffer takes chunk c+2 once every MMA that reads chunk c is done
             for (int c = 0; c + 2 < nchunks; ++c) {
                 wait1(B_FREE + (c & 1), (c >> 1) & 1);
+                if (broken) break;  // no copy into a buffer that may still be read
                 load_chunk(c + 2);
+                issued = c + 3;
                 if (c + 4 < nchunks) prefetch_chunk(c + 4);
             }
+            // after a wait ran out, the CTA exits only once its copies in flight have landed
+            // (the last request of each buffer; bounded)
+            if (broken)
+                for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c) mbar_wait(&bars[B_LD + (c & 1)], (c >> 1) & 1);
         }
         __syncwarp();
     } else if (warp < kConvWarps) {
@@ -452,7 +459,12 @@ __global__ void __launch_bounds__(pair::kThreads, 1)
             }
             __syncwarp();
         }
-        if (io) bulk_wait_all();
+        if (io) {
+            bulk_wait_all();
+            // after a wait ran out, the z tiles in flight land before the CTA exits (bounded)
+            if (broken)
+                for (int k = nchunks > 2 ? nchunks - 2 : 0; k < nchunks; ++k) mbar_wait(&bars[B_Z + (k & 1)], (k >> 1) & 1);
+        }
     } else {
         // =================================================================== preparers
         // Qs = diag(e^G) Q and K' = diag(e^{G_C - G}) K, in place; one row of 64 k per thread
