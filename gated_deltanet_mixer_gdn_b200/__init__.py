@@ -27,7 +27,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("GDN_B200_LIBRARY") or os.path.join(_PKG, "libgdn_b200.so")
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_out_workspace_size", "gdn_prefill_out",
-           "gdn_prefill_schedule", "gdn_prefill_varlen_workspace_size",
+           "gdn_prefill_schedule", "gdn_prefill_schedule_nsm", "gdn_prefill_varlen_workspace_size",
            "gdn_prefill_varlen", "gdn_decode", "gdn_decode_multi", "gdn_decode_slots", "gdn_prefill_varlen_slots",
            "gdn_in_proj", "gdn_out_proj", "gdn_prefill_hidden_workspace_size", "gdn_prefill_hidden",
            "gdn_prefill_hidden_varlen_workspace_size", "gdn_prefill_hidden_varlen",
@@ -78,6 +78,8 @@ def load_library() -> ctypes.CDLL:
         L.gdn_prefill_out.argtypes = [dp, wp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_prefill_schedule.restype = ctypes.c_int
         L.gdn_prefill_schedule.argtypes = [dp, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+        L.gdn_prefill_schedule_nsm.restype = ctypes.c_int
+        L.gdn_prefill_schedule_nsm.argtypes = [dp, i32, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
         L.gdn_prefill.argtypes = [dp, wp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_prefill_varlen.restype = ctypes.c_int
         L.gdn_prefill_varlen.argtypes = [dp, wp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -239,15 +241,20 @@ def prefill_out(qkv, z, a, b, weights, w_out, init_state=None, init_conv=None, *
     return out, final_state, final_conv
 
 
-def prefill_schedule(B: int, T: int, from_hidden: bool = False, dims: Dims = MODEL):
+def prefill_schedule(B: int, T: int, from_hidden: bool = False, dims: Dims = MODEL, nsm: int | None = None):
     """(segments, launches) of a dense prefill of B x T tokens that returns its final state, on
-    the current device: recurrence segments of the overlapped schedule (1: plain) and the number
-    of kernels the call launches (prefill, or prefill_hidden with from_hidden)."""
+    the current device (or, with nsm, on a device of nsm SMs, without one): recurrence segments
+    of the overlapped schedule (1: plain) and the number of kernels the call launches (prefill,
+    or prefill_hidden with from_hidden)."""
     L = load_library()
     dc = _dims_c(dims)
     seg, lau = ctypes.c_int32(0), ctypes.c_int32(0)
-    _check(L.gdn_prefill_schedule(ctypes.byref(dc), int(B), int(T), int(bool(from_hidden)), ctypes.byref(seg),
-                                  ctypes.byref(lau)), "gdn_prefill_schedule")
+    if nsm is None:
+        _check(L.gdn_prefill_schedule(ctypes.byref(dc), int(B), int(T), int(bool(from_hidden)), ctypes.byref(seg),
+                                      ctypes.byref(lau)), "gdn_prefill_schedule")
+    else:
+        _check(L.gdn_prefill_schedule_nsm(ctypes.byref(dc), int(B), int(T), int(bool(from_hidden)), int(nsm),
+                                          ctypes.byref(seg), ctypes.byref(lau)), "gdn_prefill_schedule_nsm")
     return seg.value, lau.value
 
 

@@ -997,25 +997,46 @@ int gdn_prefill_hidden_varlen(const gdn_dims* dims, const gdn_weights* w, int32_
                                stream);
 }
 
-int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t* segments,
-                         int32_t* launches) {
+// The schedule of a dense prefill on a device with nsm SMs (arguments already checked).
+void schedule_for(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int nsm, int32_t* segments,
+                  int32_t* launches) {
+    const bool fused = from_hidden != 0 && fused_load_ok(dims);
+    const SegPlan pl =
+        dense_plan(dims->num_k_heads, dims->num_v_heads, B, T, nsm, use_pair(B, dims->num_v_heads, nsm));
+    *segments = pl.S;
+    *launches = plan_launches(pl) + (from_hidden != 0 && !fused ? 1 : 0);  // + the unfused in_proj
+}
+
+int schedule_args(const gdn_dims* dims, int32_t B, int32_t T, int32_t* segments, int32_t* launches) {
     int st = check_dims(dims);
     if (st != GDN_OK) return st;
     if (B < 0 || T < 0 || B > 65535 || (int64_t)B * T > INT32_MAX || !segments || !launches)
         return GDN_ERR_INVALID_ARG;
     *segments = 0;
     *launches = 0;
-    if (B == 0 || T == 0) return GDN_OK;
+    return GDN_OK;
+}
+
+int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t* segments,
+                         int32_t* launches) {
+    int st = schedule_args(dims, B, T, segments, launches);
+    if (st != GDN_OK || B == 0 || T == 0) return st;
     if ((st = check_device()) != GDN_OK) return st;
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDN_ERR_CUDA;
-    const bool fused = from_hidden != 0 && fused_load_ok(dims);
-    const SegPlan pl =
-        dense_plan(dims->num_k_heads, dims->num_v_heads, B, T, nsm, use_pair(B, dims->num_v_heads, nsm));
-    *segments = pl.S;
-    *launches = plan_launches(pl) + (from_hidden != 0 && !fused ? 1 : 0);  // + the unfused in_proj
+    schedule_for(dims, B, T, from_hidden, nsm, segments, launches);
+    return GDN_OK;
+}
+
+int gdn_prefill_schedule_nsm(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t nsm,
+                             int32_t* segments, int32_t* launches) {
+    int st = schedule_args(dims, B, T, segments, launches);
+    if (st != GDN_OK) return st;
+    if (nsm < 1) return GDN_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return GDN_OK;
+    schedule_for(dims, B, T, from_hidden, nsm, segments, launches);
     return GDN_OK;
 }
 

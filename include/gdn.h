@@ -144,6 +144,16 @@ int gdn_prefill_out(const gdn_dims* dims, const gdn_weights* w, int32_t B, int32
 int gdn_prefill_schedule(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t* segments,
                          int32_t* launches);
 
+/*
+ * The same plan for a device with nsm streaming multiprocessors (nsm >= 1,
+ * else GDN_ERR_INVALID_ARG), without querying or needing a device: the
+ * recurrence runs on CTA pairs when 2 * B * num_v_heads <= nsm, and overlaps
+ * only when its CTAs + 32 <= nsm and rows hold at least 16 chunks of 64
+ * tokens.  Host-only.
+ */
+int gdn_prefill_schedule_nsm(const gdn_dims* dims, int32_t B, int32_t T, int32_t from_hidden, int32_t nsm,
+                             int32_t* segments, int32_t* launches);
+
 /* Bytes of device workspace gdn_prefill_varlen needs for N rows with
  * total_T tokens in all.  Returns 0 for invalid dims. */
 size_t gdn_prefill_varlen_workspace_size(const gdn_dims* dims, int32_t N, int32_t total_T);

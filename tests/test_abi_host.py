@@ -148,3 +148,33 @@ def test_binding_refuses_cpu_tensors():
     case = synth.dense_case(1, 1, 4)
     with pytest.raises(gdn.GdnError):
         gdn.prefill(case["qkv"], case["z"], case["a"], case["b"], case["weights"])
+
+
+def test_schedule_for_a_given_sm_count(lib):
+    """The segment planner of the dense prefill, on the host for a given SM count: the recurrence
+    runs on CTA pairs when 2 rows x heads fit the SMs, overlaps only when its CTAs leave 32 SMs and
+    rows hold 16 chunks, and one call launches 2 + 2 x segments kernels."""
+    def plan(B, T, nsm, from_hidden=False):
+        return gdn.prefill_schedule(B, T, from_hidden, nsm=nsm)
+
+    # B200 (148 SMs): one row on pairs (96 CTAs) overlaps in 3 segments; two rows on one CTA per
+    # head (96 CTAs) in 5; three rows (144 CTAs) leave too few SMs; short rows stay plain
+    assert plan(1, 8192, 148) == (3, 8)
+    assert plan(2, 65536, 148) == (5, 12)
+    assert plan(3, 8192, 148) == (1, 4)
+    assert plan(1, 15 * 64, 148) == (1, 4)
+    # 100 SMs: one row still fits as pairs (96) but then leaves only 4 SMs: plain; 95 SMs: one CTA
+    # per head (48) and overlap
+    assert plan(1, 8192, 100) == (1, 4)
+    assert plan(1, 8192, 95) == (4, 10)
+    # the fused in_proj path launches the same number (its GEMM replaces the load stage)
+    assert plan(1, 8192, 148, from_hidden=True) == (3, 8)
+    for B, T in ((1, 1), (1, 64), (2, 4096), (4, 8192), (1, 65536)):
+        s, n = plan(B, T, 148)
+        assert 1 <= s <= 8 and n == 2 + 2 * s
+    assert plan(0, 8192, 148) == (0, 0) and plan(1, 0, 148) == (0, 0)
+    d = _dims()
+    seg, lau = ctypes.c_int32(-7), ctypes.c_int32(-7)
+    assert lib.gdn_prefill_schedule_nsm(ctypes.byref(d), 1, 8192, 0, 0, ctypes.byref(seg), ctypes.byref(lau)) == -1
+    assert lib.gdn_prefill_schedule_nsm(ctypes.byref(d), -1, 8192, 0, 148, ctypes.byref(seg), ctypes.byref(lau)) == -1
+    assert lib.gdn_prefill_schedule_nsm(ctypes.byref(d), 1, 8192, 0, 148, None, None) == -1
