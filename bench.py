@@ -792,9 +792,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "hidden"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "hidden", "multi"],
                     help="decode: the 64-row decode batch (default line); prefill: only the chunked prefill; "
-                         "hidden: only the prefill from hidden states (fused in_proj + load stage)")
+                         "hidden: only the prefill from hidden states (fused in_proj + load stage); "
+                         "multi: only the multi-token decode (4 tokens per call; a small case for profiling)")
     ap.add_argument("--prefill-T", type=int, default=PREFILL_T, help="tokens of the prefill measurement")
     ap.add_argument("--headline-only", action="store_true",
                     help="only the decode batch line (headline and e2e; a small case for profiling)")
@@ -809,6 +810,11 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.workload == "multi":
+            multi = bench_decode_multi(args, local)
+            if rank == 0:
+                print(json.dumps({"metric": "GDN multi-token decode row-tokens/s", **multi}))
+            return 0
         if args.workload == "hidden":
             hid = bench_hidden(args, local)
             if rank == 0:
